@@ -1,0 +1,259 @@
+/*
+ * CPU oracle for the ball-tree build, the 45-degree rotation and ball attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+ * bench's CPU-baseline leg load this file.  It shares no code with the CUDA
+ * library (no headers, helpers or tables) and is deliberately plain and slow:
+ * every tree node is sorted afresh with qsort, attention is a triple loop in
+ * double precision.  Build: gcc -O2 -ffp-contract=off -fPIC -shared.
+ *
+ * What it follows (page titles as the sources give them):
+ *  - "Erwin: A Tree-based Hierarchical Transformer for Large-scale Physical
+ *    Systems" (bluesky thread, posts 6/N and 9/N; PMLR abstract): a ball tree
+ *    recursively splits the points into nested sets of similar size, each
+ *    covered by a ball; at every level the points of one ball are stored next
+ *    to each other.  The split rule used here (median of the axis of largest
+ *    extent, ties by original index, leaves in index order) is the reading
+ *    stated in the accompanying design notes; the pages do not print it.
+ *  - same thread, post 7/N: ball tree attention is scaled dot-product
+ *    attention computed independently inside every ball of one tree level.
+ *  - thread post "instead of shifting windows, we rotate trees": the rotated
+ *    layer rebuilds the tree on rotated coordinates (45 degrees about +z here).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_ARG 1
+#define ORC_ERR_SHAPE 2
+#define ORC_ERR_NONFINITE 3
+
+/* IEEE order-preserving map float -> uint32 (after -0 is folded into +0). */
+static uint32_t ord_key(float f)
+{
+    uint32_t u;
+    if (f == 0.0f) f = 0.0f;
+    memcpy(&u, &f, 4);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+static int cmp_u64(const void *a, const void *b)
+{
+    uint64_t x = *(const uint64_t *)a, y = *(const uint64_t *)b;
+    return (x > y) - (x < y);
+}
+
+static int cmp_u32(const void *a, const void *b)
+{
+    uint32_t x = *(const uint32_t *)a, y = *(const uint32_t *)b;
+    return (x > y) - (x < y);
+}
+
+/*
+ * One node of the tree.  ids[0..s) are local point ids of one cloud; ids >= n
+ * are dummy points that pad the cloud to m * 2^L slots.
+ *   s == m : a leaf, its points in ascending id order.
+ *   else   : extents over the real points (float max - min), the widest axis
+ *            (lowest axis on equal extents), sort by (coordinate key, id) with
+ *            dummies keyed above every real point, lower half left.
+ */
+static void build_node(const float *c, int64_t n, int32_t m, uint32_t *ids, int64_t s, uint64_t *tmp)
+{
+    if (s == m) {
+        qsort(ids, (size_t)s, sizeof(uint32_t), cmp_u32);
+        return;
+    }
+    float lo[3] = {0, 0, 0}, hi[3] = {0, 0, 0}, ext[3] = {0, 0, 0};
+    int any = 0;
+    for (int64_t i = 0; i < s; ++i) {
+        uint32_t id = ids[i];
+        if ((int64_t)id >= n) continue;
+        for (int a = 0; a < 3; ++a) {
+            float v = c[3 * (int64_t)id + a];
+            if (v == 0.0f) v = 0.0f;
+            if (!any || v < lo[a]) lo[a] = v;
+            if (!any || v > hi[a]) hi[a] = v;
+        }
+        any = 1;
+    }
+    if (any)
+        for (int a = 0; a < 3; ++a) ext[a] = hi[a] - lo[a];
+    int axis = 0;
+    if (ext[1] > ext[axis]) axis = 1;
+    if (ext[2] > ext[axis]) axis = 2;
+    for (int64_t i = 0; i < s; ++i) {
+        uint32_t id = ids[i];
+        uint64_t key = ((int64_t)id < n) ? ord_key(c[3 * (int64_t)id + axis]) : 0xFFFFFFFFu;
+        tmp[i] = (key << 32) | id;
+    }
+    qsort(tmp, (size_t)s, sizeof(uint64_t), cmp_u64);
+    for (int64_t i = 0; i < s; ++i) ids[i] = (uint32_t)tmp[i];
+    build_node(c, n, m, ids, s / 2, tmp);
+    build_node(c, n, m, ids + s / 2, s / 2, tmp);
+}
+
+static int64_t padded(int64_t n, int32_t m)
+{
+    int64_t leaves = (n + m - 1) / m, p = 1;
+    if (leaves < 1) leaves = 1;
+    while (p < leaves) p <<= 1;
+    return p * m;
+}
+
+/*
+ * Build the tree of every cloud of a batch.
+ *   coords   float [offsets[B], 3], clouds concatenated in row order
+ *   offsets  int64 [B+1]
+ *   perm_out int32 [sum of padded sizes]: slot -> global row (offsets[b] + local id), -1 for dummies
+ *   pad_out  int64 [B+1]: slot offset of every cloud
+ */
+int orc_build(const float *coords, const int64_t *offsets, int32_t B, int32_t m, int32_t *perm_out,
+              int64_t *pad_out)
+{
+    if (!coords || !offsets || !perm_out || !pad_out || B < 1) return ORC_ERR_ARG;
+    if (m < 1) return ORC_ERR_SHAPE;
+    for (int64_t i = 0; i < 3 * offsets[B]; ++i)
+        if (!isfinite(coords[i])) return ORC_ERR_NONFINITE;
+    pad_out[0] = 0;
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t n = offsets[b + 1] - offsets[b];
+        if (n < 1) return ORC_ERR_SHAPE;
+        pad_out[b + 1] = pad_out[b] + padded(n, m);
+    }
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t n = offsets[b + 1] - offsets[b], s = pad_out[b + 1] - pad_out[b];
+        uint32_t *ids = (uint32_t *)malloc((size_t)s * sizeof(uint32_t));
+        uint64_t *tmp = (uint64_t *)malloc((size_t)s * sizeof(uint64_t));
+        if (!ids || !tmp) { free(ids); free(tmp); return ORC_ERR_ARG; }
+        for (int64_t i = 0; i < s; ++i) ids[i] = (uint32_t)i;
+        build_node(coords + 3 * offsets[b], n, m, ids, s, tmp);
+        for (int64_t i = 0; i < s; ++i)
+            perm_out[pad_out[b] + i] = ((int64_t)ids[i] < n) ? (int32_t)(offsets[b] + ids[i]) : -1;
+        free(ids);
+        free(tmp);
+    }
+    return ORC_OK;
+}
+
+/*
+ * Rotation by 45 degrees counter-clockwise about +z through the origin, in
+ * float with every product and sum rounded on its own (no fused multiply-add):
+ *   x' = c*x - s*y,  y' = s*x + c*y,  z' = z,  c = s = float(sqrt(1/2)).
+ */
+void orc_rotate_z(const float *in, int64_t n, float *out)
+{
+    const uint32_t bits = 0x3F3504F3u; /* nearest float to sqrt(1/2) */
+    float c, s;
+    memcpy(&c, &bits, 4);
+    s = c;
+    for (int64_t i = 0; i < n; ++i) {
+        float x = in[3 * i], y = in[3 * i + 1], z = in[3 * i + 2];
+        volatile float cx = c * x, sy = s * y, sx = s * x, cy = c * y;
+        out[3 * i] = cx - sy;
+        out[3 * i + 1] = sx + cy;
+        out[3 * i + 2] = z;
+    }
+}
+
+/* element (row, head, k) of a [rows, H, d] tensor, widened to double */
+static double widen(const void *p, int dtype, int64_t idx)
+{
+    if (dtype == 0) return (double)((const float *)p)[idx];
+    uint32_t u = (uint32_t)((const uint16_t *)p)[idx] << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/*
+ * Attention of one query row over a list of key rows, in double:
+ *   O = sum_j softmax_j(q . k_j / sqrt(d)) v_j ; no key -> O = 0.
+ */
+static void attend(const void *Q, const void *K, const void *V, int dtype, int32_t H, int32_t d, int32_t h,
+                   int64_t qrow, const int64_t *krows, int64_t nk, double *logit, double *o)
+{
+    double scale = 1.0 / sqrt((double)d), mx = -INFINITY, den = 0.0;
+    for (int k = 0; k < d; ++k) o[k] = 0.0;
+    if (nk == 0) return;
+    for (int64_t j = 0; j < nk; ++j) {
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k)
+            acc += widen(Q, dtype, (qrow * H + h) * d + k) * widen(K, dtype, (krows[j] * H + h) * d + k);
+        logit[j] = acc * scale;
+        if (logit[j] > mx) mx = logit[j];
+    }
+    for (int64_t j = 0; j < nk; ++j) {
+        double w = exp(logit[j] - mx);
+        den += w;
+        for (int k = 0; k < d; ++k) o[k] += w * widen(V, dtype, (krows[j] * H + h) * d + k);
+    }
+    for (int k = 0; k < d; ++k) o[k] /= den;
+}
+
+/*
+ * Ball attention.  Slots are grouped in balls of m consecutive slots; slot s
+ * holds row perm[s] of Q/K/V (perm == NULL: row s), or a dummy (perm[s] < 0)
+ * that is neither a query nor a key.  Output O [rows, H, d] (double) in the
+ * original row order; only rows of the listed balls are written
+ * (balls == NULL: every ball).  dtype 0 = float32, 1 = bfloat16 bits.
+ */
+int orc_ball_attention(const void *Q, const void *K, const void *V, int dtype, const int32_t *perm, int64_t npad,
+                       int32_t m, int32_t H, int32_t d, const int64_t *balls, int64_t n_balls, double *O)
+{
+    if (!Q || !K || !V || !O || m < 1 || H < 1 || d < 1 || npad % m) return ORC_ERR_ARG;
+    int64_t nb = balls ? n_balls : npad / m;
+    int64_t *krows = (int64_t *)malloc((size_t)m * sizeof(int64_t));
+    double *logit = (double *)malloc((size_t)m * sizeof(double));
+    if (!krows || !logit) { free(krows); free(logit); return ORC_ERR_ARG; }
+    for (int64_t t = 0; t < nb; ++t) {
+        int64_t b = balls ? balls[t] : t;
+        int64_t nk = 0;
+        for (int64_t j = 0; j < m; ++j) {
+            int64_t r = perm ? perm[b * m + j] : b * m + j;
+            if (r >= 0) krows[nk++] = r;
+        }
+        for (int32_t h = 0; h < H; ++h)
+            for (int64_t i = 0; i < nk; ++i)
+                attend(Q, K, V, dtype, H, d, h, krows[i], krows, nk, logit, O + (krows[i] * H + h) * d);
+    }
+    free(krows);
+    free(logit);
+    return ORC_OK;
+}
+
+/*
+ * Full attention over all n rows (every row a key) for the listed query rows
+ * (rows == NULL: all).  Output O [n, H, d] double.
+ */
+int orc_full_attention(const void *Q, const void *K, const void *V, int dtype, int64_t n, int32_t H, int32_t d,
+                       const int64_t *rows, int64_t n_rows, double *O)
+{
+    if (!Q || !K || !V || !O || n < 1 || H < 1 || d < 1) return ORC_ERR_ARG;
+    int64_t *krows = (int64_t *)malloc((size_t)n * sizeof(int64_t));
+    double *logit = (double *)malloc((size_t)n * sizeof(double));
+    if (!krows || !logit) { free(krows); free(logit); return ORC_ERR_ARG; }
+    for (int64_t j = 0; j < n; ++j) krows[j] = j;
+    int64_t nq = rows ? n_rows : n;
+    for (int64_t t = 0; t < nq; ++t) {
+        int64_t r = rows ? rows[t] : t;
+        for (int32_t h = 0; h < H; ++h) attend(Q, K, V, dtype, H, d, h, r, krows, n, logit, O + (r * H + h) * d);
+    }
+    free(krows);
+    free(logit);
+    return ORC_OK;
+}
+
+/* inverse permutation and composition (slot maps between two trees of one cloud set) */
+void orc_invert(const int32_t *perm, int64_t npad, int32_t *inv, int64_t n_rows)
+{
+    for (int64_t r = 0; r < n_rows; ++r) inv[r] = -1;
+    for (int64_t s = 0; s < npad; ++s)
+        if (perm[s] >= 0) inv[perm[s]] = (int32_t)s;
+}
+
+void orc_compose(const int32_t *invA, const int32_t *permB, int64_t npad, int32_t *map)
+{
+    for (int64_t s = 0; s < npad; ++s) map[s] = permB[s] >= 0 ? invA[permB[s]] : -1;
+}
