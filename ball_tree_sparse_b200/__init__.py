@@ -1,0 +1,207 @@
+"""Python binding of libbts.so (ball-tree build + ball attention on B200).
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+The functions carry the names of the C entry points in ``include/bts.h``,
+take torch CUDA tensors (torch supplies device memory and the current
+stream) and raise :class:`BtsError` on a non-OK status.  There is no CPU
+fallback: importing fails loudly when the compiled library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbts.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libbts.so not found at {LIB_PATH}; build it with "
+                      "`python -m ball_tree_sparse_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+STATUS = {0: "BT_OK", 1: "BT_ERR_ARG", 2: "BT_ERR_SHAPE", 3: "BT_ERR_NONFINITE", 4: "BT_ERR_WORKSPACE",
+          5: "BT_ERR_CUDA", 6: "BT_ERR_TIMEOUT", 7: "BT_ERR_UNSUPPORTED",
+          8: "BT_ERR_INTERNAL"}
+BT_F32, BT_BF16 = 0, 1
+MAX_CLOUDS = 64
+
+_P, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+_SIGS = {
+    "bt_version": ([], ctypes.c_int32),
+    "bt_build_workspace_size": ([_P, _i32, _i32], _sz),
+    "bt_build": ([_P, _i64, _i32, _P, _P, _sz, _P], ctypes.c_int),
+    "bt_build_segmented": ([_P, _P, _i32, _i32, _P, _P, _P, _sz, _P], ctypes.c_int),
+    "bt_build_device_status": ([_P, _P], ctypes.c_int),
+    "bt_rotate_z": ([_P, _i64, _P, _P], ctypes.c_int),
+    "bt_invert_perm": ([_P, _i64, _i64, _P, _P], ctypes.c_int),
+    "bt_compose": ([_P, _P, _i64, _P, _P], ctypes.c_int),
+    "bt_gather": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
+    "bt_scatter": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
+    "bt_ball_attention": ([_P, _P, _P, _P, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
+    "bt_attention_device_status": ([_P], ctypes.c_int),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+class BtsError(RuntimeError):
+    def __init__(self, call: str, code: int):
+        super().__init__(f"{call} returned {STATUS.get(code, code)}")
+        self.code = code
+        self.status = STATUS.get(code, str(code))
+
+
+def _check(call: str, code: int) -> None:
+    if code != 0:
+        raise BtsError(call, code)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _offsets_array(offsets) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(offsets, dtype=np.int64))
+
+
+def bt_version() -> int:
+    return int(_lib.bt_version())
+
+
+version = bt_version
+
+
+def bt_build_workspace_size(offsets, m: int) -> int:
+    off = _offsets_array(offsets)
+    return int(_lib.bt_build_workspace_size(off.ctypes.data_as(_P), len(off) - 1, m))
+
+
+def workspace(offsets, m: int, device=None) -> torch.Tensor:
+    """A workspace tensor of the size bt_build_workspace_size() asks for (torch allocates it)."""
+    n = bt_build_workspace_size(offsets, m)
+    if n == 0:
+        raise BtsError("bt_build_workspace_size", 1)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def bt_build(coords: torch.Tensor, m: int, perm: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+             stream=None) -> torch.Tensor:
+    """Ball tree of one cloud of N = m * 2^L points: returns perm int32 [N] (slot -> row)."""
+    N = coords.shape[0]
+    if perm is None:
+        perm = torch.empty(N, dtype=torch.int32, device=coords.device)
+    if ws is None:
+        ws = workspace([0, N], m, coords.device)
+    _check("bt_build", _lib.bt_build(_dptr(coords), N, m, _dptr(perm), _dptr(ws), ws.numel(), _stream(stream)))
+    return perm
+
+
+def bt_build_segmented(coords: torch.Tensor, offsets, m: int, perm: torch.Tensor | None = None,
+                       ws: torch.Tensor | None = None, stream=None):
+    """Ball trees of a batch of clouds (padded with dummies).  Returns (perm int32 [sum Npad], pad_offsets)."""
+    off = _offsets_array(offsets)
+    B = len(off) - 1
+    pad = np.zeros(B + 1, np.int64)
+    if perm is None:
+        sizes = [_padded(int(off[b + 1] - off[b]), m) for b in range(B)]
+        perm = torch.empty(sum(sizes), dtype=torch.int32, device=coords.device)
+    if ws is None:
+        ws = workspace(off, m, coords.device)
+    _check("bt_build_segmented",
+           _lib.bt_build_segmented(_dptr(coords), off.ctypes.data_as(_P), B, m, _dptr(perm),
+                                   pad.ctypes.data_as(_P), _dptr(ws), ws.numel(), _stream(stream)))
+    return perm, pad
+
+
+def _padded(n: int, m: int) -> int:
+    leaves = max(1, -(-n // m))
+    return m * (1 << (leaves - 1).bit_length())
+
+
+def bt_build_device_status(ws: torch.Tensor, stream=None) -> int:
+    return int(_lib.bt_build_device_status(_dptr(ws), _stream(stream)))
+
+
+def bt_rotate_z(coords: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty_like(coords)
+    _check("bt_rotate_z", _lib.bt_rotate_z(_dptr(coords), coords.shape[0], _dptr(out), _stream(stream)))
+    return out
+
+
+def bt_invert_perm(perm: torch.Tensor, n_rows: int, inv: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if inv is None:
+        inv = torch.empty(n_rows, dtype=torch.int32, device=perm.device)
+    _check("bt_invert_perm", _lib.bt_invert_perm(_dptr(perm), perm.numel(), n_rows, _dptr(inv), _stream(stream)))
+    return inv
+
+
+def bt_compose(invA: torch.Tensor, permB: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    if out is None:
+        out = torch.empty_like(permB)
+    _check("bt_compose", _lib.bt_compose(_dptr(invA), _dptr(permB), permB.numel(), _dptr(out), _stream(stream)))
+    return out
+
+
+def bt_gather(X: torch.Tensor, idx: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y[s] = X[idx[s]] (zero row where idx[s] < 0); rows are X's trailing dimensions."""
+    npad = idx.numel()
+    if out is None:
+        out = torch.empty((npad, *X.shape[1:]), dtype=X.dtype, device=X.device)
+    row_bytes = X[0].numel() * X.element_size() if X.shape[0] else out[0].numel() * out.element_size()
+    _check("bt_gather", _lib.bt_gather(_dptr(X), _dptr(idx), npad, row_bytes, _dptr(out), _stream(stream)))
+    return out
+
+
+def bt_scatter(Y: torch.Tensor, idx: torch.Tensor, X: torch.Tensor, stream=None) -> torch.Tensor:
+    """X[idx[s]] = Y[s] for idx[s] >= 0."""
+    npad = idx.numel()
+    row_bytes = Y[0].numel() * Y.element_size()
+    _check("bt_scatter", _lib.bt_scatter(_dptr(Y), _dptr(idx), npad, row_bytes, _dptr(X), _stream(stream)))
+    return X
+
+
+def bt_ball_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.Tensor | None, m: int,
+                      out: torch.Tensor | None = None, npad: int | None = None, stream=None) -> torch.Tensor:
+    """Attention inside every ball of m slots.  Q/K/V/O [rows, H, d] fp32 or bf16 in original row order;
+    perm int32 [npad] slot -> row (-1 dummy) or None (row s in slot s)."""
+    rows, H, d = Q.shape
+    if Q.dtype == torch.float32:
+        dt = BT_F32
+    elif Q.dtype == torch.bfloat16:
+        dt = BT_BF16
+    else:
+        raise TypeError("Q/K/V must be float32 or bfloat16")
+    if not (K.dtype == V.dtype == Q.dtype):
+        raise TypeError("Q, K and V must share one dtype")
+    if npad is None:
+        npad = perm.numel() if perm is not None else rows
+    if out is None:
+        out = torch.empty_like(Q)
+    _check("bt_ball_attention",
+           _lib.bt_ball_attention(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, m, H, d, dt, _dptr(out),
+                                  _stream(stream)))
+    return out
+
+
+def bt_attention_device_status(stream=None) -> int:
+    return int(_lib.bt_attention_device_status(_stream(stream)))

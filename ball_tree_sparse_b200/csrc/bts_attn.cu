@@ -1,0 +1,438 @@
+// Ball Tree Attention ("Erwin: A Tree-based Hierarchical Transformer for
+// Large-scale Physical Systems", author's thread post 7/N; PMLR abstract):
+// scaled dot-product attention restricted to every ball of m consecutive
+// tree slots, all balls and heads in parallel.
+//
+// Two kernels:
+//  - k_ball_attn_tc   bf16, m dividing 128: one CTA per (128-slot tile, head).
+//                     Q/K/V rows are gathered through perm with cp.async into
+//                     the no-swizzle canonical tensor-core layouts, S = QK^T
+//                     runs on tcgen05 (M=128, N=128) into TMEM, the softmax
+//                     reads S back with tcgen05.ld (one row per thread), writes
+//                     P (bf16, unnormalised) to shared memory, O = PV runs on
+//                     tcgen05 (N=d) into the TMEM columns S used, and the
+//                     epilogue scales by 1/rowsum and scatters O through perm.
+//                     Balls smaller than 128 share a tile; keys of other balls
+//                     and dummy keys get weight 0.
+//  - k_ball_attn_simt fp32 (and any other shape): one CTA per (ball, head) on
+//                     the CUDA cores, exact two-pass softmax.
+#include <cuda_bf16.h>
+
+#include "bts_internal.cuh"
+
+namespace bts {
+
+__device__ uint32_t g_attn_status;
+
+// ---------------------------------------------------------------------------
+// CUDA-core kernel
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T>
+__device__ __forceinline__ T from_f(float v);
+template <>
+__device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+template <typename T, int D>
+__global__ void k_ball_attn_simt(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
+                                 const int32_t *__restrict__ perm, int m, int H, float scale, T *__restrict__ O)
+{
+    extern __shared__ __align__(16) float fsm[];
+    float *sK = fsm, *sV = fsm + m * D;
+    int32_t *sRow = reinterpret_cast<int32_t *>(sV + m * D);
+    const int64_t b = blockIdx.x;
+    const int h = blockIdx.y;
+    for (int j = threadIdx.x; j < m; j += blockDim.x) sRow[j] = perm ? perm[b * m + j] : int32_t(b * m + j);
+    __syncthreads();
+    for (int e = threadIdx.x; e < m * D; e += blockDim.x) {
+        const int j = e / D, k = e - j * D;
+        const int32_t r = sRow[j];
+        float kv = 0.0f, vv = 0.0f;
+        if (r >= 0) {
+            const size_t off = (size_t(r) * H + h) * D + k;
+            kv = to_f(K[off]);
+            vv = to_f(V[off]);
+        }
+        sK[e] = kv;
+        sV[e] = vv;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < m; i += blockDim.x) {
+        const int32_t r = sRow[i];
+        if (r < 0) continue;
+        float q[D];
+#pragma unroll
+        for (int k = 0; k < D; ++k) q[k] = to_f(Q[(size_t(r) * H + h) * D + k]);
+        float mx = -INFINITY;
+        for (int j = 0; j < m; ++j) {
+            if (sRow[j] < 0) continue;
+            float s = 0.0f;
+#pragma unroll
+            for (int k = 0; k < D; ++k) s = fmaf(q[k], sK[j * D + k], s);
+            mx = fmaxf(mx, s * scale);
+        }
+        float den = 0.0f, acc[D];
+#pragma unroll
+        for (int k = 0; k < D; ++k) acc[k] = 0.0f;
+        for (int j = 0; j < m; ++j) {
+            if (sRow[j] < 0) continue;
+            float s = 0.0f;
+#pragma unroll
+            for (int k = 0; k < D; ++k) s = fmaf(q[k], sK[j * D + k], s);
+            const float w = expf(s * scale - mx);
+            den += w;
+#pragma unroll
+            for (int k = 0; k < D; ++k) acc[k] = fmaf(w, sV[j * D + k], acc[k]);
+        }
+        const float inv = 1.0f / den;
+#pragma unroll
+        for (int k = 0; k < D; ++k) O[(size_t(r) * H + h) * D + k] = from_f<T>(acc[k] * inv);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 / TMEM kernel
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory matrix descriptor, no swizzle: start, leading-dimension byte
+// offset (between core matrices along K), stride byte offset (between core
+// matrices along M/N), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t(lbo >> 4) << 16) | (uint64_t(sbo >> 4) << 32) |
+           (uint64_t(1) << 46);
+}
+
+// Instruction descriptor for kind::f16: bf16 A and B, f32 accumulator, M=128.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n, bool b_mn_major)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn_major) << 16) | (uint32_t(n >> 3) << 17) |
+           (uint32_t(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase; false (and an error recorded) if it never completes.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    for (int i = 0; i < (1 << 18); ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    record_error(&g_attn_status, BT_ERR_TIMEOUT);
+    return false;
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+constexpr int kTcThreads = 128;
+constexpr int kTcCols = 128;  // TMEM columns: S [128 x 128] f32; O reuses columns 0..d-1
+
+template <int D>
+__host__ __device__ constexpr size_t tc_smem_bytes()
+{
+    // P (32 KB, aliased by Q and K before it is written) + V; padded so that at
+    // most four CTAs share an SM, which is what their TMEM columns allow.
+    return size_t(128 * 128 * 2 + D * 256) > size_t(50 * 1024) ? size_t(128 * 128 * 2 + D * 256)
+                                                                 : size_t(50 * 1024);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 4)
+    k_ball_attn_tc(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+                   const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ perm, int64_t npad, int lm, int H,
+                   float sl2, __nv_bfloat16 *__restrict__ O)
+{
+    constexpr int KCH = D / 8;                // 16-byte chunks per row of one head
+    constexpr uint32_t QK_SBO = KCH * 128;    // bytes between 8-row groups of Q and K
+    constexpr uint32_t P_SBO = 16 * 128;      // bytes between 8-row groups of P (128 keys)
+    constexpr uint32_t V_SBO = 16 * 128;      // bytes between 8-column groups of V (128 keys)
+    constexpr uint32_t V_OFF = 128 * 128 * 2;
+    constexpr uint32_t IDESC_S = idesc_bf16(128, false);
+    constexpr uint32_t IDESC_O = idesc_bf16(D, true);
+    extern __shared__ __align__(1024) uint8_t tsm[];
+    __shared__ int32_t sRow[128];
+    __shared__ uint32_t sKeyMask[4];
+    __shared__ __align__(8) uint64_t sBar;
+    __shared__ uint32_t sTmem;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m = 1 << lm;
+    const int h = blockIdx.y;
+    const int64_t slot = int64_t(blockIdx.x) * 128 + tid;
+    uint8_t *sQ = tsm, *sK = tsm + D * 256, *sP = tsm, *sV = tsm + V_OFF;
+
+    const int32_t row = slot < npad ? (perm ? perm[slot] : int32_t(slot)) : -1;
+    sRow[tid] = row;
+    const uint32_t vb = __ballot_sync(0xffffffffu, row >= 0);
+    if (lane == 0) sKeyMask[warp] = vb;
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sTmem)),
+                     "r"(kTcCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    // gather Q, K (K-major core matrices) and V (MN-major core matrices) of head h
+    for (int u = tid; u < 128 * KCH; u += kTcThreads) {
+        const int r = u / KCH, c = u - r * KCH;
+        const int32_t rr = sRow[r];
+        const size_t goff = rr >= 0 ? (size_t(rr) * H + h) * D + c * 8 : 0;
+        const uint32_t so = (r >> 3) * QK_SBO + c * 128 + (r & 7) * 16;
+        cp_async16(sQ + so, Q + goff, rr >= 0);
+        cp_async16(sK + so, K + goff, rr >= 0);
+        cp_async16(sV + c * V_SBO + r * 16, V + goff, rr >= 0);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sTmem;
+    const uint32_t bar = smem_u32(&sBar);
+
+    // S = Q K^T  (M=128, N=128, K=D)
+    if (tid == 0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16(tmem, smem_desc(smem_u32(sQ) + kk * 256, 128, QK_SBO),
+                     smem_desc(smem_u32(sK) + kk * 256, 128, QK_SBO), IDESC_S, kk > 0);
+        mma_commit(bar);
+    }
+    bool ok = mbar_wait(bar, 0);
+    tc_fence_after();
+
+    // softmax of row tid over the keys of its ball
+    const int r = tid;
+    const int W = m >= 32 ? m : 32;
+    const int c0 = m >= 32 ? ((r >> lm) << lm) : warp * 32;
+    const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
+    float mx = -INFINITY;
+    for (int cc = c0; cc < c0 + W; cc += 32) {
+        uint32_t v[32];
+        tmem_ld32(trow + cc, v);
+        const uint32_t km = sKeyMask[cc >> 5];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const bool kv = ((km >> j) & 1u) && (((cc + j) >> lm) == (r >> lm));
+            if (kv) mx = fmaxf(mx, __uint_as_float(v[j]));
+        }
+    }
+    const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
+    float sum = 0.0f;
+    uint8_t *prow = sP + (r >> 3) * P_SBO + (r & 7) * 16;
+    // all reads of S by this warp are complete before P (aliasing Q/K) is written
+    for (int cc = 0; cc < 128; cc += 32) {
+        uint32_t pk[16];
+        if (cc >= c0 && cc < c0 + W) {
+            uint32_t v[32];
+            tmem_ld32(trow + cc, v);
+            const uint32_t km = sKeyMask[cc >> 5];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+                float p0 = 0.0f, p1 = 0.0f;
+                if (((km >> j) & 1u) && (((cc + j) >> lm) == (r >> lm)))
+                    p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+                if (((km >> (j + 1)) & 1u) && (((cc + j + 1) >> lm) == (r >> lm)))
+                    p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
+                const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                sum += __low2float(pb) + __high2float(pb);
+                pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = 0u;
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+            *reinterpret_cast<uint4 *>(prow + ((cc >> 3) + t) * 128) =
+                make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // O = P V  (M=128, N=D, K=128); O overwrites TMEM columns 0..D-1
+    if (tid == 0 && ok) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(tmem, smem_desc(smem_u32(sP) + kk * 256, 128, P_SBO),
+                     smem_desc(smem_u32(sV) + kk * 256, 128, V_SBO), IDESC_O, kk > 0);
+        mma_commit(bar);
+    }
+    ok = __syncthreads_and(ok);
+    if (ok) ok = mbar_wait(bar, 1);
+    tc_fence_after();
+
+    const int32_t qrow = sRow[r];
+    if (ok) {
+        const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+#pragma unroll
+        for (int c32 = 0; c32 < D; c32 += 32) {
+            uint32_t o[32];
+            tmem_ld32(trow + c32, o);
+            if (qrow >= 0) {
+                uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qrow) * H + h) * D + c32);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * t + 2 * e]) * inv,
+                                                                        __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                    }
+                    dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcCols) : "memory");
+    }
+}
+
+template <typename T, int D>
+static bt_status launch_simt(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad, int m,
+                             int H, void *O, cudaStream_t st)
+{
+    const size_t smem = size_t(2) * m * D * 4 + size_t(m) * 4;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(k_ball_attn_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)))
+        return BT_ERR_CUDA;
+    const int threads = ((m + 31) / 32) * 32;
+    dim3 grid(unsigned(npad / m), unsigned(H));
+    k_ball_attn_simt<T, D><<<grid, threads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(K),
+                                                        static_cast<const T *>(V), perm, m, H,
+                                                        1.0f / sqrtf(float(D)), static_cast<T *>(O));
+    return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
+}
+
+template <int D>
+static bt_status launch_tc(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad, int lm,
+                           int H, void *O, cudaStream_t st)
+{
+    constexpr size_t smem = tc_smem_bytes<D>();
+    static bool set[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
+    if (dev >= 64 || !set[dev]) {
+        if (cudaFuncSetAttribute(k_ball_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)))
+            return BT_ERR_CUDA;
+        if (dev < 64) set[dev] = true;
+    }
+    dim3 grid(unsigned((npad + 127) / 128), unsigned(H));
+    const float sl2 = 1.4426950408889634f / sqrtf(float(D));
+    k_ball_attn_tc<D><<<grid, kTcThreads, smem, st>>>(
+        static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(K),
+        static_cast<const __nv_bfloat16 *>(V), perm, npad, lm, H, sl2, static_cast<__nv_bfloat16 *>(O));
+    return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
+}
+
+}  // namespace bts
+
+using namespace bts;
+
+extern "C" bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
+                                       int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream)
+{
+    if (!Q || !K || !V || !O || npad < 0 || H < 1) return BT_ERR_ARG;
+    if (m < 1 || m > 256 || (d != 32 && d != 64)) return BT_ERR_SHAPE;
+    if (npad % m) return BT_ERR_SHAPE;
+    if (dt != BT_F32 && dt != BT_BF16) return BT_ERR_ARG;
+    if (npad == 0) return BT_OK;
+    if (npad / m > 0x7FFFFFFF || int64_t(H) > 65535) return BT_ERR_UNSUPPORTED;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) |
+                         reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(O);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dt == BT_BF16 && (m == 16 || m == 32 || m == 64 || m == 128)) {
+        if (al % 16) return BT_ERR_ARG;
+        const int lm = m == 16 ? 4 : m == 32 ? 5 : m == 64 ? 6 : 7;
+        return d == 32 ? launch_tc<32>(Q, K, V, perm, npad, lm, H, O, st)
+                       : launch_tc<64>(Q, K, V, perm, npad, lm, H, O, st);
+    }
+    if (dt == BT_BF16)
+        return d == 32 ? launch_simt<__nv_bfloat16, 32>(Q, K, V, perm, npad, m, H, O, st)
+                       : launch_simt<__nv_bfloat16, 64>(Q, K, V, perm, npad, m, H, O, st);
+    return d == 32 ? launch_simt<float, 32>(Q, K, V, perm, npad, m, H, O, st)
+                   : launch_simt<float, 64>(Q, K, V, perm, npad, m, H, O, st);
+}
+
+extern "C" bt_status bt_attention_device_status(void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t h = 0, zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&h, g_attn_status, sizeof(h), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return BT_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BT_ERR_CUDA;
+    if (h && cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(zero)) != cudaSuccess) return BT_ERR_CUDA;
+    return static_cast<bt_status>(h);
+}

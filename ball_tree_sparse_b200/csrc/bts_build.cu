@@ -1,0 +1,657 @@
+// Ball-tree build on the GPU: median split along the widest axis, emitted as a
+// permutation (the tree of "Erwin: A Tree-based Hierarchical Transformer for
+// Large-scale Physical Systems", author's thread posts 6/N, 9/N and 15/N).
+//
+// Design (sm_100a, one cloud or a batch of clouds):
+//   1. k_init       - per point: fold -0, reject NaN/Inf, write the order-
+//                     preserving keys of x, y, z, the index list, and the
+//                     digit histograms of all four radix passes.
+//   2. k_sort_pass  - four stable 8-bit LSD radix passes that sort, inside
+//                     every cloud, the point ids by each axis' key (ties by
+//                     id).  One launch per pass, tiles chained by a bounded
+//                     decoupled look-back.  Result: lists X, Y, Z.
+//   3. k_level      - one launch per "wide" tree level (nodes larger than the
+//                     shared-memory tail).  A node's widest axis comes from
+//                     the two ends of its sorted lists, its median is the
+//                     element at position s/2 of that axis' list, and all four
+//                     lists (X, Y, Z and the index list I) are split by a
+//                     stable partition, so each stays sorted inside every
+//                     child.  No select pass is needed at any level.
+//   4. k_tail       - one CTA per node of at most T slots finishes all
+//                     remaining levels in shared memory and writes perm from
+//                     the index list (leaves come out in ascending index).
+#include <algorithm>
+#include <cstring>
+
+#include "bts_internal.cuh"
+
+namespace bts {
+
+constexpr int kSortTile = 4096;
+constexpr int kSortThreads = 512;
+constexpr int kLevelThreads = 512;
+constexpr int kLevelTileMax = 2048;
+constexpr int kTailThreads = 1024;
+constexpr int kTailMax = 4096;
+constexpr int kCounterLevel0 = 8;
+
+struct Plan {
+    int32_t B, m, T, TP, nlev, sort_tiles;
+    int64_t npad;
+    int64_t pad[BT_MAX_CLOUDS + 1];
+    int64_t n[BT_MAX_CLOUDS];
+    int64_t row0[BT_MAX_CLOUDS];
+    int32_t sort_tile0[BT_MAX_CLOUDS + 1];
+    int32_t glev[BT_MAX_CLOUDS];
+    int32_t tail0[BT_MAX_CLOUDS + 1];
+};
+
+struct Layout {
+    size_t counters, hist, sst, lst, ctrl_end, keys, sk, sv, lists, total;
+};
+
+static int ilog2(int64_t v)
+{
+    int r = 0;
+    while ((int64_t(1) << (r + 1)) <= v) ++r;
+    return r;
+}
+
+static int64_t padded_size(int64_t n, int32_t m)
+{
+    int64_t leaves = max64(1, (n + m - 1) / m), p = 1;
+    while (p < leaves) p <<= 1;
+    return p * m;
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Fills the plan; returns BT_OK or an argument/shape error.
+static bt_status make_plan(const int64_t *offsets, int32_t B, int32_t m, Plan &P)
+{
+    if (!offsets || B < 1) return BT_ERR_ARG;
+    if (B > BT_MAX_CLOUDS) return BT_ERR_UNSUPPORTED;
+    if (m < 1 || m > 1024) return BT_ERR_SHAPE;
+    if (offsets[0] != 0) return BT_ERR_ARG;
+    std::memset(&P, 0, sizeof(P));
+    P.B = B;
+    P.m = m;
+    P.T = m << ilog2(kTailMax / m);
+    P.TP = m << ilog2(kLevelTileMax / m);
+    const int t = ilog2(P.T / m);
+    int64_t pad = 0;
+    int32_t st = 0, tt = 0, nlev = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t n = offsets[b + 1] - offsets[b];
+        if (n < 1) return BT_ERR_ARG;
+        int64_t np = padded_size(n, m);
+        P.pad[b] = pad;
+        P.n[b] = n;
+        P.row0[b] = offsets[b];
+        P.sort_tile0[b] = st;
+        P.tail0[b] = tt;
+        int L = ilog2(np / m);
+        P.glev[b] = std::max(0, L - t);
+        nlev = std::max(nlev, P.glev[b]);
+        st += int32_t((np + kSortTile - 1) / kSortTile);
+        tt += int32_t(1) << P.glev[b];
+        pad += np;
+    }
+    P.pad[B] = pad;
+    P.sort_tile0[B] = st;
+    P.tail0[B] = tt;
+    P.sort_tiles = st;
+    P.nlev = nlev;
+    P.npad = pad;
+    if (pad > (int64_t(1) << 30) || offsets[B] > (int64_t(1) << 30)) return BT_ERR_UNSUPPORTED;
+    return BT_OK;
+}
+
+static Layout make_layout(const Plan &P)
+{
+    Layout L{};
+    const size_t np = size_t(P.npad);
+    L.counters = 64;  // word 0 is the device status
+    L.hist = 512;
+    L.sst = L.hist + size_t(3) * P.B * 4 * 256 * 4;
+    L.lst = L.sst + size_t(4) * 3 * P.sort_tiles * 256 * 4;
+    L.ctrl_end = align256(L.lst + size_t(std::max(P.nlev, 1)) * (np / P.TP) * 4 * 4);
+    L.keys = L.ctrl_end;
+    L.sk = align256(L.keys + 3 * np * 4);
+    L.sv = align256(L.sk + 2 * 3 * np * 4);
+    L.lists = align256(L.sv + 2 * 3 * np * 4);
+    L.total = align256(L.lists + 2 * 4 * np * 4);
+    return L;
+}
+
+// ---------------------------------------------------------------------------
+// 1. keys, index list, digit histograms
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kSortThreads) k_init(Plan P, const float *__restrict__ coords,
+                                                       uint32_t *__restrict__ keys, uint32_t *__restrict__ ilist,
+                                                       uint32_t *__restrict__ hist, uint32_t *status)
+{
+    __shared__ uint32_t sh[3 * 4 * 256];
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int i = tid; i < 3 * 4 * 256; i += kSortThreads) sh[i] = 0;
+    __syncthreads();
+    const int r = blockIdx.x;
+    int b = 0;
+    while (b + 1 < P.B && P.sort_tile0[b + 1] <= r) ++b;
+    const int k = r - P.sort_tile0[b];
+    const int64_t base = P.pad[b] + int64_t(k) * kSortTile;
+    const int cnt = int(min64(kSortTile, P.pad[b + 1] - base));
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int e0 = 0; e0 < kSortTile; e0 += kSortThreads) {
+        const int e = e0 + tid;
+        const bool ok = e < cnt;
+        const int64_t pid = base + e;
+        const int64_t local = pid - P.pad[b];
+        const bool real = ok && local < P.n[b];
+        uint32_t key[3];
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            key[a] = kDummyKey;
+            if (real) {
+                float c = coords[(P.row0[b] + local) * 3 + a];
+                if (!isfinite(c)) record_error(status, BT_ERR_NONFINITE);
+                key[a] = float_key(c);
+            }
+            if (ok) keys[int64_t(a) * P.npad + pid] = key[a];
+        }
+        if (ok) ilist[pid] = uint32_t(pid);
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const uint32_t d = ok ? ((key[a] >> (8 * p)) & 255u) : (256u + lane);
+                const uint32_t peers = __match_any_sync(0xffffffffu, d);
+                if (ok && (peers & lt) == 0u) atomicAdd(&sh[(a * 4 + p) * 256 + d], __popc(peers));
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < 3 * 4 * 256; i += kSortThreads) {
+        const uint32_t v = sh[i];
+        if (v) {
+            const int a = i >> 10, rest = i & 1023;
+            atomicAdd(&hist[(size_t(a) * P.B + b) * 1024 + rest], v);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2. one stable LSD radix pass over 8 bits, all (axis, cloud) segments at once
+// ---------------------------------------------------------------------------
+template <int PASS>
+__global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32_t *__restrict__ kin,
+                                                            const uint32_t *__restrict__ vin,
+                                                            uint32_t *__restrict__ kout, uint32_t *__restrict__ vout,
+                                                            const uint32_t *__restrict__ hist, uint32_t *sst,
+                                                            uint32_t *counters, uint32_t *status)
+{
+    constexpr int NT = kSortThreads, NW = NT / 32, PER_WARP = kSortTile / NW, ROUNDS = PER_WARP / 32;
+    constexpr int SHIFT = 8 * PASS;
+    extern __shared__ __align__(16) uint32_t dyn[];
+    uint32_t *skey = dyn, *sval = dyn + kSortTile;
+    __shared__ uint32_t whist[NW][256];
+    __shared__ uint32_t tstart[256], gpos[256];
+    __shared__ uint32_t scratch[NT / 32 + 1];
+    __shared__ uint32_t s_tile;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) s_tile = atomicAdd(&counters[PASS], 1u);
+    for (int i = tid; i < NW * 256; i += NT) (&whist[0][0])[i] = 0;
+    __syncthreads();
+    const int id = int(s_tile);
+    const int a = id / P.sort_tiles, r = id - a * P.sort_tiles;
+    int b = 0;
+    while (b + 1 < P.B && P.sort_tile0[b + 1] <= r) ++b;
+    const int k = r - P.sort_tile0[b];
+    const int64_t seg_size = P.pad[b + 1] - P.pad[b];
+    const int64_t seg_base = int64_t(a) * P.npad + P.pad[b];
+    const int64_t tile_base = seg_base + int64_t(k) * kSortTile;
+    const int cnt = int(min64(kSortTile, seg_size - int64_t(k) * kSortTile));
+
+    uint32_t key[ROUNDS], val[ROUNDS], dig[ROUNDS], rnk[ROUNDS];
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int q = 0; q < ROUNDS; ++q) {
+        const int e = warp * PER_WARP + q * 32 + lane;
+        const bool ok = e < cnt;
+        key[q] = ok ? kin[tile_base + e] : 0u;
+        if (PASS == 0)
+            val[q] = uint32_t(P.pad[b] + int64_t(k) * kSortTile + e);
+        else
+            val[q] = ok ? vin[tile_base + e] : 0u;
+        dig[q] = ok ? ((key[q] >> SHIFT) & 255u) : (256u + lane);
+    }
+    // stable rank of every element among equal digits of its warp, warp counts
+#pragma unroll
+    for (int q = 0; q < ROUNDS; ++q) {
+        const uint32_t peers = __match_any_sync(0xffffffffu, dig[q]);
+        const bool ok = dig[q] < 256u;
+        const uint32_t base = ok ? whist[warp][dig[q]] : 0u;
+        __syncwarp();
+        if (ok && (peers & lt) == 0u) whist[warp][dig[q]] = base + __popc(peers);
+        __syncwarp();
+        rnk[q] = base + __popc(peers & lt);
+    }
+    __syncthreads();
+    uint32_t dcount = 0;
+    if (tid < 256) {
+        uint32_t run = 0;
+        for (int w = 0; w < NW; ++w) {
+            const uint32_t c = whist[w][tid];
+            whist[w][tid] = run;
+            run += c;
+        }
+        dcount = run;
+    }
+    const uint32_t ts = block_exclusive_scan<NT, uint32_t>(tid < 256 ? dcount : 0u, scratch, nullptr);
+    const int g = a * P.B + b;
+    const uint32_t hc = tid < 256 ? hist[(size_t(g) * 4 + PASS) * 256 + tid] : 0u;
+    const uint32_t gb = block_exclusive_scan<NT, uint32_t>(hc, scratch, nullptr);
+    if (tid < 256) {
+        const uint32_t excl =
+            lookback(&sst[(size_t(PASS) * 3 * P.sort_tiles + id) * 256 + tid], 256, k, dcount, status);
+        tstart[tid] = ts;
+        gpos[tid] = gb + excl - ts;  // modulo 2^32; + local index gives the position in the segment
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < ROUNDS; ++q) {
+        if (dig[q] < 256u) {
+            const uint32_t j = tstart[dig[q]] + whist[warp][dig[q]] + rnk[q];
+            skey[j] = key[q];
+            sval[j] = val[q];
+        }
+    }
+    __syncthreads();
+    for (int j = tid; j < cnt; j += NT) {
+        const uint32_t kk = skey[j];
+        const uint32_t d = (kk >> SHIFT) & 255u;
+        const int64_t rel = int64_t(uint32_t(gpos[d] + uint32_t(j)));
+        if (rel >= seg_size) {  // counts disagree with the histogram: never write outside the segment
+            record_error(status, BT_ERR_INTERNAL);
+            continue;
+        }
+        if (PASS < 3) kout[seg_base + rel] = kk;
+        vout[seg_base + rel] = sval[j];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. one wide level: split every node larger than T at the median of its widest axis
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const uint32_t *__restrict__ keys,
+                                                         const uint32_t *__restrict__ lin, uint32_t *__restrict__ lout,
+                                                         uint32_t *lst, uint32_t *counters, uint32_t *status)
+{
+    constexpr int NT = kLevelThreads;
+    __shared__ uint32_t sl[4][kLevelTileMax];
+    __shared__ unsigned long long scratch[NT / 32 + 1];
+    __shared__ uint32_t s_tile, s_excl[4];
+    __shared__ int s_axis;
+    __shared__ float s_ext[3];
+    __shared__ unsigned long long s_piv;
+    const int tid = threadIdx.x;
+    if (tid == 0) s_tile = atomicAdd(&counters[kCounterLevel0 + lev], 1u);
+    __syncthreads();
+    const int id = int(s_tile);
+    const int64_t np = P.npad;
+    const int TP = P.TP;
+    int b = 0;
+    int64_t r = id;
+    for (;;) {
+        const int64_t sb = P.pad[b + 1] - P.pad[b];
+        const int64_t nt = ((sb >> lev) > P.T) ? sb / TP : 0;
+        if (r < nt || b + 1 >= P.B) break;
+        r -= nt;
+        ++b;
+    }
+    const int64_t s = (P.pad[b + 1] - P.pad[b]) >> lev, half = s >> 1;
+    const int64_t tps = s / TP, kseg = r / tps;
+    const int j = int(r - kseg * tps);
+    const int64_t seg = P.pad[b] + kseg * s;
+    const int64_t nreal = max64(0, min64(s, P.n[b] - kseg * s));
+    if (tid < 3) {
+        float e = 0.0f;
+        if (nreal > 0) {
+            const uint32_t p0 = lin[tid * np + seg], p1 = lin[tid * np + seg + nreal - 1];
+            e = __fsub_rn(key_float(keys[tid * np + p1]), key_float(keys[tid * np + p0]));
+        }
+        s_ext[tid] = e;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int ax = 0;
+        if (s_ext[1] > s_ext[ax]) ax = 1;
+        if (s_ext[2] > s_ext[ax]) ax = 2;
+        const uint32_t pp = lin[ax * np + seg + half];
+        s_axis = ax;
+        s_piv = (static_cast<unsigned long long>(keys[ax * np + pp]) << 32) | pp;
+    }
+    const int64_t tile0 = seg + int64_t(j) * TP;
+    for (int l = 0; l < 4; ++l)
+        for (int i = tid; i < TP; i += NT) sl[l][i] = lin[l * np + tile0 + i];
+    __syncthreads();
+    const int ax = s_axis;
+    const unsigned long long piv = s_piv;
+    const int EPT = (TP + NT - 1) / NT;
+    const int i0 = tid * EPT;
+    uint32_t v[4][4];
+    uint32_t lbits[4] = {0, 0, 0, 0};
+    unsigned long long packed = 0;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q;
+            v[l][q] = 0;
+            if (q < EPT && i < TP) {
+                const uint32_t pid = sl[l][i];
+                v[l][q] = pid;
+                bool left;
+                if (l == ax)
+                    left = int64_t(j) * TP + i < half;
+                else
+                    left = ((static_cast<unsigned long long>(keys[ax * np + pid]) << 32) | pid) < piv;
+                if (left) {
+                    lbits[l] |= 1u << q;
+                    packed += 1ull << (16 * l);
+                }
+            }
+        }
+    }
+    unsigned long long tot = 0;
+    const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, &tot);
+    if (tid < 4)
+        s_excl[tid] = lookback(&lst[(size_t(lev) * (np / TP) + id) * 4 + tid], 4, j,
+                               uint32_t((tot >> (16 * tid)) & 0xFFFFu), status);
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+        const int nl = int((tot >> (16 * l)) & 0xFFFFu);
+        int run = int((ex >> (16 * l)) & 0xFFFFu);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int i = i0 + q;
+            if (q < EPT && i < TP) {
+                const bool left = (lbits[l] >> q) & 1u;
+                const int pos = left ? run : nl + (i - run);
+                run += left;
+                sl[l][pos] = v[l][q];
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+        const int nl = int((tot >> (16 * l)) & 0xFFFFu);
+        const int64_t exl = s_excl[l];
+        for (int i = tid; i < TP; i += NT) {
+            const int64_t dst = i < nl ? exl + i : half + (int64_t(j) * TP - exl) + (i - nl);
+            if ((i < nl && dst >= half) || dst < 0 || dst >= s) {  // left count != s/2: a broken invariant
+                record_error(status, BT_ERR_INTERNAL);
+                continue;
+            }
+            lout[l * np + seg + dst] = sl[l][i];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 4. the remaining levels of one node of at most T slots, in shared memory
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int find_local(const uint32_t *ps, int n, uint32_t pid)
+{
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (ps[mid] < pid)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kTailThreads) k_tail(Plan P, const uint32_t *__restrict__ keys,
+                                                       const uint32_t *__restrict__ lists, int32_t *__restrict__ perm,
+                                                       uint32_t *status)
+{
+    constexpr int NT = kTailThreads;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ unsigned long long scratch[NT / 32 + 1];
+    const int T = P.T;
+    uint32_t *ps = reinterpret_cast<uint32_t *>(dsm);            // [T] point ids, ascending
+    uint32_t *k3 = ps + T;                                       // [3][T] keys by local index
+    unsigned long long *piv = reinterpret_cast<unsigned long long *>(k3 + 3 * T);  // [T/2]
+    unsigned long long *segpre = piv + T / 2;                    // [T/2]
+    uint16_t *lst = reinterpret_cast<uint16_t *>(segpre + T / 2);  // [2][4][T]
+    uint8_t *axs = reinterpret_cast<uint8_t *>(lst + 8 * T);     // [T/2]
+
+    const int tid = threadIdx.x;
+    const int id = blockIdx.x;
+    int b = 0;
+    while (b + 1 < P.B && P.tail0[b + 1] <= id) ++b;
+    const int k = id - P.tail0[b];
+    const int64_t np = P.npad;
+    const int sT = int(min64(P.pad[b + 1] - P.pad[b], T));
+    const int64_t seg = P.pad[b] + int64_t(k) * sT;
+    const int nreal = int(max64(0, min64(sT, P.n[b] - int64_t(k) * sT)));
+    const uint32_t *lin = lists + size_t(P.glev[b] & 1) * 4 * np;
+    const int m = P.m;
+
+    for (int e = tid; e < sT; e += NT) ps[e] = lin[3 * np + seg + e];
+    __syncthreads();
+    for (int e = tid; e < sT; e += NT) {
+        const uint32_t pid = ps[e];
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            k3[a * T + e] = keys[a * np + pid];
+            const uint32_t pid_a = lin[a * np + seg + e];
+            const int loc = find_local(ps, sT, pid_a);
+            if (ps[loc] != pid_a) record_error(status, BT_ERR_INTERNAL);  // lists disagree on the node's points
+            lst[a * T + e] = uint16_t(loc);
+        }
+        lst[3 * T + e] = uint16_t(e);
+    }
+    __syncthreads();
+
+    int cur = 0;
+    const int EPT = (sT + NT - 1) / NT;
+    const int i0 = tid * EPT;
+    for (int sz = sT; sz > m; sz >>= 1) {
+        const int half = sz >> 1, nsub = sT / sz;
+        uint16_t *L = lst + cur * 4 * T, *Ln = lst + (cur ^ 1) * 4 * T;
+        for (int q = tid; q < nsub; q += NT) {
+            const int start = q * sz;
+            const int nr = max(0, min(sz, nreal - start));
+            float ext[3] = {0.0f, 0.0f, 0.0f};
+            if (nr > 0) {
+#pragma unroll
+                for (int a = 0; a < 3; ++a)
+                    ext[a] = __fsub_rn(key_float(k3[a * T + L[a * T + start + nr - 1]]),
+                                       key_float(k3[a * T + L[a * T + start]]));
+            }
+            int ax = 0;
+            if (ext[1] > ext[ax]) ax = 1;
+            if (ext[2] > ext[ax]) ax = 2;
+            const uint32_t pv = L[ax * T + start + half];
+            axs[q] = uint8_t(ax);
+            piv[q] = (static_cast<unsigned long long>(k3[ax * T + pv]) << 32) | pv;
+        }
+        __syncthreads();
+        uint32_t lbits[4] = {0, 0, 0, 0};
+        unsigned long long packed = 0;
+        for (int q = 0; q < EPT; ++q) {
+            const int e = i0 + q;
+            if (e >= sT) break;
+            const int sub = e / sz;
+            const int ax = axs[sub];
+            const unsigned long long pv = piv[sub];
+#pragma unroll
+            for (int l = 0; l < 4; ++l) {
+                const uint32_t v = L[l * T + e];
+                const bool left = (l == ax) ? (e - sub * sz) < half
+                                            : ((static_cast<unsigned long long>(k3[ax * T + v]) << 32) | v) < pv;
+                if (left) {
+                    lbits[l] |= 1u << q;
+                    packed += 1ull << (16 * l);
+                }
+            }
+        }
+        const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, nullptr);
+        {
+            unsigned long long run = ex;
+            for (int q = 0; q < EPT; ++q) {
+                const int e = i0 + q;
+                if (e >= sT) break;
+                if (e % sz == 0) segpre[e / sz] = run;
+#pragma unroll
+                for (int l = 0; l < 4; ++l)
+                    if ((lbits[l] >> q) & 1u) run += 1ull << (16 * l);
+            }
+        }
+        __syncthreads();
+        {
+            unsigned long long run = ex;
+            for (int q = 0; q < EPT; ++q) {
+                const int e = i0 + q;
+                if (e >= sT) break;
+                const int sub = e / sz, start = sub * sz;
+                const unsigned long long sp = segpre[sub];
+#pragma unroll
+                for (int l = 0; l < 4; ++l) {
+                    const int pre = int(((run >> (16 * l)) & 0xFFFFu) - ((sp >> (16 * l)) & 0xFFFFu));
+                    const bool left = (lbits[l] >> q) & 1u;
+                    const int dst = left ? start + pre : start + half + (e - start - pre);
+                    if ((left && pre >= half) || dst < start || dst >= start + sz) {
+                        record_error(status, BT_ERR_INTERNAL);  // never write outside the node
+                    } else {
+                        Ln[l * T + dst] = L[l * T + e];
+                    }
+                    if (left) run += 1ull << (16 * l);
+                }
+            }
+        }
+        __syncthreads();
+        cur ^= 1;
+    }
+    const uint16_t *L = lst + cur * 4 * T;
+    for (int e = tid; e < sT; e += NT) {
+        const uint32_t pid = ps[L[3 * T + e]];
+        const int64_t li = int64_t(pid) - P.pad[b];
+        perm[seg + e] = li < P.n[b] ? int32_t(P.row0[b] + li) : -1;
+    }
+}
+
+static size_t tail_smem_bytes(int T)
+{
+    return size_t(T) * 4 + size_t(3) * T * 4 + size_t(T / 2) * 8 * 2 + size_t(8) * T * 2 + size_t(T / 2);
+}
+
+static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm, void *ws, size_t ws_bytes,
+                              cudaStream_t st)
+{
+    const Layout L = make_layout(P);
+    if (!ws) return BT_ERR_WORKSPACE;
+    if (ws_bytes < L.total) return BT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return BT_ERR_ARG;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    uint32_t *status = reinterpret_cast<uint32_t *>(w);
+    uint32_t *counters = reinterpret_cast<uint32_t *>(w + L.counters);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(w + L.hist);
+    uint32_t *sst = reinterpret_cast<uint32_t *>(w + L.sst);
+    uint32_t *lstat = reinterpret_cast<uint32_t *>(w + L.lst);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(w + L.keys);
+    uint32_t *sk = reinterpret_cast<uint32_t *>(w + L.sk);
+    uint32_t *sv = reinterpret_cast<uint32_t *>(w + L.sv);
+    uint32_t *lists = reinterpret_cast<uint32_t *>(w + L.lists);
+    const size_t np = size_t(P.npad);
+
+    static bool attrs_set[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
+    const size_t sort_smem = size_t(2) * kSortTile * 4;
+    const size_t tail_smem = tail_smem_bytes(P.T);
+    if (dev < 64 && !attrs_set[dev]) {
+        if (cudaFuncSetAttribute(k_sort_pass<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
+            cudaFuncSetAttribute(k_sort_pass<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
+            cudaFuncSetAttribute(k_sort_pass<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
+            cudaFuncSetAttribute(k_sort_pass<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
+            cudaFuncSetAttribute(k_tail, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(tail_smem_bytes(kTailMax))))
+            return BT_ERR_CUDA;
+        attrs_set[dev] = true;
+    }
+    if (cudaMemsetAsync(ws, 0, L.ctrl_end, st) != cudaSuccess) return BT_ERR_CUDA;
+    k_init<<<P.sort_tiles, kSortThreads, 0, st>>>(P, coords, keys, lists + 3 * np, hist, status);
+    const int sort_grid = 3 * P.sort_tiles;
+    k_sort_pass<0><<<sort_grid, kSortThreads, sort_smem, st>>>(P, keys, nullptr, sk, sv, hist, sst, counters, status);
+    k_sort_pass<1><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk, sv, sk + 3 * np, sv + 3 * np, hist, sst,
+                                                               counters, status);
+    k_sort_pass<2><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk + 3 * np, sv + 3 * np, sk, sv, hist, sst,
+                                                               counters, status);
+    k_sort_pass<3><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk, sv, nullptr, lists, hist, sst, counters,
+                                                               status);
+    for (int lev = 0; lev < P.nlev; ++lev) {
+        int64_t tiles = 0;
+        for (int b = 0; b < P.B; ++b) {
+            const int64_t sb = P.pad[b + 1] - P.pad[b];
+            if ((sb >> lev) > P.T) tiles += sb / P.TP;
+        }
+        const uint32_t *lin = lists + size_t(lev & 1) * 4 * np;
+        uint32_t *lout = lists + size_t((lev + 1) & 1) * 4 * np;
+        k_level<<<unsigned(tiles), kLevelThreads, 0, st>>>(P, lev, keys, lin, lout, lstat, counters, status);
+    }
+    k_tail<<<P.tail0[P.B], kTailThreads, tail_smem, st>>>(P, keys, lists, perm, status);
+    return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
+}
+
+}  // namespace bts
+
+using namespace bts;
+
+extern "C" size_t bt_build_workspace_size(const int64_t *offsets, int32_t B, int32_t m)
+{
+    Plan P;
+    if (make_plan(offsets, B, m, P) != BT_OK) return 0;
+    return make_layout(P).total;
+}
+
+extern "C" bt_status bt_build_segmented(const float *coords, const int64_t *offsets, int32_t B, int32_t m,
+                                        int32_t *perm, int64_t *pad_offsets, void *ws, size_t ws_bytes,
+                                        void *stream)
+{
+    if (!coords || !perm) return BT_ERR_ARG;
+    Plan P;
+    const bt_status s = make_plan(offsets, B, m, P);
+    if (s != BT_OK) return s;
+    for (int b = 1; b <= B; ++b)
+        if (offsets[b] <= offsets[b - 1]) return BT_ERR_ARG;
+    if (pad_offsets)
+        for (int b = 0; b <= B; ++b) pad_offsets[b] = P.pad[b];
+    return launch_build(coords, P, perm, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bt_status bt_build(const float *coords, int64_t N, int32_t m, int32_t *perm, void *ws, size_t ws_bytes,
+                              void *stream)
+{
+    if (!coords || !perm || N < 1) return BT_ERR_ARG;
+    if (m < 1 || m > 1024 || N % m) return BT_ERR_SHAPE;
+    const int64_t leaves = N / m;
+    if (leaves & (leaves - 1)) return BT_ERR_SHAPE;
+    const int64_t offsets[2] = {0, N};
+    return bt_build_segmented(coords, offsets, 1, m, perm, nullptr, ws, ws_bytes, stream);
+}
+
+extern "C" bt_status bt_build_device_status(const void *ws, void *stream)
+{
+    if (!ws) return BT_ERR_ARG;
+    uint32_t h = 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return BT_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return BT_ERR_CUDA;
+    return static_cast<bt_status>(h);
+}

@@ -1,0 +1,398 @@
+"""Throughput of the ball-tree hot path on one B200 (or N replicas under torchrun).
+
+One step = both layers of the Gaussian-mixture workload (4 clouds x 16,384
+points, m = 128, H = 8, d = 32, bf16):
+  layer A: tree build on the original coordinates + ball attention
+           (gather through perm and scatter back fused into the attention);
+  layer B: rotation by 45 deg about z, tree build on the rotated coordinates,
+           inverse of tree A and the A->B slot map, ball attention on tree B.
+Metric: points per second per layer = 2 layers * 65,536 points / step time.
+
+The step is captured once as a CUDA graph and replayed; every timed replay is
+bracketed by CUDA events on the replay stream, with a 256 MB write between
+replays to flush L2.  Kernel durations of the dominant kernel (ball attention)
+come from event nodes inside the graph.  `--impl reference` times the CPU
+oracle instead (bounded samples of the same workload on the host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "points/sec per layer (tree build + ball attention) at N=65,536; % roofline"
+UNIT = "points/s"
+LAYERS = 2
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.rows = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        self.marks = []
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        t0, t1 = (self.marks + [0, 0])[:2] if len(self.marks) >= 2 else (0, 1e30)
+        rows = [r for t, r in self.rows if t0 <= t <= t1] or [r for _, r in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 3 + i and r[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _cudart():
+    for line in open("/proc/self/maps"):
+        if "libcudart.so" in line:
+            return ctypes.CDLL(line.split()[-1])
+    return ctypes.CDLL("libcudart.so.12")
+
+
+# ---------------------------------------------------------------------------
+class Step:
+    """Device buffers and the captured graph of one step."""
+
+    def __init__(self, bts, wl, dev):
+        self.bts, self.wl, self.dev = bts, wl, dev
+        n = wl.n_total
+        self.n = n
+        self.coords = torch.from_numpy(wl.coords).to(dev)
+        self.qkv = []
+        for L in wl.layers:
+            self.qkv.append([torch.from_numpy(t.view(np.int16)).to(dev).view(torch.bfloat16) for t in (L.q, L.k, L.v)])
+        self.out = [torch.empty_like(self.qkv[0][0]) for _ in wl.layers]
+        self.npad = int(wl.pad_offsets()[-1])
+        self.perm = [torch.empty(self.npad, dtype=torch.int32, device=dev) for _ in range(2)]
+        self.rot = torch.empty_like(self.coords)
+        self.inv = torch.empty(n, dtype=torch.int32, device=dev)
+        self.map = torch.empty(self.npad, dtype=torch.int32, device=dev)
+        self.ws = bts.workspace(wl.offsets, wl.m, dev)
+        self.rt = _cudart()
+        self.rt.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        self.ev = {k: torch.cuda.Event(enable_timing=True) for k in ("a0", "a1", "a2", "b0", "b1", "b2")}
+
+    def _mark(self, key, capturing):
+        s = torch.cuda.current_stream()
+        if capturing:  # an event node inside the graph (cudaEventRecordExternal)
+            rc = self.rt.cudaEventRecordWithFlags(ctypes.c_void_p(self.ev[key].cuda_event),
+                                                  ctypes.c_void_p(s.cuda_stream), 1)
+            if rc != 0:
+                raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+        else:
+            self.ev[key].record(s)
+
+    def body(self, capturing=False):
+        bts, wl = self.bts, self.wl
+        self._mark("a0", capturing)
+        bts.bt_build_segmented(self.coords, wl.offsets, wl.m, perm=self.perm[0], ws=self.ws)
+        self._mark("a1", capturing)
+        bts.bt_ball_attention(*self.qkv[0], self.perm[0], wl.m, out=self.out[0])
+        self._mark("a2", capturing)
+        bts.bt_rotate_z(self.coords, out=self.rot)
+        bts.bt_build_segmented(self.rot, wl.offsets, wl.m, perm=self.perm[1], ws=self.ws)
+        bts.bt_invert_perm(self.perm[0], self.n, inv=self.inv)
+        bts.bt_compose(self.inv, self.perm[1], out=self.map)
+        self._mark("b1", capturing)
+        bts.bt_ball_attention(*self.qkv[1], self.perm[1], wl.m, out=self.out[1])
+        self._mark("b2", capturing)
+
+    def capture(self):
+        for _ in range(3):
+            self.body()
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.body(capturing=True)
+        torch.cuda.synchronize()
+
+    def times(self):
+        e = self.ev
+        return {"build_a": e["a0"].elapsed_time(e["a1"]), "attn_a": e["a1"].elapsed_time(e["a2"]),
+                "layer_b_prep": e["a2"].elapsed_time(e["b1"]), "attn_b": e["b1"].elapsed_time(e["b2"])}
+
+
+def kernels_per_step(wl) -> int:
+    """Launches of this library's kernels in one step (memsets excluded)."""
+    m = wl.m
+    T = m << int(math.floor(math.log2(4096 // m)))
+    t = int(math.log2(T // m))
+    nlev = 0
+    for b in range(wl.batch):
+        npad = workloads.padded_size(int(wl.offsets[b + 1] - wl.offsets[b]), m)
+        nlev = max(nlev, int(math.log2(npad // m)) - t)
+    build = 1 + 4 + nlev + 1
+    return 2 * build + 2 + 3
+
+
+# ---------------------------------------------------------------------------
+def cpu_baseline(wl, n_clouds=1):
+    """The oracle, as it stands, on one cloud of the workload (both layers in full), single-threaded."""
+    import oracle
+    oracle.compile_oracle()
+    t = time.perf_counter()
+    pts_done = 0
+    for c in range(n_clouds):
+        lo, hi = int(wl.offsets[c]), int(wl.offsets[c + 1])
+        pts = wl.coords[lo:hi]
+        for li, L in enumerate(wl.layers):
+            p = oracle.rotate_z(pts) if L.rotated else pts
+            perm, _ = oracle.build(p, wl.m)
+            if L.rotated:
+                pa, _ = oracle.build(pts, wl.m)
+                oracle.compose(oracle.invert(pa, hi - lo), perm)
+            oracle.ball_attention(L.q[lo:hi], L.k[lo:hi], L.v[lo:hi], wl.m, perm)
+        pts_done += hi - lo
+    dt = time.perf_counter() - t
+    return {"value": LAYERS * pts_done / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n_clouds} of {wl.batch} clouds ({pts_done} points): both layers in full (tree builds, "
+                      f"rotation, slot map, fp64 ball attention), single-threaded C, {dt:.1f} s"}
+
+
+def run_reference(args, wl):
+    """Reference arm: the oracle on the host cores, each step a bounded sample of the workload."""
+    import oracle
+    oracle.compile_oracle()
+    total = args.steps + args.warmup
+    budget = 150.0
+    # calibrate one ball of attention and one cloud's builds
+    lo, hi = int(wl.offsets[0]), int(wl.offsets[1])
+    L = wl.layers[0]
+    t = time.perf_counter()
+    perm, _ = oracle.build(wl.coords[lo:hi], wl.m)
+    t_build = time.perf_counter() - t
+    t = time.perf_counter()
+    oracle.ball_attention(L.q[lo:hi], L.k[lo:hi], L.v[lo:hi], wl.m, perm, balls=[0])
+    t_ball = time.perf_counter() - t
+    per_step = budget / total
+    nballs = int(max(1, min((hi - lo) // wl.m, (per_step - 3 * t_build) / max(2 * t_ball, 1e-6))))
+    step_times = []
+    for i in range(total):
+        c = i % wl.batch
+        lo, hi = int(wl.offsets[c]), int(wl.offsets[c + 1])
+        pts = wl.coords[lo:hi]
+        balls = np.arange(nballs) * ((hi - lo) // wl.m // nballs)
+        t = time.perf_counter()
+        pa, _ = oracle.build(pts, wl.m)
+        t_att = 0.0
+        for L in wl.layers:
+            if L.rotated:
+                pr = oracle.rotate_z(pts)
+                perm, _ = oracle.build(pr, wl.m)
+                oracle.compose(oracle.invert(pa, hi - lo), perm)
+            else:
+                perm = pa
+            ta = time.perf_counter()
+            oracle.ball_attention(L.q[lo:hi], L.k[lo:hi], L.v[lo:hi], wl.m, perm, balls=balls)
+            t_att += time.perf_counter() - ta
+        t_tot = time.perf_counter() - t
+        full = (t_tot - t_att) + t_att * ((hi - lo) // wl.m) / nballs
+        if i >= args.warmup:
+            step_times.append(full)
+    ms = 1e3 * statistics.mean(step_times)
+    value = LAYERS * (wl.n_total // wl.batch) / (ms / 1e3)
+    sample = (f"per step one cloud of {wl.n_total // wl.batch} points: both tree builds, rotation and slot map in "
+              f"full, fp64 ball attention on {nballs} of {(hi - lo) // wl.m} balls per layer, time extrapolated to "
+              f"all balls")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "gauss_mix 4x16384 (m=128, H=8, d=32), layers: original + rotated tree",
+                       "global_batch": 4, "seq_len": 16384, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, workloads.gauss_mix())
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+    import ball_tree_sparse_b200 as bts
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = workloads.gauss_mix()
+    st = Step(bts, wl, dev)
+    st.capture()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    clocks = ClockSampler(local)
+    for _ in range(args.warmup):
+        flush.zero_()
+        st.graph.replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ms, attn_ms, parts = [], [], {"build_a": 0.0, "attn_a": 0.0, "layer_b_prep": 0.0, "attn_b": 0.0}
+    for _ in range(args.steps):
+        flush.zero_()
+        s0.record()
+        st.graph.replay()
+        s1.record()
+        s1.synchronize()
+        step_ms.append(s0.elapsed_time(s1))
+        tt = st.times()
+        attn_ms += [tt["attn_a"], tt["attn_b"]]
+        for k in parts:
+            parts[k] += tt[k]
+    torch.cuda.synchronize()
+    clocks.mark()
+    if dist:
+        dist.barrier()
+    clocks.stop()
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * LAYERS * wl.n_total * args.steps / (total_ms / 1e3)
+
+    # end to end through the public API: pinned host inputs in, outputs back to pinned host memory
+    host_in = [torch.from_numpy(wl.coords).pin_memory()]
+    for L in wl.layers:
+        host_in += [torch.from_numpy(t.view(np.int16)).pin_memory() for t in (L.q, L.k, L.v)]
+    dev_in = [st.coords] + [t.view(torch.int16) for qkv in st.qkv for t in qkv]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.out]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    e_ms = []
+    for _ in range(e2e_steps):
+        flush.zero_()
+        s0.record()
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        st.graph.replay()
+        for h, d in zip(host_out, st.out):
+            h.copy_(d, non_blocking=True)
+        s1.record()
+        s1.synchronize()
+        e_ms.append(s0.elapsed_time(s1))
+    e_total = sum(e_ms)
+    if dist:
+        t = torch.tensor([e_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_total = float(t.item())
+    e2e_value = world * LAYERS * wl.n_total * e2e_steps / (e_total / 1e3)
+
+    peak, peak_kind = _peaks()
+    attn_bytes = 4 * wl.n_total * wl.H * wl.d * 2 + 4 * st.npad  # Q, K, V read + O written, perm read
+    attn_avg_ms = statistics.mean(attn_ms)
+    achieved = attn_bytes / (attn_avg_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "gauss_mix 4x16384 (m=128, H=8, d=32), layers: original + rotated tree",
+                   "global_batch": 4 * world, "seq_len": 16384, "parallelism": f"replicas{world}",
+                   "l2": "256 MB write between timed steps", "graph": "one CUDA graph per step"},
+        "roofline": {"bound": "hbm", "kernel": "k_ball_attn_tc<32>", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "bytes_per_launch": attn_bytes, "avg_launch_ms": attn_avg_ms, "traffic": None},
+        "breakdown_ms_per_step": {k: v / args.steps for k, v in parts.items()},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": kernels_per_step(wl) * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del st
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

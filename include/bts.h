@@ -1,0 +1,184 @@
+/*
+ * bts.h - C ABI of libbts.so: ball-tree build, rotated rebuild, row movement
+ * and ball attention on one NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title, then place on the page):
+ *  [E6]  "Erwin: A Tree-based Hierarchical Transformer for Large-scale Physical
+ *        Systems", author's thread, post 6/N: a ball tree recursively
+ *        partitions points into nested sets of similar size, each covered by
+ *        a ball.
+ *  [E7]  same thread, post 7/N: pick a tree level and compute attention
+ *        within every ball of it in parallel (Ball Tree Attention).
+ *  [E9]  same thread, post 9/N: at every level the points of one ball are
+ *        stored next to each other, so ball operations are views.
+ *  [E15] same thread, post 15/N: the tree construction is a native,
+ *        parallel component.
+ *  [ROT] thread post on cross-ball exchange: instead of shifting windows
+ *        (Swin), the tree is rotated.
+ *  [ABS] PMLR abstract of the same paper: linear-time attention in
+ *        fixed-size neighbourhoods of a ball tree partition.
+ *
+ * The split rule is the one these sources imply and leave open: every node
+ * of s slots is cut into two halves of s/2 at the median of the axis of
+ * largest extent (float max - min over its real points, lowest axis on equal
+ * extents), points ordered by (coordinate, original index) with -0 equal to
+ * +0; leaves list their points in ascending original index.
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers owned by the caller unless marked "host".
+ *    The library allocates nothing; scratch comes from a caller workspace.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument errors are returned before anything is
+ *    enqueued.  Errors found on the device (non-finite coordinates, an
+ *    inter-block wait that ran out) are recorded in the workspace and read
+ *    back by bt_build_device_status().  No call traps, aborts or prints.
+ *  - Arrays are row-major and contiguous.  Coordinates are float [rows, 3].
+ *    Q/K/V/O are [rows, H, d] (H heads of d values per row).
+ */
+#ifndef BTS_H
+#define BTS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BT_OK = 0,
+    BT_ERR_ARG = 1,         /* NULL pointer, size out of range, misaligned pointer */
+    BT_ERR_SHAPE = 2,       /* N is not m * 2^L (bt_build), m / d / H not supported */
+    BT_ERR_NONFINITE = 3,   /* a coordinate is NaN or infinite (found on the device) */
+    BT_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than *_workspace_size() */
+    BT_ERR_CUDA = 5,        /* a CUDA runtime call failed */
+    BT_ERR_TIMEOUT = 6,     /* an inter-block wait gave up (found on the device) */
+    BT_ERR_UNSUPPORTED = 7, /* a valid request this build does not handle */
+    BT_ERR_INTERNAL = 8     /* a consistency check inside a kernel failed (found on the device);
+                               the output of that call is not valid */
+} bt_status;
+
+typedef enum { BT_F32 = 0, BT_BF16 = 1 } bt_dtype;
+
+/* Largest batch (number of clouds) one segmented build accepts. */
+#define BT_MAX_CLOUDS 64
+
+/* Library version as 10000*major + 100*minor + patch. */
+int32_t bt_version(void);
+
+/*
+ * Workspace bytes for a (segmented) build of B clouds with ball size m.
+ *   offsets  host int64 [B+1]: cloud b is rows offsets[b] .. offsets[b+1]-1.
+ * Returns 0 for invalid arguments.  The same workspace may be reused by any
+ * later build whose workspace size is not larger; one workspace must not be
+ * used by two builds in flight at the same time.
+ */
+size_t bt_build_workspace_size(const int64_t *offsets, int32_t B, int32_t m);
+
+/*
+ * Ball tree of one cloud [E6][E9][E15].
+ *   coords  float [N, 3]
+ *   N       number of points; must equal m * 2^L for some L >= 0
+ *           (otherwise BT_ERR_SHAPE; padding is bt_build_segmented's job)
+ *   m       leaf (ball) size, 1 <= m <= 1024
+ *   perm    int32 [N] out: perm[slot] = row of the point stored in that slot.
+ *           Ball b is slots b*m .. b*m+m-1; a node of level l is a run of
+ *           N/2^l consecutive slots.
+ *   ws      workspace of at least bt_build_workspace_size({0,N}, 1, m) bytes,
+ *           256-byte aligned
+ */
+bt_status bt_build(const float *coords, int64_t N, int32_t m, int32_t *perm, void *ws, size_t ws_bytes,
+                   void *stream);
+
+/*
+ * Ball trees of a batch of clouds of any sizes [E6][E9].  Cloud b (n_b points)
+ * is padded with dummy points to Npad_b = m * 2^ceil(log2(ceil(n_b/m))) slots;
+ * a dummy is keyed above every real point on every axis, never counts in an
+ * extent, and so ends in the rightmost slots of its cloud.
+ *   coords      float [offsets[B], 3], clouds concatenated
+ *   offsets     host int64 [B+1], strictly increasing, offsets[0] = 0
+ *   B           1 <= B <= BT_MAX_CLOUDS
+ *   perm        int32 [sum Npad_b] out: cloud b owns slots pad[b]..pad[b+1]-1;
+ *               perm[slot] = global row (offsets[b] + index in cloud), or -1
+ *               for a dummy slot
+ *   pad_offsets host int64 [B+1] out (may be NULL): the slot offsets pad[b]
+ */
+bt_status bt_build_segmented(const float *coords, const int64_t *offsets, int32_t B, int32_t m, int32_t *perm,
+                             int64_t *pad_offsets, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Device-side status of the last build that used `ws`: synchronises `stream`,
+ * returns BT_OK, BT_ERR_NONFINITE, BT_ERR_TIMEOUT or BT_ERR_INTERNAL (or
+ * BT_ERR_CUDA).
+ */
+bt_status bt_build_device_status(const void *ws, void *stream);
+
+/*
+ * Rotation by 45 degrees counter-clockwise about +z through the origin [ROT],
+ * in float with each product and sum rounded separately (no FMA):
+ *   x' = c*x - s*y,  y' = s*x + c*y,  z' = z,  c = s = float(sqrt(1/2)).
+ *   in, out  float [N, 3]; may be the same buffer.
+ */
+bt_status bt_rotate_z(const float *in, int64_t N, float *out, void *stream);
+
+/*
+ * Inverse of a tree permutation [E9]: inv[perm[s]] = s for every real slot.
+ *   perm    int32 [npad] (dummies -1); its real slots must hold every row
+ *           0..n_rows-1 exactly once (as bt_build* produces)
+ *   inv     int32 [n_rows] out
+ */
+bt_status bt_invert_perm(const int32_t *perm, int64_t npad, int64_t n_rows, int32_t *inv, void *stream);
+
+/*
+ * Slot map between two trees of the same points [ROT][E9]:
+ *   map[s] = invA[permB[s]] (or -1 where permB[s] < 0), so that rows held in
+ *   tree-A slot order move to tree-B slot order by Y[s] = X[map[s]].
+ *   invA int32 [rows], permB int32 [npad], map int32 [npad] out
+ */
+bt_status bt_compose(const int32_t *invA, const int32_t *permB, int64_t npad, int32_t *map, void *stream);
+
+/*
+ * Row gather into tree order [E9]: Y[s] = X[idx[s]] for idx[s] >= 0, a zero
+ * row where idx[s] < 0.  Rows are row_bytes bytes (1 <= row_bytes <= 65536).
+ *   X  [rows, row_bytes] (idx values must be < rows), Y [npad, row_bytes] out
+ */
+bt_status bt_gather(const void *X, const int32_t *idx, int64_t npad, int32_t row_bytes, void *Y, void *stream);
+
+/*
+ * Row scatter back to the original order [E9]: X[idx[s]] = Y[s] for
+ * idx[s] >= 0; slots with idx[s] < 0 are dropped.  Real idx values must be
+ * distinct.
+ */
+bt_status bt_scatter(const void *Y, const int32_t *idx, int64_t npad, int32_t row_bytes, void *X, void *stream);
+
+/*
+ * Ball Tree Attention [E7][ABS]: for every ball b (slots b*m .. b*m+m-1) and
+ * head h, every real query row i of the ball gets
+ *     O[i,h,:] = sum_j softmax_j(Q[i,h,:] . K[j,h,:] / sqrt(d)) V[j,h,:]
+ * over the real rows j of the same ball.  No bias, no positional term.
+ *   Q, K, V  [rows, H, d] of dtype dt (BT_F32: float, BT_BF16: bfloat16)
+ *   perm     int32 [npad] slot -> row (dummy slots -1: neither query nor
+ *            key, nothing written), or NULL: row s sits in slot s (rows =
+ *            npad, no dummies).  Gathering by perm and scattering O back is
+ *            fused into the attention kernel.
+ *   npad     number of slots, a multiple of m
+ *   m        1 <= m <= 256;  H >= 1;  d in {32, 64}
+ *   O        [rows, H, d] out, dtype dt, original row order
+ * Accumulation and softmax are in float.  BT_BF16 with m dividing 128 runs on
+ * the tcgen05 tensor cores; other shapes run on the CUDA cores.
+ */
+bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
+                            int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream);
+
+/*
+ * Device-side status of the attention kernels on the current device:
+ * synchronises `stream`, returns BT_OK or BT_ERR_TIMEOUT (a tensor-core
+ * completion wait that gave up) and clears the recorded code.
+ */
+bt_status bt_attention_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BTS_H */

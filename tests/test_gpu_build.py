@@ -1,0 +1,160 @@
+"""GPU parity of the tree build, rotation and slot maps against the oracle (bit-exact)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from treecheck import check_tree, padded
+
+pytestmark = pytest.mark.gpu
+
+bts = pytest.importorskip("ball_tree_sparse_b200")
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _gpu_build(coords, m, offsets=None):
+    n = coords.shape[0]
+    c = _dev(coords)
+    if offsets is None:
+        ws = bts.workspace([0, n], m)
+        perm = bts.bt_build(c, m, ws=ws)
+    else:
+        ws = bts.workspace(offsets, m)
+        perm, _ = bts.bt_build_segmented(c, offsets, m, ws=ws)
+    assert bts.bt_build_device_status(ws) == 0
+    return perm.cpu().numpy()
+
+
+SINGLE = [
+    # (n, m, kind): tail only, several wide levels, many tiles per node, odd m, m = 1
+    (1024, 32, "uniform"),
+    (32 * 2 ** 9, 32, "uniform"),
+    (32 * 2 ** 9, 32, "tied"),
+    (128 * 2 ** 10, 128, "uniform"),
+    (3 * 2 ** 12, 3, "tied"),
+    (2 ** 13, 1, "tied"),
+    (7 * 2 ** 11, 7, "uniform"),
+    (100 * 2 ** 7, 100, "signed"),
+    (128, 128, "uniform"),
+    (1, 1, "uniform"),
+    (1024 * 8, 1024, "uniform"),
+]
+
+
+def _points(n, kind, seed):
+    if kind == "uniform":
+        return workloads.uniform_cloud(n, seed)
+    if kind == "tied":
+        return workloads.tied_cloud(n, seed, levels=6)
+    sign = np.where(workloads.tied_cloud(n, seed + 1, levels=2) > 0, -1, 1).astype(np.float32)
+    return workloads.tied_cloud(n, seed, levels=3) * sign
+
+
+@pytest.mark.parametrize("n,m,kind", SINGLE)
+def test_build_single_bit_exact(orc, n, m, kind):
+    pts = _points(n, kind, n + m)
+    want, _ = orc.build(pts, m)
+    got = _gpu_build(pts, m)
+    assert np.array_equal(got, want)
+    if n <= 1 << 15:
+        check_tree(got, pts, m)
+
+
+@pytest.mark.parametrize("sizes,m", [([1, 5, 100, 3000, 40000], 128), ([17, 4096, 4097, 300], 16),
+                                     ([2000] * 8, 1), ([5, 1, 9], 4)])
+def test_build_segmented_bit_exact(orc, sizes, m):
+    pts = np.concatenate([workloads.tied_cloud(s, 70 + i, levels=9) for i, s in enumerate(sizes)])
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    want, pad = orc.build(pts, m, offsets)
+    got = _gpu_build(pts, m, offsets)
+    assert np.array_equal(got, want)
+    check_tree(got, pts, m, offsets)
+
+
+def test_workload_tiny(orc):
+    wl = workloads.tiny()
+    assert np.array_equal(_gpu_build(wl.coords, wl.m), orc.build(wl.coords, wl.m)[0])
+
+
+def test_workload_gauss_mix_both_trees(orc):
+    wl = workloads.gauss_mix()
+    got = _gpu_build(wl.coords, wl.m, wl.offsets)
+    assert np.array_equal(got, orc.build(wl.coords, wl.m, wl.offsets)[0])
+    rot = bts.bt_rotate_z(_dev(wl.coords)).cpu().numpy()
+    assert np.array_equal(rot.view(np.uint32), orc.rotate_z(wl.coords).view(np.uint32))
+    got_b = _gpu_build(rot, wl.m, wl.offsets)
+    assert np.array_equal(got_b, orc.build(rot, wl.m, wl.offsets)[0])
+
+
+def test_workload_ellipsoid(orc):
+    wl = workloads.ellipsoid()
+    assert np.array_equal(_gpu_build(wl.coords, wl.m), orc.build(wl.coords, wl.m)[0])
+
+
+def test_workload_box_cluster_full_size(orc):
+    wl = workloads.box_cluster(with_qkv=False)
+    got = _gpu_build(wl.coords, wl.m)
+    assert np.array_equal(got, orc.build(wl.coords, wl.m)[0])
+    rot = orc.rotate_z(wl.coords)
+    assert np.array_equal(bts.bt_rotate_z(_dev(wl.coords)).cpu().numpy().view(np.uint32), rot.view(np.uint32))
+    assert np.array_equal(_gpu_build(rot, wl.m), orc.build(rot, wl.m)[0])
+
+
+def test_workload_ragged_full_size(orc):
+    wl = workloads.ragged()
+    got = _gpu_build(wl.coords, wl.m, wl.offsets)
+    want, pad = orc.build(wl.coords, wl.m, wl.offsets)
+    assert np.array_equal(got, want)
+    assert np.array_equal(pad, wl.pad_offsets())
+
+
+def test_repeat_and_reuse_workspace(orc):
+    # one workspace reused by a smaller build and by the same build twice in a row
+    big = workloads.uniform_cloud(128 * 2 ** 8, 1)
+    small = workloads.tied_cloud(128 * 2 ** 5, 2, levels=4)
+    ws = bts.workspace([0, len(big)], 128)
+    for pts in (big, small, big):
+        perm = bts.bt_build(_dev(pts), 128, ws=ws).cpu().numpy()
+        assert bts.bt_build_device_status(ws) == 0
+        assert np.array_equal(perm, orc.build(pts, 128)[0])
+
+
+def test_rotate_bit_exact_special_values(orc):
+    pts = np.array([[1, 0, 0], [0, 1, 0], [-0.0, -0.0, 3], [1e-40, -1e-40, 0], [3e38, 3e38, -1],
+                    [-2.5, 7.25, 1e-3]], np.float32)
+    pts = np.concatenate([pts, (workloads.uniform_cloud(5000, 4) - 0.5) * 100])
+    got = bts.bt_rotate_z(_dev(pts)).cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), orc.rotate_z(pts).view(np.uint32))
+
+
+def test_invert_compose_bit_exact(orc):
+    wl = workloads.ragged(batch=3, n_min=300, n_max=3000)
+    pa = _gpu_build(wl.coords, wl.m, wl.offsets)
+    rot = orc.rotate_z(wl.coords)
+    pb = _gpu_build(rot, wl.m, wl.offsets)
+    n = wl.n_total
+    inv = bts.bt_invert_perm(_dev(pa), n).cpu().numpy()
+    assert np.array_equal(inv, orc.invert(pa, n))
+    mp = bts.bt_compose(_dev(inv), _dev(pb)).cpu().numpy()
+    assert np.array_equal(mp, orc.compose(inv, pb))
+
+
+def test_gather_scatter_exact():
+    g = np.random.Generator(np.random.PCG64(3))
+    n, npad = 1000, 1024
+    perm = np.full(npad, -1, np.int32)
+    perm[g.permutation(npad)[:n]] = np.arange(n, dtype=np.int32)
+    for shape, dt in (((n, 8, 32), torch.bfloat16), ((n, 2, 32), torch.float32), ((n, 3), torch.float32),
+                      ((n, 5), torch.uint8)):
+        X = (torch.randn(shape, generator=torch.Generator().manual_seed(1)) * 10).to(dt).cuda()
+        Y = bts.bt_gather(X, _dev(perm))
+        Xc, Yc = X.cpu(), Y.cpu()
+        for s in range(npad):
+            want = Xc[perm[s]] if perm[s] >= 0 else torch.zeros_like(Xc[0])
+            assert torch.equal(Yc[s], want)
+        Z = torch.zeros_like(X)
+        bts.bt_scatter(Y, _dev(perm), Z)
+        assert torch.equal(Z.cpu(), Xc)
