@@ -49,6 +49,7 @@ def test_segmented_argument_errors():
     for offsets in ([0, 5, 5, 10], [1, 10], [0, 11, 10]):
         with pytest.raises(bts.BtsError):
             bts.bt_build_segmented(c, offsets, 4)
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
     with pytest.raises(bts.BtsError) as e:
-        bts.bt_build_segmented(c, list(range(0, 66)), 1)  # 65 clouds
+        bts.bt_build_segmented(c, list(range(0, 66)), 1, ws=ws)  # 65 clouds
     assert e.value.status == "BT_ERR_UNSUPPORTED"
