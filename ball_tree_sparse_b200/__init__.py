@@ -36,6 +36,7 @@ _SIGS = {
     "bt_build": ([_P, _i64, _i32, _P, _P, _sz, _P], ctypes.c_int),
     "bt_build_segmented": ([_P, _P, _i32, _i32, _P, _P, _P, _sz, _P], ctypes.c_int),
     "bt_build_device_status": ([_P, _P], ctypes.c_int),
+    "bt_build_noalloc": ([_P, _i64, _i32, _P, _P, _P], ctypes.c_int),
     "bt_rotate_z": ([_P, _i64, _P, _P], ctypes.c_int),
     "bt_invert_perm": ([_P, _i64, _i64, _P, _P], ctypes.c_int),
     "bt_compose": ([_P, _P, _i64, _P, _P], ctypes.c_int),
@@ -135,6 +136,14 @@ def bt_build_segmented(coords: torch.Tensor, offsets, m: int, perm: torch.Tensor
 def _padded(n: int, m: int) -> int:
     leaves = max(1, -(-n // m))
     return m * (1 << (leaves - 1).bit_length())
+
+
+def bt_build_noalloc(coords: torch.Tensor, m: int, perm: torch.Tensor, status: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """bt_build with the library's own static scratch (N <= 65,536); allocates nothing."""
+    _check("bt_build_noalloc", _lib.bt_build_noalloc(_dptr(coords), coords.shape[0], m, _dptr(perm),
+                                                     _dptr(status), _stream(stream)))
+    return perm
 
 
 def bt_build_device_status(ws: torch.Tensor, stream=None) -> int:

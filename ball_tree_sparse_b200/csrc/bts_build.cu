@@ -655,3 +655,57 @@ extern "C" bt_status bt_build_device_status(const void *ws, void *stream)
     if (cudaStreamSynchronize(st) != cudaSuccess) return BT_ERR_CUDA;
     return static_cast<bt_status>(h);
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of bt_build.
+//
+// Some callers cannot allocate device memory at the point where they build a
+// tree: code inside a region being captured into a CUDA graph (where a
+// cudaMalloc would break or end the capture), plug-ins hosted by a framework
+// that owns every device allocation through its own pool, and real-time hosts
+// that fix their memory budget at start-up.  For them this entry point takes
+// its scratch from one file-scope device array of kStaticWsBytes (8 MiB) that
+// every GPU which loads this library holds until the process exits, instead
+// of a caller workspace.  It serves clouds of at most kStaticMaxPoints points.
+//
+// The array is shared by every call on a device and keeps the last call's
+// contents; each call clears the part that must start at zero.  Two calls
+// whose work overlaps on the GPU (different streams, or host threads racing)
+// race on the array and produce garbage: serialise them.
+// ---------------------------------------------------------------------------
+namespace bts {
+constexpr size_t kStaticWsBytes = size_t(8) << 20;
+constexpr int64_t kStaticMaxPoints = 65536;
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+static void *g_static_ws_addr[64] = {};  // device address of g_static_ws, per device ordinal
+}  // namespace bts
+
+extern "C" bt_status bt_build_noalloc(const float *coords, int64_t N, int32_t m, int32_t *perm, int32_t *status_out,
+                                      void *stream)
+{
+    if (!coords || !perm || N < 1) return BT_ERR_ARG;
+    if (m < 1 || m > 1024 || N % m) return BT_ERR_SHAPE;
+    const int64_t leaves = N / m;
+    if (leaves & (leaves - 1)) return BT_ERR_SHAPE;
+    if (N > kStaticMaxPoints) return BT_ERR_UNSUPPORTED;  // beyond the static scratch
+    const int64_t offsets[2] = {0, N};
+    Plan P;
+    bt_status s = make_plan(offsets, 1, m, P);
+    if (s != BT_OK) return s;
+    if (make_layout(P).total > kStaticWsBytes) return BT_ERR_UNSUPPORTED;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BT_ERR_CUDA;
+    if (!g_static_ws_addr[dev]) {
+        // host code only sees a stand-in for the array: ask the runtime for its device address
+        void *addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_static_ws) != cudaSuccess || !addr) return BT_ERR_CUDA;
+        g_static_ws_addr[dev] = addr;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = launch_build(coords, P, perm, g_static_ws_addr[dev], kStaticWsBytes, st);
+    if (s == BT_OK && status_out &&
+        cudaMemcpyAsync(status_out, g_static_ws_addr[dev], sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+            cudaSuccess)
+        return BT_ERR_CUDA;
+    return s;
+}

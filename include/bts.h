@@ -107,6 +107,25 @@ bt_status bt_build_segmented(const float *coords, const int64_t *offsets, int32_
                              int64_t *pad_offsets, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * bt_build without a caller workspace, for callers that cannot allocate
+ * device memory when they build a tree: code inside a region being captured
+ * into a CUDA graph, plug-ins whose host framework owns every device
+ * allocation, real-time hosts with a memory budget fixed at start-up.  The
+ * pages have no counterpart; this is a deployment variant of bt_build.
+ *   coords, N, m, perm  as for bt_build; N <= 65,536 (else BT_ERR_UNSUPPORTED,
+ *                       returned before anything is enqueued)
+ *   status_out          device int32 (may be NULL): receives, in stream order,
+ *                       the device-side status (BT_OK, BT_ERR_NONFINITE, ...)
+ * Scratch is one 8 MiB array inside the library, held on every GPU that
+ * loads it until the process exits, and shared by all calls on that device:
+ * calls whose work overlaps on the GPU race and must be serialised.  The
+ * first call on each device looks up the array's device address; make that
+ * first call before any stream capture.  Allocates nothing.
+ */
+bt_status bt_build_noalloc(const float *coords, int64_t N, int32_t m, int32_t *perm, int32_t *status_out,
+                           void *stream);
+
+/*
  * Device-side status of the last build that used `ws`: synchronises `stream`,
  * returns BT_OK, BT_ERR_NONFINITE, BT_ERR_TIMEOUT or BT_ERR_INTERNAL (or
  * BT_ERR_CUDA).
