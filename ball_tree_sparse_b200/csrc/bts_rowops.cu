@@ -1,6 +1,6 @@
 // Element- and row-wise kernels around the tree: the 45-degree rotation for the
-// rotated-tree layers (author's thread: "instead of shifting windows, we
-// rotate trees"), inverse / composed slot maps, and row gather / scatter into
+// rotated-tree layers (author's thread: cross-partition exchange comes from
+// rotating the tree, the counterpart of Swin's window shift), inverse / composed slot maps, and row gather / scatter into
 // and out of tree order (thread post 9/N: a ball's points are contiguous).
 // All of them are HBM-bound streams; each thread moves 16-byte vectors where
 // the layout allows.

@@ -5,16 +5,16 @@
  * Sources (page title, then place on the page):
  *  [E6]  "Erwin: A Tree-based Hierarchical Transformer for Large-scale Physical
  *        Systems", author's thread, post 6/N: a ball tree recursively
- *        partitions points into nested sets of similar size, each covered by
- *        a ball.
+ *        divides the points into nested groups of about equal size, each
+ *        enclosed by a ball.
  *  [E7]  same thread, post 7/N: pick a tree level and compute attention
  *        within every ball of it in parallel (Ball Tree Attention).
  *  [E9]  same thread, post 9/N: at every level the points of one ball are
- *        stored next to each other, so ball operations are views.
+ *        kept contiguous in memory, so ball operations are views.
  *  [E15] same thread, post 15/N: the tree construction is a native,
  *        parallel component.
- *  [ROT] thread post on cross-ball exchange: instead of shifting windows
- *        (Swin), the tree is rotated.
+ *  [ROT] thread post on cross-ball exchange: the tree is rotated, where
+ *        Swin would shift its windows.
  *  [ABS] PMLR abstract of the same paper: linear-time attention in
  *        fixed-size neighbourhoods of a ball tree partition.
  *

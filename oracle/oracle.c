@@ -10,15 +10,16 @@
  * What it follows (page titles as the sources give them):
  *  - "Erwin: A Tree-based Hierarchical Transformer for Large-scale Physical
  *    Systems" (bluesky thread, posts 6/N and 9/N; PMLR abstract): a ball tree
- *    recursively splits the points into nested sets of similar size, each
- *    covered by a ball; at every level the points of one ball are stored next
- *    to each other.  The split rule used here (median of the axis of largest
- *    extent, ties by original index, leaves in index order) is the reading
- *    stated in the accompanying design notes; the pages do not print it.
+ *    recursively divides the points into nested groups of about equal size, each
+ *    covered by a ball; at every level a ball's points are contiguous.  The
+ *    pages do not print a split rule; this oracle takes the plainest one:
+ *    median of the axis of largest extent, ties by original index, leaves in
+ *    index order.
  *  - same thread, post 7/N: ball tree attention is scaled dot-product
  *    attention computed independently inside every ball of one tree level.
- *  - thread post "instead of shifting windows, we rotate trees": the rotated
- *    layer rebuilds the tree on rotated coordinates (45 degrees about +z here).
+ *  - thread post on cross-partition exchange (the tree is rotated where Swin
+ *    would shift its windows): the rotated layer rebuilds the tree on rotated
+ *    coordinates (45 degrees about +z here).
  */
 #include <math.h>
 #include <stdint.h>
