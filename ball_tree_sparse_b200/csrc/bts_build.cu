@@ -27,12 +27,15 @@
 
 namespace bts {
 
-constexpr int kSortTile = 4096;
-constexpr int kSortThreads = 512;
-constexpr int kLevelThreads = 512;
-constexpr int kLevelTileMax = 2048;
-constexpr int kTailThreads = 1024;
-constexpr int kTailMax = 4096;
+constexpr int kSortTile = 1024;      // keys per radix tile
+constexpr int kSortThreads = 256;
+constexpr int kLevelThreads = 128;
+constexpr int kLevelTileTarget = 512;  // slots per list per wide-level tile (m * 2^k, or m when m > 512)
+constexpr int kLevelTileMax = 1024;
+constexpr int kLevelEpt = kLevelTileMax / kLevelThreads;
+constexpr int kTailMax = 4096;         // largest node finished in shared memory
+constexpr int kTailMin = 512;          // smallest tail node (for m <= 512)
+constexpr int kTailCtasWanted = 2 * 148;  // aim for two tail CTAs per SM
 constexpr int kCounterLevel0 = 8;
 
 struct Plan {
@@ -76,9 +79,26 @@ static bt_status make_plan(const int64_t *offsets, int32_t B, int32_t m, Plan &P
     std::memset(&P, 0, sizeof(P));
     P.B = B;
     P.m = m;
-    P.T = m << ilog2(kTailMax / m);
-    P.TP = m << ilog2(kLevelTileMax / m);
+    P.TP = m <= kLevelTileTarget ? (m << ilog2(kLevelTileTarget / m)) : m;
+    int64_t npad_all = 0;
+    for (int b = 0; b < B; ++b) {
+        const int64_t n = offsets[b + 1] - offsets[b];
+        if (n < 1) return BT_ERR_ARG;
+        npad_all += padded_size(n, m);
+    }
+    // tail node size T = m * 2^t: small enough that the tail runs on about kTailCtasWanted CTAs
+    // when the batch is large, but never below max(4m, 512) slots (each wide level is a launch,
+    // so tiny batches keep their levels in shared memory) and never above kTailMax
+    {
+        const int tmax = ilog2(kTailMax / m);
+        const int tmin = std::min(tmax, std::max(2, m <= kTailMin ? ilog2(kTailMin / m) : 0));
+        int t = npad_all >= int64_t(kTailCtasWanted) * m ? ilog2(npad_all / (int64_t(kTailCtasWanted) * m)) : 0;
+        t = std::max(std::min(t, tmax), tmin);
+        P.T = m << t;
+    }
     const int t = ilog2(P.T / m);
+    // every wide node has at least 2T slots: a wide-level tile must not be larger
+    P.TP = std::min(P.TP, 2 * P.T);
     int64_t pad = 0;
     int32_t st = 0, tt = 0, nlev = 0;
     for (int b = 0; b < B; ++b) {
@@ -104,6 +124,13 @@ static bt_status make_plan(const int64_t *offsets, int32_t B, int32_t m, Plan &P
     P.nlev = nlev;
     P.npad = pad;
     if (pad > (int64_t(1) << 30) || offsets[B] > (int64_t(1) << 30)) return BT_ERR_UNSUPPORTED;
+    // invariants the kernels rely on: every wide node splits into whole tiles, tails fit shared memory
+    for (int b = 0; b < B; ++b)
+        for (int lev = 0; lev < P.glev[b]; ++lev) {
+            const int64_t sn = (P.pad[b + 1] - P.pad[b]) >> lev;
+            if (sn <= P.T || sn % P.TP || sn / P.TP < 1) return BT_ERR_INTERNAL;
+        }
+    if (P.TP > kLevelTileMax || P.T > kTailMax || P.T < m || (P.T & 1)) return BT_ERR_INTERNAL;
     return BT_OK;
 }
 
@@ -141,7 +168,6 @@ __global__ void __launch_bounds__(kSortThreads) k_init(Plan P, const float *__re
     const int k = r - P.sort_tile0[b];
     const int64_t base = P.pad[b] + int64_t(k) * kSortTile;
     const int cnt = int(min64(kSortTile, P.pad[b + 1] - base));
-    const uint32_t lt = (1u << lane) - 1u;
     for (int e0 = 0; e0 < kSortTile; e0 += kSortThreads) {
         const int e = e0 + tid;
         const bool ok = e < cnt;
@@ -160,13 +186,19 @@ __global__ void __launch_bounds__(kSortThreads) k_init(Plan P, const float *__re
             if (ok) keys[int64_t(a) * P.npad + pid] = key[a];
         }
         if (ok) ilist[pid] = uint32_t(pid);
+        const bool full = __all_sync(0xffffffffu, ok);
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-                const uint32_t d = ok ? ((key[a] >> (8 * p)) & 255u) : (256u + lane);
-                const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                if (ok && (peers & lt) == 0u) atomicAdd(&sh[(a * 4 + p) * 256 + d], __popc(peers));
+                const uint32_t d = (key[a] >> (8 * p)) & 255u;
+                // high bytes are usually equal across a warp: one atomic instead of 32 colliding ones
+                const uint32_t d0 = __shfl_sync(0xffffffffu, d, 0);
+                if (full && __all_sync(0xffffffffu, d == d0)) {
+                    if (lane == 0) atomicAdd(&sh[(a * 4 + p) * 256 + d], 32u);
+                } else if (ok) {
+                    atomicAdd(&sh[(a * 4 + p) * 256 + d], 1u);
+                }
             }
         }
     }
@@ -283,17 +315,22 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
 // ---------------------------------------------------------------------------
 // 3. one wide level: split every node larger than T at the median of its widest axis
 // ---------------------------------------------------------------------------
+// (key, id) < (pivot key, pivot id): the composite order that makes every key distinct
+__device__ __forceinline__ bool before(uint32_t key, uint32_t id, uint32_t pkey, uint32_t pid)
+{
+    return key < pkey || (key == pkey && id < pid);
+}
+
 __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const uint32_t *__restrict__ keys,
                                                          const uint32_t *__restrict__ lin, uint32_t *__restrict__ lout,
                                                          uint32_t *lst, uint32_t *counters, uint32_t *status)
 {
-    constexpr int NT = kLevelThreads;
+    constexpr int NT = kLevelThreads, EPT = kLevelEpt;
     __shared__ uint32_t sl[4][kLevelTileMax];
     __shared__ unsigned long long scratch[NT / 32 + 1];
-    __shared__ uint32_t s_tile, s_excl[4];
+    __shared__ uint32_t s_tile, s_excl[4], s_pkey, s_pid;
     __shared__ int s_axis;
     __shared__ float s_ext[3];
-    __shared__ unsigned long long s_piv;
     const int tid = threadIdx.x;
     if (tid == 0) s_tile = atomicAdd(&counters[kCounterLevel0 + lev], 1u);
     __syncthreads();
@@ -310,7 +347,12 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
         ++b;
     }
     const int64_t s = (P.pad[b + 1] - P.pad[b]) >> lev, half = s >> 1;
-    const int64_t tps = s / TP, kseg = r / tps;
+    const int64_t tps = s / TP;
+    if (tps < 1) {  // cannot happen for a valid plan; never divide by zero or index out of the lists
+        if (tid == 0) record_error(status, BT_ERR_INTERNAL);
+        return;
+    }
+    const int64_t kseg = r / tps;
     const int j = int(r - kseg * tps);
     const int64_t seg = P.pad[b] + kseg * s;
     const int64_t nreal = max64(0, min64(s, P.n[b] - kseg * s));
@@ -329,33 +371,31 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
         if (s_ext[2] > s_ext[ax]) ax = 2;
         const uint32_t pp = lin[ax * np + seg + half];
         s_axis = ax;
-        s_piv = (static_cast<unsigned long long>(keys[ax * np + pp]) << 32) | pp;
+        s_pid = pp;
+        s_pkey = keys[ax * np + pp];
     }
     const int64_t tile0 = seg + int64_t(j) * TP;
     for (int l = 0; l < 4; ++l)
         for (int i = tid; i < TP; i += NT) sl[l][i] = lin[l * np + tile0 + i];
     __syncthreads();
     const int ax = s_axis;
-    const unsigned long long piv = s_piv;
-    const int EPT = (TP + NT - 1) / NT;
-    const int i0 = tid * EPT;
-    uint32_t v[4][4];
+    const uint32_t pkey = s_pkey, ppid = s_pid;
+    const uint32_t *kax = keys + ax * np;
+    const int ept = (TP + NT - 1) / NT;
+    const int i0 = tid * ept;
+    uint32_t v[4][EPT];
     uint32_t lbits[4] = {0, 0, 0, 0};
     unsigned long long packed = 0;
 #pragma unroll
     for (int l = 0; l < 4; ++l) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < EPT; ++q) {
             const int i = i0 + q;
             v[l][q] = 0;
-            if (q < EPT && i < TP) {
+            if (q < ept && i < TP) {
                 const uint32_t pid = sl[l][i];
                 v[l][q] = pid;
-                bool left;
-                if (l == ax)
-                    left = int64_t(j) * TP + i < half;
-                else
-                    left = ((static_cast<unsigned long long>(keys[ax * np + pid]) << 32) | pid) < piv;
+                const bool left = (l == ax) ? int64_t(j) * TP + i < half : before(kax[pid], pid, pkey, ppid);
                 if (left) {
                     lbits[l] |= 1u << q;
                     packed += 1ull << (16 * l);
@@ -373,9 +413,9 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
         const int nl = int((tot >> (16 * l)) & 0xFFFFu);
         int run = int((ex >> (16 * l)) & 0xFFFFu);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < EPT; ++q) {
             const int i = i0 + q;
-            if (q < EPT && i < TP) {
+            if (q < ept && i < TP) {
                 const bool left = (lbits[l] >> q) & 1u;
                 const int pos = left ? run : nl + (i - run);
                 run += left;
@@ -400,34 +440,27 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
 }
 
 // ---------------------------------------------------------------------------
-// 4. the remaining levels of one node of at most T slots, in shared memory
+// 4. the remaining levels of one node of at most T slots, in shared memory.
+//    Points are renamed to local indices 0..sT-1 in ascending id order (the
+//    node's index list), so the index list itself is the identity and every
+//    list fits in 16 bits.  `loc` is a global scratch array pid -> local index.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ int find_local(const uint32_t *ps, int n, uint32_t pid)
+template <int NT>
+__global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict__ keys,
+                                             const uint32_t *__restrict__ lists, uint32_t *__restrict__ loc,
+                                             int32_t *__restrict__ perm, uint32_t *status)
 {
-    int lo = 0, hi = n - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (ps[mid] < pid)
-            lo = mid + 1;
-        else
-            hi = mid;
-    }
-    return lo;
-}
-
-__global__ void __launch_bounds__(kTailThreads) k_tail(Plan P, const uint32_t *__restrict__ keys,
-                                                       const uint32_t *__restrict__ lists, int32_t *__restrict__ perm,
-                                                       uint32_t *status)
-{
-    constexpr int NT = kTailThreads;
+    constexpr int EPT = 4;  // slots per thread: T <= 1024 runs with 256 threads, T <= 4096 with 1024
+    static_assert(kTailMax <= 1024 * EPT && 1024 <= 256 * EPT, "tail slots per thread");
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ unsigned long long scratch[NT / 32 + 1];
     const int T = P.T;
     uint32_t *ps = reinterpret_cast<uint32_t *>(dsm);            // [T] point ids, ascending
     uint32_t *k3 = ps + T;                                       // [3][T] keys by local index
-    unsigned long long *piv = reinterpret_cast<unsigned long long *>(k3 + 3 * T);  // [T/2]
-    unsigned long long *segpre = piv + T / 2;                    // [T/2]
-    uint16_t *lst = reinterpret_cast<uint16_t *>(segpre + T / 2);  // [2][4][T]
+    unsigned long long *segpre = reinterpret_cast<unsigned long long *>(k3 + 3 * T);  // [T/2]
+    uint32_t *pkey = reinterpret_cast<uint32_t *>(segpre + T / 2);  // [T/2] pivot keys
+    uint16_t *ppv = reinterpret_cast<uint16_t *>(pkey + T / 2);     // [T/2] pivot local index
+    uint16_t *lst = ppv + T / 2;                                 // [2][4][T]
     uint8_t *axs = reinterpret_cast<uint8_t *>(lst + 8 * T);     // [T/2]
 
     const int tid = threadIdx.x;
@@ -442,25 +475,33 @@ __global__ void __launch_bounds__(kTailThreads) k_tail(Plan P, const uint32_t *_
     const uint32_t *lin = lists + size_t(P.glev[b] & 1) * 4 * np;
     const int m = P.m;
 
-    for (int e = tid; e < sT; e += NT) ps[e] = lin[3 * np + seg + e];
-    __syncthreads();
     for (int e = tid; e < sT; e += NT) {
-        const uint32_t pid = ps[e];
+        const uint32_t pid = lin[3 * np + seg + e];
+        ps[e] = pid;
+        loc[pid] = uint32_t(e);
+#pragma unroll
+        for (int a = 0; a < 3; ++a) k3[a * T + e] = keys[a * np + pid];
+        lst[3 * T + e] = uint16_t(e);
+    }
+    __syncthreads();  // loc[] of this node is written (block-wide visibility of global stores)
+    for (int e = tid; e < sT; e += NT) {
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
-            k3[a * T + e] = keys[a * np + pid];
-            const uint32_t pid_a = lin[a * np + seg + e];
-            const int loc = find_local(ps, sT, pid_a);
-            if (ps[loc] != pid_a) record_error(status, BT_ERR_INTERNAL);  // lists disagree on the node's points
-            lst[a * T + e] = uint16_t(loc);
+            const uint32_t pid = lin[a * np + seg + e];
+            const uint32_t l = loc[pid];
+            if (l >= uint32_t(sT) || ps[l] != pid) {  // lists disagree on the node's points
+                record_error(status, BT_ERR_INTERNAL);
+                lst[a * T + e] = 0;
+            } else {
+                lst[a * T + e] = uint16_t(l);
+            }
         }
-        lst[3 * T + e] = uint16_t(e);
     }
     __syncthreads();
 
     int cur = 0;
-    const int EPT = (sT + NT - 1) / NT;
-    const int i0 = tid * EPT;
+    const int ept = (sT + NT - 1) / NT;
+    const int i0 = tid * ept;
     for (int sz = sT; sz > m; sz >>= 1) {
         const int half = sz >> 1, nsub = sT / sz;
         uint16_t *L = lst + cur * 4 * T, *Ln = lst + (cur ^ 1) * 4 * T;
@@ -479,59 +520,80 @@ __global__ void __launch_bounds__(kTailThreads) k_tail(Plan P, const uint32_t *_
             if (ext[2] > ext[ax]) ax = 2;
             const uint32_t pv = L[ax * T + start + half];
             axs[q] = uint8_t(ax);
-            piv[q] = (static_cast<unsigned long long>(k3[ax * T + pv]) << 32) | pv;
+            ppv[q] = uint16_t(pv);
+            pkey[q] = k3[ax * T + pv];
         }
         __syncthreads();
         uint32_t lbits[4] = {0, 0, 0, 0};
         unsigned long long packed = 0;
+        int sub = i0 / sz, sub_start = sub * sz;
+#pragma unroll
         for (int q = 0; q < EPT; ++q) {
             const int e = i0 + q;
-            if (e >= sT) break;
-            const int sub = e / sz;
-            const int ax = axs[sub];
-            const unsigned long long pv = piv[sub];
+            if (q < ept && e < sT) {
+                if (e - sub_start >= sz) {
+                    ++sub;
+                    sub_start += sz;
+                }
+                const int ax = axs[sub];
+                const uint32_t pk = pkey[sub], pv = ppv[sub];
+                const uint32_t *ka = k3 + ax * T;
 #pragma unroll
-            for (int l = 0; l < 4; ++l) {
-                const uint32_t v = L[l * T + e];
-                const bool left = (l == ax) ? (e - sub * sz) < half
-                                            : ((static_cast<unsigned long long>(k3[ax * T + v]) << 32) | v) < pv;
-                if (left) {
-                    lbits[l] |= 1u << q;
-                    packed += 1ull << (16 * l);
+                for (int l = 0; l < 4; ++l) {
+                    const uint32_t v = L[l * T + e];
+                    const bool left = (l == ax) ? (e - sub_start) < half : before(ka[v], v, pk, pv);
+                    if (left) {
+                        lbits[l] |= 1u << q;
+                        packed += 1ull << (16 * l);
+                    }
                 }
             }
         }
         const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, nullptr);
         {
             unsigned long long run = ex;
+            int sub2 = i0 / sz, st2 = sub2 * sz;
+#pragma unroll
             for (int q = 0; q < EPT; ++q) {
                 const int e = i0 + q;
-                if (e >= sT) break;
-                if (e % sz == 0) segpre[e / sz] = run;
+                if (q < ept && e < sT) {
+                    if (e - st2 >= sz) {
+                        ++sub2;
+                        st2 += sz;
+                    }
+                    if (e == st2) segpre[sub2] = run;
 #pragma unroll
-                for (int l = 0; l < 4; ++l)
-                    if ((lbits[l] >> q) & 1u) run += 1ull << (16 * l);
+                    for (int l = 0; l < 4; ++l)
+                        if ((lbits[l] >> q) & 1u) run += 1ull << (16 * l);
+                }
             }
         }
         __syncthreads();
         {
             unsigned long long run = ex;
+            int sub3 = i0 / sz, start = sub3 * sz;
+            unsigned long long sp = ept > 0 && i0 < sT ? segpre[sub3] : 0ull;
+#pragma unroll
             for (int q = 0; q < EPT; ++q) {
                 const int e = i0 + q;
-                if (e >= sT) break;
-                const int sub = e / sz, start = sub * sz;
-                const unsigned long long sp = segpre[sub];
-#pragma unroll
-                for (int l = 0; l < 4; ++l) {
-                    const int pre = int(((run >> (16 * l)) & 0xFFFFu) - ((sp >> (16 * l)) & 0xFFFFu));
-                    const bool left = (lbits[l] >> q) & 1u;
-                    const int dst = left ? start + pre : start + half + (e - start - pre);
-                    if ((left && pre >= half) || dst < start || dst >= start + sz) {
-                        record_error(status, BT_ERR_INTERNAL);  // never write outside the node
-                    } else {
-                        Ln[l * T + dst] = L[l * T + e];
+                if (q < ept && e < sT) {
+                    if (e - start >= sz) {
+                        ++sub3;
+                        start += sz;
+                        sp = segpre[sub3];
                     }
-                    if (left) run += 1ull << (16 * l);
+#pragma unroll
+                    for (int l = 0; l < 4; ++l) {
+                        const int pre = int(((run >> (16 * l)) & 0xFFFFu) - ((sp >> (16 * l)) & 0xFFFFu));
+                        const bool left = (lbits[l] >> q) & 1u;
+                        const int dst = left ? start + pre : start + half + (e - start - pre);
+                        if ((left && pre >= half) || dst < start || dst >= start + sz) {
+                            record_error(status, BT_ERR_INTERNAL);  // never write outside the node
+                        } else {
+                            Ln[l * T + dst] = L[l * T + e];
+                        }
+                        if (left) run += 1ull << (16 * l);
+                    }
                 }
             }
         }
@@ -548,7 +610,8 @@ __global__ void __launch_bounds__(kTailThreads) k_tail(Plan P, const uint32_t *_
 
 static size_t tail_smem_bytes(int T)
 {
-    return size_t(T) * 4 + size_t(3) * T * 4 + size_t(T / 2) * 8 * 2 + size_t(8) * T * 2 + size_t(T / 2);
+    // ps + k3 (16 B) + segpre (4 B) + pivot key (2 B) + pivot index (1 B) + lists (16 B) + axis (0.5 B) per slot
+    return size_t(T) * 16 + size_t(T / 2) * (8 + 4 + 2 + 1) + size_t(8) * T * 2 + 16;
 }
 
 static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm, void *ws, size_t ws_bytes,
@@ -580,7 +643,9 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
             cudaFuncSetAttribute(k_sort_pass<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
             cudaFuncSetAttribute(k_sort_pass<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
             cudaFuncSetAttribute(k_sort_pass<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
-            cudaFuncSetAttribute(k_tail, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(k_tail<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(tail_smem_bytes(1024))) ||
+            cudaFuncSetAttribute(k_tail<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(tail_smem_bytes(kTailMax))))
             return BT_ERR_CUDA;
         attrs_set[dev] = true;
@@ -605,7 +670,11 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
         uint32_t *lout = lists + size_t((lev + 1) & 1) * 4 * np;
         k_level<<<unsigned(tiles), kLevelThreads, 0, st>>>(P, lev, keys, lin, lout, lstat, counters, status);
     }
-    k_tail<<<P.tail0[P.B], kTailThreads, tail_smem, st>>>(P, keys, lists, perm, status);
+    // the sort buffers are dead after the last radix pass: reuse one as the pid -> local index map
+    if (P.T <= 1024)
+        k_tail<256><<<P.tail0[P.B], 256, tail_smem, st>>>(P, keys, lists, sk, perm, status);
+    else
+        k_tail<1024><<<P.tail0[P.B], 1024, tail_smem, st>>>(P, keys, lists, sk, perm, status);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 
