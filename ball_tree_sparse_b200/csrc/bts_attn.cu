@@ -4,13 +4,14 @@
 // tree slots, all balls and heads in parallel.
 //
 // Two kernels:
-//  - k_ball_attn_tc   bf16, m dividing 128: one CTA per (128-slot tile, head).
-//                     Q/K/V rows are gathered through perm with cp.async into
-//                     the no-swizzle canonical tensor-core layouts, S = QK^T
-//                     runs on tcgen05 (M=128, N=128) into TMEM, the softmax
-//                     reads S back with tcgen05.ld (one row per thread), writes
-//                     P (bf16, unnormalised) to shared memory, O = PV runs on
-//                     tcgen05 (N=d) into the TMEM columns S used, and the
+//  - k_ball_attn_tc2  bf16, m dividing 128: persistent CTAs over work items
+//                     (128-slot tile, head).  Q/K/V rows are gathered through
+//                     perm with cp.async into the no-swizzle canonical
+//                     tensor-core layouts, a few items ahead; S = QK^T runs on
+//                     tcgen05 (M=128, N=128) into TMEM, the softmax reads S back
+//                     with tcgen05.ld (one row per thread) and writes P (bf16,
+//                     unnormalised) to shared memory, O = PV and the row sums
+//                     (P times a ones column) run on tcgen05 into TMEM, and the
 //                     epilogue scales by 1/rowsum and scatters O through perm.
 //                     Balls smaller than 128 share a tile; keys of other balls
 //                     and dummy keys get weight 0.
@@ -185,178 +186,275 @@ __device__ __forceinline__ float ex2(float x)
 }
 
 constexpr int kTcThreads = 128;
-constexpr int kTcCols = 128;  // TMEM columns: S [128 x 128] f32; O reuses columns 0..d-1
 
+// ---------------------------------------------------------------------------
+// Persistent, pipelined tcgen05 kernel.  Each CTA walks work items
+// (128-slot tile, head) with heads fastest.  While item i computes, the Q/K/V
+// rows of the CTA's next item are in flight (cp.async, gathered through perm)
+// and the perm entries of the item after that are loading into registers.
+//   S = Q K^T          -> TMEM cols [0,128)            (tcgen05, M=128 N=128 K=d)
+//   softmax per row     (tcgen05.ld), P = exp2(...) as bf16 written back over
+//                       S: TMEM cols [0,64), two keys per column (tcgen05.st)
+//   O = P V            -> TMEM cols [64,64+d)          (A = P from TMEM)
+//   rowsum(P) = P e0   -> TMEM col 64+d                (B = a ones column)
+//   O / rowsum -> bf16 -> the query's row.
+// ---------------------------------------------------------------------------
 template <int D>
-__host__ __device__ constexpr size_t tc_smem_bytes()
+struct TcPipe {
+    static constexpr int NS = 2;                                // stages of Q/K/V
+    static constexpr uint32_t QK_BYTES = 128 * D * 2;           // one of Q or K
+    static constexpr uint32_t STAGE = 3 * QK_BYTES;             // Q, K, V of one item
+    static constexpr uint32_t ONES_OFF = NS * STAGE;
+    static constexpr uint32_t BYTES = ONES_OFF + 16 * 128 * 2;  // + ones operand (N=16, K=128)
+    static constexpr uint32_t COLS = D == 32 ? 128 : 256;       // S/P 128, O d, rowsum 16
+    static constexpr int PER_SM = D == 32 ? 4 : 2;              // CTAs per SM that TMEM and smem allow
+};
+
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t &r)
 {
-    // P (32 KB, aliased by Q and K before it is written) + V; padded so that at
-    // most four CTAs share an SM, which is what their TMEM columns allow.
-    return size_t(128 * 128 * 2 + D * 256) > size_t(50 * 1024) ? size_t(128 * 128 * 2 + D * 256)
-                                                                 : size_t(50 * 1024);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                            uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 4)
-    k_ball_attn_tc(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
-                   const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ perm, int64_t npad, int lm, int H,
-                   float sl2, __nv_bfloat16 *__restrict__ O)
+__global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
+    k_ball_attn_tc2(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+                    const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ perm, int64_t npad, int lm,
+                    int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O)
 {
-    constexpr int KCH = D / 8;                // 16-byte chunks per row of one head
-    constexpr uint32_t QK_SBO = KCH * 128;    // bytes between 8-row groups of Q and K
-    constexpr uint32_t P_SBO = 16 * 128;      // bytes between 8-row groups of P (128 keys)
-    constexpr uint32_t V_SBO = 16 * 128;      // bytes between 8-column groups of V (128 keys)
-    constexpr uint32_t V_OFF = 128 * 128 * 2;
+    using L = TcPipe<D>;
+    constexpr int KCH = D / 8;                 // 16-byte chunks per row of one head
+    constexpr int UPT = 128 * KCH / kTcThreads;  // 16-byte chunks per thread and tensor
+    constexpr uint32_t QK_SBO = KCH * 128;
+    constexpr uint32_t V_SBO = 16 * 128, ONES_SBO = 16 * 128;
     constexpr uint32_t IDESC_S = idesc_bf16(128, false);
     constexpr uint32_t IDESC_O = idesc_bf16(D, true);
+    constexpr uint32_t IDESC_SUM = idesc_bf16(16, false);
     extern __shared__ __align__(1024) uint8_t tsm[];
-    __shared__ int32_t sRow[128];
     __shared__ uint32_t sKeyMask[4];
-    __shared__ __align__(8) uint64_t sBar;
+    __shared__ __align__(8) uint64_t sBarS, sBarO;
     __shared__ uint32_t sTmem;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m = 1 << lm;
-    const int h = blockIdx.y;
-    const int64_t slot = int64_t(blockIdx.x) * 128 + tid;
-    uint8_t *sQ = tsm, *sK = tsm + D * 256, *sP = tsm, *sV = tsm + V_OFF;
+    const uint32_t base = smem_u32(tsm);
 
-    const int32_t row = slot < npad ? (perm ? perm[slot] : int32_t(slot)) : -1;
-    sRow[tid] = row;
-    const uint32_t vb = __ballot_sync(0xffffffffu, row >= 0);
-    if (lane == 0) sKeyMask[warp] = vb;
+    // the ones operand (K-major, N=16 x K=128): row 0 all 1.0, rows 1..15 zero
+    for (int i = tid; i < 16 * 128 * 2 / 16; i += kTcThreads) {
+        const int c = i >> 4, rr = i & 15;
+        const uint32_t off = (rr >> 3) * ONES_SBO + c * 128 + (rr & 7) * 16;
+        const uint32_t one = (rr == 0) ? 0x3F803F80u : 0u;
+        *reinterpret_cast<uint4 *>(tsm + L::ONES_OFF + off) = make_uint4(one, one, one, one);
+    }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sTmem)),
-                     "r"(kTcCols)
+                     "r"(L::COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBar)) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarS)) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarO)) : "memory");
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    __syncthreads();
-
-    // gather Q, K (K-major core matrices) and V (MN-major core matrices) of head h
-    for (int u = tid; u < 128 * KCH; u += kTcThreads) {
-        const int r = u / KCH, c = u - r * KCH;
-        const int32_t rr = sRow[r];
-        const size_t goff = rr >= 0 ? (size_t(rr) * H + h) * D + c * 8 : 0;
-        const uint32_t so = (r >> 3) * QK_SBO + c * 128 + (r & 7) * 16;
-        cp_async16(sQ + so, Q + goff, rr >= 0);
-        cp_async16(sK + so, K + goff, rr >= 0);
-        cp_async16(sV + c * V_SBO + r * 16, V + goff, rr >= 0);
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sTmem;
-    const uint32_t bar = smem_u32(&sBar);
+    const uint32_t tmem = sTmem, tS = tmem, tO = tmem + 64, tSum = tmem + 64 + D;
+    const uint32_t barS = smem_u32(&sBarS), barO = smem_u32(&sBarO);
+    const uint32_t lanebase = uint32_t(warp * 32) << 16;
 
-    // S = Q K^T  (M=128, N=128, K=D)
-    if (tid == 0) {
+    auto row_of = [&](int64_t item, int r) -> int32_t {
+        if (item >= items) return -1;
+        const int64_t slot = (item / H) * 128 + r;
+        return slot < npad ? (perm ? __ldg(perm + slot) : int32_t(slot)) : -1;
+    };
+    // rows whose chunks this thread copies: chunk u = tid + i*128 belongs to row u / KCH
+    auto load_rows = [&](int64_t item, int32_t (&rows)[UPT]) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-            mma_bf16(tmem, smem_desc(smem_u32(sQ) + kk * 256, 128, QK_SBO),
-                     smem_desc(smem_u32(sK) + kk * 256, 128, QK_SBO), IDESC_S, kk > 0);
-        mma_commit(bar);
-    }
-    bool ok = mbar_wait(bar, 0);
-    tc_fence_after();
-
-    // softmax of row tid over the keys of its ball
-    const int r = tid;
-    const int W = m >= 32 ? m : 32;
-    const int c0 = m >= 32 ? ((r >> lm) << lm) : warp * 32;
-    const uint32_t trow = tmem + (uint32_t(warp * 32) << 16);
-    float mx = -INFINITY;
-    for (int cc = c0; cc < c0 + W; cc += 32) {
-        uint32_t v[32];
-        tmem_ld32(trow + cc, v);
-        const uint32_t km = sKeyMask[cc >> 5];
+        for (int i = 0; i < UPT; ++i) rows[i] = row_of(item, (tid + i * kTcThreads) / KCH);
+    };
+    // gather Q, K (K-major core matrices) and V (MN-major core matrices) of one item into a stage
+    auto issue = [&](int64_t item, int stage, const int32_t (&rows)[UPT]) {
+        if (item < items) {
+            const int h = int(item % H);
+            uint8_t *sq = tsm + stage * L::STAGE, *sk = sq + L::QK_BYTES, *sv = sk + L::QK_BYTES;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const bool kv = ((km >> j) & 1u) && (((cc + j) >> lm) == (r >> lm));
-            if (kv) mx = fmaxf(mx, __uint_as_float(v[j]));
-        }
-    }
-    const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
-    float sum = 0.0f;
-    uint8_t *prow = sP + (r >> 3) * P_SBO + (r & 7) * 16;
-    // all reads of S by this warp are complete before P (aliasing Q/K) is written
-    for (int cc = 0; cc < 128; cc += 32) {
-        uint32_t pk[16];
-        if (cc >= c0 && cc < c0 + W) {
-            uint32_t v[32];
-            tmem_ld32(trow + cc, v);
-            const uint32_t km = sKeyMask[cc >> 5];
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                float p0 = 0.0f, p1 = 0.0f;
-                if (((km >> j) & 1u) && (((cc + j) >> lm) == (r >> lm)))
-                    p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-                if (((km >> (j + 1)) & 1u) && (((cc + j + 1) >> lm) == (r >> lm)))
-                    p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
-                const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                sum += __low2float(pb) + __high2float(pb);
-                pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+            for (int i = 0; i < UPT; ++i) {
+                const int u = tid + i * kTcThreads;
+                const int r = u / KCH, c = u - r * KCH;
+                const int32_t rr = rows[i];
+                const size_t goff = rr >= 0 ? (size_t(rr) * H + h) * D + c * 8 : 0;
+                const uint32_t so = (r >> 3) * QK_SBO + c * 128 + (r & 7) * 16;
+                cp_async16(sq + so, Q + goff, rr >= 0);
+                cp_async16(sk + so, K + goff, rr >= 0);
+                cp_async16(sv + c * V_SBO + r * 16, V + goff, rr >= 0);
             }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) pk[j] = 0u;
         }
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-            *reinterpret_cast<uint4 *>(prow + ((cc >> 3) + t) * 128) =
-                make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
 
-    // O = P V  (M=128, N=D, K=128); O overwrites TMEM columns 0..D-1
-    if (tid == 0 && ok) {
+    const int64_t first = blockIdx.x, stride = gridDim.x;
+    int32_t rows[UPT];
+    load_rows(first, rows);
+    issue(first, 0, rows);
+    load_rows(first + stride, rows);  // rows of the next item, used at the top of the loop
+    int32_t qcur = row_of(first, tid), qnext = row_of(first + stride, tid);
+    bool ok = true;
+    int it = 0;
+    for (int64_t item = first; item < items; item += stride, ++it) {
+        const int stage = it & 1;
+        issue(item + stride, stage ^ 1, rows);
+        load_rows(item + 2 * stride, rows);  // consumed one iteration later
+        const int32_t qafter = row_of(item + 2 * stride, tid);
+        const uint32_t kb = __ballot_sync(0xffffffffu, qcur >= 0);
+        if (lane == 0) sKeyMask[warp] = kb;
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t sq = base + stage * L::STAGE, sk = sq + L::QK_BYTES, sv = sk + L::QK_BYTES;
+        if (tid == 0 && ok) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            mma_bf16(tmem, smem_desc(smem_u32(sP) + kk * 256, 128, P_SBO),
-                     smem_desc(smem_u32(sV) + kk * 256, 128, V_SBO), IDESC_O, kk > 0);
-        mma_commit(bar);
-    }
-    ok = __syncthreads_and(ok);
-    if (ok) ok = mbar_wait(bar, 1);
-    tc_fence_after();
+            for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16(tS, smem_desc(sq + kk * 256, 128, QK_SBO), smem_desc(sk + kk * 256, 128, QK_SBO), IDESC_S,
+                         kk > 0);
+            mma_commit(barS);
+        }
+        ok = ok && mbar_wait(barS, it & 1);
+        tc_fence_after();
 
-    const int32_t qrow = sRow[r];
-    if (ok) {
-        const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+        // softmax of row tid; keys outside its ball or dummy get weight 0
+        const int ball0 = (tid >> lm) << lm;
+        uint32_t cmask[4];
 #pragma unroll
-        for (int c32 = 0; c32 < D; c32 += 32) {
-            uint32_t o[32];
-            tmem_ld32(trow + c32, o);
-            if (qrow >= 0) {
-                uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qrow) * H + h) * D + c32);
+        for (int c = 0; c < 4; ++c) {
+            uint32_t bm;  // keys of chunk c that lie in this row's ball
+            if (m >= 32)
+                bm = (c * 32 >= ball0 && c * 32 < ball0 + m) ? 0xffffffffu : 0u;
+            else
+                bm = (c * 32 <= ball0 && ball0 < c * 32 + 32) ? (((1u << m) - 1u) << (ball0 - c * 32)) : 0u;
+            cmask[c] = bm & sKeyMask[c];
+        }
+        float mx = -INFINITY;
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    uint32_t w[4];
+        for (int c = 0; c < 4; ++c) {
+            if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
+                uint32_t v[32];
+                tmem_ld32(tS + lanebase + c * 32, v);
+                if (cmask[c] == 0xffffffffu) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * t + 2 * e]) * inv,
-                                                                        __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
-                        w[e] = *reinterpret_cast<const uint32_t *>(&pb);
-                    }
-                    dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if ((cmask[c] >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]));
                 }
             }
         }
+        const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
+        // chunk c of S (cols 32c..32c+31) becomes P cols 16c..16c+15: every S column a P store
+        // overwrites has been read into registers by this thread before (its own TMEM lane)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+            if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
+                uint32_t v[32];
+                tmem_ld32(tS + lanebase + c * 32, v);
+                const uint32_t cm = cmask[c];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+                    float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
+                    if (cm != 0xffffffffu) {
+                        p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
+                        p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                    }
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                    pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pk[j] = 0u;
+            }
+            tmem_st16(tS + lanebase + c * 16, pk);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && ok) {
+            const uint32_t so1 = base + L::ONES_OFF;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16_ts(tO, tS + kk * 8, smem_desc(sv + kk * 256, 128, V_SBO), IDESC_O, kk > 0);
+                mma_bf16_ts(tSum, tS + kk * 8, smem_desc(so1 + kk * 256, 128, ONES_SBO), IDESC_SUM, kk > 0);
+            }
+            mma_commit(barO);
+        }
+        ok = ok && mbar_wait(barO, it & 1);
+        tc_fence_after();
+        if (ok) {
+            uint32_t sum_bits;
+            tmem_ld1(tSum + lanebase, sum_bits);
+            const float sum = __uint_as_float(sum_bits);
+            const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+            const int h = int(item % H);
+#pragma unroll
+            for (int c32 = 0; c32 < D; c32 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + lanebase + c32, o);
+                if (qcur >= 0) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qcur) * H + h) * D + c32);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 pb = __floats2bfloat162_rn(
+                                __uint_as_float(o[8 * t + 2 * e]) * inv, __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
+                            w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                        }
+                        dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+        }
+        qcur = qnext;
+        qnext = qafter;
+        tc_fence_before();
+        __syncthreads();  // every read of S/P, O and of this stage is done before they are reused
+        tc_fence_after();
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::COLS) : "memory");
     }
 }
 
@@ -380,20 +478,29 @@ template <int D>
 static bt_status launch_tc(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad, int lm,
                            int H, void *O, cudaStream_t st)
 {
-    constexpr size_t smem = tc_smem_bytes<D>();
+    constexpr size_t smem = TcPipe<D>::BYTES;
     static bool set[64] = {false};
+    static int sms[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
     if (dev >= 64 || !set[dev]) {
-        if (cudaFuncSetAttribute(k_ball_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)))
+        if (cudaFuncSetAttribute(k_ball_attn_tc2<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)))
             return BT_ERR_CUDA;
-        if (dev < 64) set[dev] = true;
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BT_ERR_CUDA;
+        if (dev < 64) {
+            sms[dev] = n;
+            set[dev] = true;
+        }
     }
-    dim3 grid(unsigned((npad + 127) / 128), unsigned(H));
+    const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
+    const int64_t items = (npad + 127) / 128 * H;
+    const int per_sm = TcPipe<D>::PER_SM;
+    const int64_t grid = items < int64_t(nsm) * per_sm ? items : int64_t(nsm) * per_sm;
     const float sl2 = 1.4426950408889634f / sqrtf(float(D));
-    k_ball_attn_tc<D><<<grid, kTcThreads, smem, st>>>(
+    k_ball_attn_tc2<D><<<unsigned(grid), kTcThreads, smem, st>>>(
         static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(K),
-        static_cast<const __nv_bfloat16 *>(V), perm, npad, lm, H, sl2, static_cast<__nv_bfloat16 *>(O));
+        static_cast<const __nv_bfloat16 *>(V), perm, npad, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O));
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 

@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
     const uint32_t gb = block_exclusive_scan<NT, uint32_t>(hc, scratch, nullptr);
     if (tid < 256) {
         const uint32_t excl =
-            lookback(&sst[(size_t(PASS) * 3 * P.sort_tiles + id) * 256 + tid], 256, k, dcount, status);
+            lookback<16>(&sst[(size_t(PASS) * 3 * P.sort_tiles + id) * 256 + tid], 256, k, dcount, status);
         tstart[tid] = ts;
         gpos[tid] = gb + excl - ts;  // modulo 2^32; + local index gives the position in the segment
     }
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
     constexpr int NT = kLevelThreads, EPT = kLevelEpt;
     __shared__ uint32_t sl[4][kLevelTileMax];
     __shared__ unsigned long long scratch[NT / 32 + 1];
-    __shared__ uint32_t s_tile, s_excl[4], s_pkey, s_pid;
+    __shared__ uint32_t s_tile, s_excl[4], s_pkey, s_pid, s_cand[3], s_ckey[3];
     __shared__ int s_axis;
     __shared__ float s_ext[3];
     const int tid = threadIdx.x;
@@ -356,27 +356,30 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
     const int j = int(r - kseg * tps);
     const int64_t seg = P.pad[b] + kseg * s;
     const int64_t nreal = max64(0, min64(s, P.n[b] - kseg * s));
+    const int64_t tile0 = seg + int64_t(j) * TP;
     if (tid < 3) {
+        // extent and candidate pivot of axis tid, all loads independent of the axis choice
+        const uint32_t pp = lin[tid * np + seg + half];
         float e = 0.0f;
         if (nreal > 0) {
             const uint32_t p0 = lin[tid * np + seg], p1 = lin[tid * np + seg + nreal - 1];
             e = __fsub_rn(key_float(keys[tid * np + p1]), key_float(keys[tid * np + p0]));
         }
         s_ext[tid] = e;
+        s_cand[tid] = pp;
+        s_ckey[tid] = keys[tid * np + pp];
     }
+    for (int l = 0; l < 4; ++l)
+        for (int i = tid; i < TP; i += NT) sl[l][i] = lin[l * np + tile0 + i];
     __syncthreads();
     if (tid == 0) {
         int ax = 0;
         if (s_ext[1] > s_ext[ax]) ax = 1;
         if (s_ext[2] > s_ext[ax]) ax = 2;
-        const uint32_t pp = lin[ax * np + seg + half];
         s_axis = ax;
-        s_pid = pp;
-        s_pkey = keys[ax * np + pp];
+        s_pid = s_cand[ax];
+        s_pkey = s_ckey[ax];
     }
-    const int64_t tile0 = seg + int64_t(j) * TP;
-    for (int l = 0; l < 4; ++l)
-        for (int i = tid; i < TP; i += NT) sl[l][i] = lin[l * np + tile0 + i];
     __syncthreads();
     const int ax = s_axis;
     const uint32_t pkey = s_pkey, ppid = s_pid;
@@ -406,7 +409,7 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
     unsigned long long tot = 0;
     const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, &tot);
     if (tid < 4)
-        s_excl[tid] = lookback(&lst[(size_t(lev) * (np / TP) + id) * 4 + tid], 4, j,
+        s_excl[tid] = lookback<16>(&lst[(size_t(lev) * (np / TP) + id) * 4 + tid], 4, j,
                                uint32_t((tot >> (16 * tid)) & 0xFFFFu), status);
 #pragma unroll
     for (int l = 0; l < 4; ++l) {

@@ -61,6 +61,7 @@ constexpr uint32_t kLbInclusive = 2u << 30;
 constexpr uint32_t kLbValue = (1u << 30) - 1u;
 constexpr int kSpinLimit = 1 << 20;
 
+template <int LB>
 __device__ __forceinline__ uint32_t lookback(uint32_t *self, int stride, int k_in_segment, uint32_t aggregate,
                                              uint32_t *status)
 {
@@ -70,20 +71,31 @@ __device__ __forceinline__ uint32_t lookback(uint32_t *self, int stride, int k_i
     }
     st_relaxed(self, kLbAggregate | aggregate);
     uint32_t excl = 0;
-    const uint32_t *p = self - stride;
-    for (int k = k_in_segment - 1; k >= 0; --k, p -= stride) {
-        uint32_t w;
-        int spins = 0;
-        while (((w = ld_relaxed(p)) >> 30) == 0u) {
-            if (++spins > kSpinLimit) {
-                record_error(status, BT_ERR_TIMEOUT);
-                w = kLbInclusive;
-                break;
+    // predecessors are read LB at a time with independent loads, nearest first, so a tile that
+    // has to sum many aggregates pays one round trip per LB predecessors, not one per predecessor
+    for (int q0 = k_in_segment - 1; q0 >= 0; q0 -= LB) {
+        uint32_t w[LB];
+#pragma unroll
+        for (int i = 0; i < LB; ++i) w[i] = (q0 - i >= 0) ? ld_relaxed(self - (k_in_segment - q0 + i) * stride) : 0u;
+        bool done = false;
+#pragma unroll
+        for (int i = 0; i < LB; ++i) {
+            if (done || q0 - i < 0) break;
+            uint32_t x = w[i];
+            int spins = 0;
+            while ((x >> 30) == 0u) {
+                if (++spins > kSpinLimit) {
+                    record_error(status, BT_ERR_TIMEOUT);
+                    x = kLbInclusive;
+                    break;
+                }
+                __nanosleep(32);
+                x = ld_relaxed(self - (k_in_segment - q0 + i) * stride);
             }
-            __nanosleep(32);
+            excl += x & kLbValue;
+            done = (x >> 30) == 2u;
         }
-        excl += w & kLbValue;
-        if ((w >> 30) == 2u) break;
+        if (done) break;
     }
     st_relaxed(self, kLbInclusive | (excl + aggregate));
     return excl;
