@@ -42,7 +42,7 @@ _SIGS = {
     "bt_compose": ([_P, _P, _i64, _P, _P], ctypes.c_int),
     "bt_gather": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
     "bt_scatter": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
-    "bt_ball_attention": ([_P, _P, _P, _P, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
+    "bt_ball_attention": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
     "bt_attention_device_status": ([_P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -207,8 +207,8 @@ def bt_ball_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: t
     if out is None:
         out = torch.empty_like(Q)
     _check("bt_ball_attention",
-           _lib.bt_ball_attention(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, m, H, d, dt, _dptr(out),
-                                  _stream(stream)))
+           _lib.bt_ball_attention(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, rows, m, H, d, dt,
+                                  _dptr(out), _stream(stream)))
     return out
 
 

@@ -39,14 +39,22 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return
 
 template <typename T, int D>
 __global__ void k_ball_attn_simt(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
-                                 const int32_t *__restrict__ perm, int m, int H, float scale, T *__restrict__ O)
+                                 const int32_t *__restrict__ perm, int64_t rows, int m, int H, float scale,
+                                 T *__restrict__ O)
 {
     extern __shared__ __align__(16) float fsm[];
     float *sK = fsm, *sV = fsm + m * D;
     int32_t *sRow = reinterpret_cast<int32_t *>(sV + m * D);
     const int64_t b = blockIdx.x;
     const int h = blockIdx.y;
-    for (int j = threadIdx.x; j < m; j += blockDim.x) sRow[j] = perm ? perm[b * m + j] : int32_t(b * m + j);
+    for (int j = threadIdx.x; j < m; j += blockDim.x) {
+        int32_t r = perm ? perm[b * m + j] : int32_t(b * m + j);
+        if (r >= rows) {  // not a row of Q/K/V: never read or write it
+            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            r = -1;
+        }
+        sRow[j] = r;
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < m * D; e += blockDim.x) {
         const int j = e / D, k = e - j * D;
@@ -240,8 +248,8 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, ui
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
     k_ball_attn_tc2(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
-                    const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ perm, int64_t npad, int lm,
-                    int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O)
+                    const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ perm, int64_t npad,
+                    int64_t rows, int lm, int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O)
 {
     using L = TcPipe<D>;
     constexpr int KCH = D / 8;                 // 16-byte chunks per row of one head
@@ -289,15 +297,22 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
     auto row_of = [&](int64_t item, int r) -> int32_t {
         if (item >= items) return -1;
         const int64_t slot = (item / H) * 128 + r;
-        return slot < npad ? (perm ? __ldg(perm + slot) : int32_t(slot)) : -1;
+        if (slot >= npad) return -1;
+        if (!perm) return int32_t(slot);
+        const int32_t row = __ldg(perm + slot);
+        if (row >= rows) {  // not a row of Q/K/V: never read or write it
+            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            return -1;
+        }
+        return row;
     };
     // rows whose chunks this thread copies: chunk u = tid + i*128 belongs to row u / KCH
-    auto load_rows = [&](int64_t item, int32_t (&rows)[UPT]) {
+    auto load_rows = [&](int64_t item, int32_t (&rr)[UPT]) {
 #pragma unroll
-        for (int i = 0; i < UPT; ++i) rows[i] = row_of(item, (tid + i * kTcThreads) / KCH);
+        for (int i = 0; i < UPT; ++i) rr[i] = row_of(item, (tid + i * kTcThreads) / KCH);
     };
     // gather Q, K (K-major core matrices) and V (MN-major core matrices) of one item into a stage
-    auto issue = [&](int64_t item, int stage, const int32_t (&rows)[UPT]) {
+    auto issue = [&](int64_t item, int stage, const int32_t (&rw)[UPT]) {
         if (item < items) {
             const int h = int(item % H);
             uint8_t *sq = tsm + stage * L::STAGE, *sk = sq + L::QK_BYTES, *sv = sk + L::QK_BYTES;
@@ -305,7 +320,7 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
             for (int i = 0; i < UPT; ++i) {
                 const int u = tid + i * kTcThreads;
                 const int r = u / KCH, c = u - r * KCH;
-                const int32_t rr = rows[i];
+                const int32_t rr = rw[i];
                 const size_t goff = rr >= 0 ? (size_t(rr) * H + h) * D + c * 8 : 0;
                 const uint32_t so = (r >> 3) * QK_SBO + c * 128 + (r & 7) * 16;
                 cp_async16(sq + so, Q + goff, rr >= 0);
@@ -317,17 +332,17 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
     };
 
     const int64_t first = blockIdx.x, stride = gridDim.x;
-    int32_t rows[UPT];
-    load_rows(first, rows);
-    issue(first, 0, rows);
-    load_rows(first + stride, rows);  // rows of the next item, used at the top of the loop
+    int32_t nrows[UPT];
+    load_rows(first, nrows);
+    issue(first, 0, nrows);
+    load_rows(first + stride, nrows);  // rows of the next item, used at the top of the loop
     int32_t qcur = row_of(first, tid), qnext = row_of(first + stride, tid);
     bool ok = true;
     int it = 0;
     for (int64_t item = first; item < items; item += stride, ++it) {
         const int stage = it & 1;
-        issue(item + stride, stage ^ 1, rows);
-        load_rows(item + 2 * stride, rows);  // consumed one iteration later
+        issue(item + stride, stage ^ 1, nrows);
+        load_rows(item + 2 * stride, nrows);  // consumed one iteration later
         const int32_t qafter = row_of(item + 2 * stride, tid);
         const uint32_t kb = __ballot_sync(0xffffffffu, qcur >= 0);
         if (lane == 0) sKeyMask[warp] = kb;
@@ -459,8 +474,8 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
 }
 
 template <typename T, int D>
-static bt_status launch_simt(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad, int m,
-                             int H, void *O, cudaStream_t st)
+static bt_status launch_simt(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
+                             int64_t rows, int m, int H, void *O, cudaStream_t st)
 {
     const size_t smem = size_t(2) * m * D * 4 + size_t(m) * 4;
     if (smem > 48 * 1024 &&
@@ -469,14 +484,14 @@ static bt_status launch_simt(const void *Q, const void *K, const void *V, const 
     const int threads = ((m + 31) / 32) * 32;
     dim3 grid(unsigned(npad / m), unsigned(H));
     k_ball_attn_simt<T, D><<<grid, threads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(K),
-                                                        static_cast<const T *>(V), perm, m, H,
+                                                        static_cast<const T *>(V), perm, rows, m, H,
                                                         1.0f / sqrtf(float(D)), static_cast<T *>(O));
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 
 template <int D>
-static bt_status launch_tc(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad, int lm,
-                           int H, void *O, cudaStream_t st)
+static bt_status launch_tc(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
+                           int64_t rows, int lm, int H, void *O, cudaStream_t st)
 {
     constexpr size_t smem = TcPipe<D>::BYTES;
     static bool set[64] = {false};
@@ -500,7 +515,7 @@ static bt_status launch_tc(const void *Q, const void *K, const void *V, const in
     const float sl2 = 1.4426950408889634f / sqrtf(float(D));
     k_ball_attn_tc2<D><<<unsigned(grid), kTcThreads, smem, st>>>(
         static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(K),
-        static_cast<const __nv_bfloat16 *>(V), perm, npad, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O));
+        static_cast<const __nv_bfloat16 *>(V), perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O));
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 
@@ -509,28 +524,29 @@ static bt_status launch_tc(const void *Q, const void *K, const void *V, const in
 using namespace bts;
 
 extern "C" bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
-                                       int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream)
+                                       int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream)
 {
-    if (!Q || !K || !V || !O || npad < 0 || H < 1) return BT_ERR_ARG;
+    if (!Q || !K || !V || !O || npad < 0 || rows < 0 || H < 1) return BT_ERR_ARG;
     if (m < 1 || m > 256 || (d != 32 && d != 64)) return BT_ERR_SHAPE;
     if (npad % m) return BT_ERR_SHAPE;
     if (dt != BT_F32 && dt != BT_BF16) return BT_ERR_ARG;
+    if (!perm && rows < npad) return BT_ERR_ARG;
     if (npad == 0) return BT_OK;
-    if (npad / m > 0x7FFFFFFF || int64_t(H) > 65535) return BT_ERR_UNSUPPORTED;
+    if (npad / m > 0x7FFFFFFF || int64_t(H) > 65535 || rows > 0x7FFFFFFF) return BT_ERR_UNSUPPORTED;
     const uintptr_t al = reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) |
                          reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(O);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dt == BT_BF16 && (m == 16 || m == 32 || m == 64 || m == 128)) {
         if (al % 16) return BT_ERR_ARG;
         const int lm = m == 16 ? 4 : m == 32 ? 5 : m == 64 ? 6 : 7;
-        return d == 32 ? launch_tc<32>(Q, K, V, perm, npad, lm, H, O, st)
-                       : launch_tc<64>(Q, K, V, perm, npad, lm, H, O, st);
+        return d == 32 ? launch_tc<32>(Q, K, V, perm, npad, rows, lm, H, O, st)
+                       : launch_tc<64>(Q, K, V, perm, npad, rows, lm, H, O, st);
     }
     if (dt == BT_BF16)
-        return d == 32 ? launch_simt<__nv_bfloat16, 32>(Q, K, V, perm, npad, m, H, O, st)
-                       : launch_simt<__nv_bfloat16, 64>(Q, K, V, perm, npad, m, H, O, st);
-    return d == 32 ? launch_simt<float, 32>(Q, K, V, perm, npad, m, H, O, st)
-                   : launch_simt<float, 64>(Q, K, V, perm, npad, m, H, O, st);
+        return d == 32 ? launch_simt<__nv_bfloat16, 32>(Q, K, V, perm, npad, rows, m, H, O, st)
+                       : launch_simt<__nv_bfloat16, 64>(Q, K, V, perm, npad, rows, m, H, O, st);
+    return d == 32 ? launch_simt<float, 32>(Q, K, V, perm, npad, rows, m, H, O, st)
+                   : launch_simt<float, 64>(Q, K, V, perm, npad, rows, m, H, O, st);
 }
 
 extern "C" bt_status bt_attention_device_status(void *stream)

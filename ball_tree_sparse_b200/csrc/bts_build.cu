@@ -29,7 +29,7 @@ namespace bts {
 
 constexpr int kSortTile = 1024;      // keys per radix tile
 constexpr int kSortThreads = 256;
-constexpr int kLevelThreads = 128;
+constexpr int kLevelThreads = 512;     // one slot of each list per thread (two when m > 512)
 constexpr int kLevelTileTarget = 512;  // slots per list per wide-level tile (m * 2^k, or m when m > 512)
 constexpr int kLevelTileMax = 1024;
 constexpr int kLevelEpt = kLevelTileMax / kLevelThreads;
@@ -357,13 +357,22 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
     const int64_t seg = P.pad[b] + kseg * s;
     const int64_t nreal = max64(0, min64(s, P.n[b] - kseg * s));
     const int64_t tile0 = seg + int64_t(j) * TP;
+    const uint32_t id_lo = uint32_t(P.pad[b]), id_hi = uint32_t(P.pad[b + 1]);  // ids of this cloud
     if (tid < 3) {
         // extent and candidate pivot of axis tid, all loads independent of the axis choice
-        const uint32_t pp = lin[tid * np + seg + half];
+        uint32_t pp = lin[tid * np + seg + half];
         float e = 0.0f;
         if (nreal > 0) {
-            const uint32_t p0 = lin[tid * np + seg], p1 = lin[tid * np + seg + nreal - 1];
+            uint32_t p0 = lin[tid * np + seg], p1 = lin[tid * np + seg + nreal - 1];
+            if (p0 < id_lo || p0 >= id_hi || p1 < id_lo || p1 >= id_hi) {  // never index with a foreign id
+                record_error(status, BT_ERR_INTERNAL);
+                p0 = p1 = id_lo;
+            }
             e = __fsub_rn(key_float(keys[tid * np + p1]), key_float(keys[tid * np + p0]));
+        }
+        if (pp < id_lo || pp >= id_hi) {
+            record_error(status, BT_ERR_INTERNAL);
+            pp = id_lo;
         }
         s_ext[tid] = e;
         s_cand[tid] = pp;
@@ -398,7 +407,15 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
             if (q < ept && i < TP) {
                 const uint32_t pid = sl[l][i];
                 v[l][q] = pid;
-                const bool left = (l == ax) ? int64_t(j) * TP + i < half : before(kax[pid], pid, pkey, ppid);
+                bool left;
+                if (l == ax) {
+                    left = int64_t(j) * TP + i < half;
+                } else if (pid < id_lo || pid >= id_hi) {
+                    record_error(status, BT_ERR_INTERNAL);
+                    left = false;
+                } else {
+                    left = before(kax[pid], pid, pkey, ppid);
+                }
                 if (left) {
                     lbits[l] |= 1u << q;
                     packed += 1ull << (16 * l);
@@ -448,6 +465,14 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
 //    node's index list), so the index list itself is the identity and every
 //    list fits in 16 bits.  `loc` is a global scratch array pid -> local index.
 // ---------------------------------------------------------------------------
+// A local index read from a tail list; out of range only after an invariant broke (then recorded)
+__device__ __forceinline__ uint32_t local_ok(uint32_t v, int sT, uint32_t *status)
+{
+    if (v < uint32_t(sT)) return v;
+    record_error(status, BT_ERR_INTERNAL);
+    return 0;
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict__ keys,
                                              const uint32_t *__restrict__ lists, uint32_t *__restrict__ loc,
@@ -478,10 +503,16 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
     const uint32_t *lin = lists + size_t(P.glev[b] & 1) * 4 * np;
     const int m = P.m;
 
+    const uint32_t id_lo = uint32_t(P.pad[b]), id_hi = uint32_t(P.pad[b + 1]);  // ids of this cloud
     for (int e = tid; e < sT; e += NT) {
-        const uint32_t pid = lin[3 * np + seg + e];
+        uint32_t pid = lin[3 * np + seg + e];
+        if (pid < id_lo || pid >= id_hi) {  // never index with a foreign id
+            record_error(status, BT_ERR_INTERNAL);
+            pid = id_lo;
+        } else {
+            loc[pid] = uint32_t(e);
+        }
         ps[e] = pid;
-        loc[pid] = uint32_t(e);
 #pragma unroll
         for (int a = 0; a < 3; ++a) k3[a * T + e] = keys[a * np + pid];
         lst[3 * T + e] = uint16_t(e);
@@ -491,7 +522,7 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
             const uint32_t pid = lin[a * np + seg + e];
-            const uint32_t l = loc[pid];
+            const uint32_t l = (pid >= id_lo && pid < id_hi) ? loc[pid] : 0xFFFFFFFFu;
             if (l >= uint32_t(sT) || ps[l] != pid) {  // lists disagree on the node's points
                 record_error(status, BT_ERR_INTERNAL);
                 lst[a * T + e] = 0;
@@ -515,13 +546,13 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
             if (nr > 0) {
 #pragma unroll
                 for (int a = 0; a < 3; ++a)
-                    ext[a] = __fsub_rn(key_float(k3[a * T + L[a * T + start + nr - 1]]),
-                                       key_float(k3[a * T + L[a * T + start]]));
+                    ext[a] = __fsub_rn(key_float(k3[a * T + local_ok(L[a * T + start + nr - 1], sT, status)]),
+                                       key_float(k3[a * T + local_ok(L[a * T + start], sT, status)]));
             }
             int ax = 0;
             if (ext[1] > ext[ax]) ax = 1;
             if (ext[2] > ext[ax]) ax = 2;
-            const uint32_t pv = L[ax * T + start + half];
+            const uint32_t pv = local_ok(L[ax * T + start + half], sT, status);
             axs[q] = uint8_t(ax);
             ppv[q] = uint16_t(pv);
             pkey[q] = k3[ax * T + pv];
@@ -543,7 +574,7 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
                 const uint32_t *ka = k3 + ax * T;
 #pragma unroll
                 for (int l = 0; l < 4; ++l) {
-                    const uint32_t v = L[l * T + e];
+                    const uint32_t v = local_ok(L[l * T + e], sT, status);
                     const bool left = (l == ax) ? (e - sub_start) < half : before(ka[v], v, pk, pv);
                     if (left) {
                         lbits[l] |= 1u << q;
@@ -605,7 +636,7 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
     }
     const uint16_t *L = lst + cur * 4 * T;
     for (int e = tid; e < sT; e += NT) {
-        const uint32_t pid = ps[L[3 * T + e]];
+        const uint32_t pid = ps[local_ok(L[3 * T + e], sT, status)];
         const int64_t li = int64_t(pid) - P.pad[b];
         perm[seg + e] = li < P.n[b] ? int32_t(P.row0[b] + li) : -1;
     }

@@ -11,16 +11,16 @@ namespace bts {
 // ---------------------------------------------------------------------------
 // Device status word: the first error recorded wins; 0 = no error.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void record_error(uint32_t *status, uint32_t code)
-{
-    atomicCAS(status, 0u, code);
-}
-
 __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t *p)
 {
     uint32_t v;
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ void record_error(uint32_t *status, uint32_t code)
+{
+    if (ld_relaxed(status) == 0u) atomicCAS(status, 0u, code);  // read first: no atomic storm once set
 }
 
 __device__ __forceinline__ void st_relaxed(uint32_t *p, uint32_t v)

@@ -177,22 +177,27 @@ bt_status bt_scatter(const void *Y, const int32_t *idx, int64_t npad, int32_t ro
  * over the real rows j of the same ball.  No bias, no positional term.
  *   Q, K, V  [rows, H, d] of dtype dt (BT_F32: float, BT_BF16: bfloat16)
  *   perm     int32 [npad] slot -> row (dummy slots -1: neither query nor
- *            key, nothing written), or NULL: row s sits in slot s (rows =
+ *            key, nothing written), or NULL: row s sits in slot s (rows >=
  *            npad, no dummies).  Gathering by perm and scattering O back is
- *            fused into the attention kernel.
+ *            fused into the attention kernel.  An entry >= rows is never
+ *            dereferenced: the slot is treated as a dummy and BT_ERR_INTERNAL
+ *            is recorded for bt_attention_device_status().
  *   npad     number of slots, a multiple of m
+ *   rows     number of rows of Q, K, V and O
  *   m        1 <= m <= 256;  H >= 1;  d in {32, 64}
- *   O        [rows, H, d] out, dtype dt, original row order
+ *   O        [rows, H, d] out, dtype dt, original row order; rows no slot
+ *            names are left untouched
  * Accumulation and softmax are in float.  BT_BF16 with m dividing 128 runs on
  * the tcgen05 tensor cores; other shapes run on the CUDA cores.
  */
 bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
-                            int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream);
+                            int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream);
 
 /*
  * Device-side status of the attention kernels on the current device:
- * synchronises `stream`, returns BT_OK or BT_ERR_TIMEOUT (a tensor-core
- * completion wait that gave up) and clears the recorded code.
+ * synchronises `stream`, returns BT_OK, BT_ERR_TIMEOUT (a tensor-core
+ * completion wait that gave up) or BT_ERR_INTERNAL (a perm entry >= rows),
+ * and clears the recorded code.
  */
 bt_status bt_attention_device_status(void *stream);
 

@@ -55,10 +55,11 @@ def test_argument_errors_before_any_launch(lib):
     P = ctypes.c_void_p
     lib.bt_build.argtypes = [P, ctypes.c_int64, ctypes.c_int32, P, P, ctypes.c_size_t, P]
     assert lib.bt_build(None, 1024, 32, None, None, 0, None) == 1          # BT_ERR_ARG
-    lib.bt_ball_attention.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
-                                      ctypes.c_int, P, P]
+    lib.bt_ball_attention.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, ctypes.c_int, P, P]
     one = ctypes.c_void_p(16)
-    assert lib.bt_ball_attention(one, one, one, None, 128, 32, 2, 48, 1, one, None) == 2  # d = 48
-    assert lib.bt_ball_attention(one, one, one, None, 100, 32, 2, 32, 1, one, None) == 2  # npad % m
+    assert lib.bt_ball_attention(one, one, one, None, 128, 128, 32, 2, 48, 1, one, None) == 2  # d = 48
+    assert lib.bt_ball_attention(one, one, one, None, 100, 100, 32, 2, 32, 1, one, None) == 2  # npad % m
+    assert lib.bt_ball_attention(one, one, one, None, 128, 64, 32, 2, 32, 1, one, None) == 1  # rows < npad
     lib.bt_gather.argtypes = [P, P, ctypes.c_int64, ctypes.c_int32, P, P]
     assert lib.bt_gather(one, one, 10, 0, one, None) == 1                   # row_bytes < 1

@@ -53,3 +53,22 @@ def test_segmented_argument_errors():
     with pytest.raises(bts.BtsError) as e:
         bts.bt_build_segmented(c, list(range(0, 66)), 1, ws=ws)  # 65 clouds
     assert e.value.status == "BT_ERR_UNSUPPORTED"
+
+
+def test_attention_perm_entry_out_of_range_is_recorded_not_read(orc):
+    n, m, H, d = 256, 128, 2, 32
+    q, k, v = workloads.random_qkv(n, H, d, workloads.BF16, 17)
+    perm = np.arange(n, dtype=np.int32)
+    perm[5] = 10 ** 6  # not a row of Q/K/V
+    Q, K, V = (torch.from_numpy(t.view(np.int16)).cuda().view(torch.bfloat16) for t in (q, k, v))
+    out = torch.full_like(Q, 7.0)
+    bts.bt_ball_attention(Q, K, V, torch.from_numpy(perm).cuda(), m, out=out)
+    assert bts.bt_attention_device_status() == 8  # BT_ERR_INTERNAL, then cleared
+    assert bts.bt_attention_device_status() == 0
+    got = out.float().cpu().numpy()
+    assert np.all(got[5] == 7.0)  # the slot was treated as a dummy: row 5 is named by no valid slot
+    ref_perm = perm.copy()
+    ref_perm[5] = -1
+    want = orc.ball_attention(q, k, v, m, ref_perm)
+    keep = np.arange(n) != 5
+    assert np.abs(got[keep] - want[keep]).max() <= 2e-2
