@@ -11,7 +11,7 @@ The arithmetic lives in ``oracle.c`` (single-threaded C, compiled with
 Pinned functions (each checked by ``tests/test_oracle_*.py`` against worked
 examples, brute force, closed forms or a library routine): ``build``,
 ``rotate_z``, ``ball_attention``, ``full_attention``, ``invert``,
-``compose``.
+``compose``, ``bsa``.
 """
 from __future__ import annotations
 
@@ -55,6 +55,9 @@ def _load():
         lib.orc_invert.restype = None
         lib.orc_compose.argtypes = [P, P, i64, P]
         lib.orc_compose.restype = None
+        lib.orc_bsa.argtypes = [P, P, P, ctypes.c_int, P, i64, i64, i32, i32, i32, P, i32, P, P, i32, i32, P,
+                                P, i64, P, P, P, P, P, P, P]
+        lib.orc_bsa.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -146,3 +149,31 @@ def compose(invA: np.ndarray, permB: np.ndarray) -> np.ndarray:
     out = np.empty(len(permB), np.int32)
     _load().orc_compose(_ptr(invA), _ptr(permB), len(permB), _ptr(out))
     return out
+
+
+def bsa(q, k, v, m: int, perm, x, w_g, b_g=None, topk: int = 8, mask_own: bool = True, sel_in=None,
+        branches: bool = False, groups=None):
+    """Ball Sparse Attention in float64 (see oracle.c, orc_bsa).  Returns O [rows, H, d]; with branches=True
+    a dict with O, O_ball, O_cmp, O_slc, gates [rows, H, 3], sel [nb, H, topk] and scores [nb, H, nb]."""
+    q, k, v = (np.ascontiguousarray(t) for t in (q, k, v))
+    rows, H, d = q.shape
+    npad = rows if perm is None else len(perm)
+    nb = npad // m
+    perm_a = None if perm is None else np.ascontiguousarray(perm, dtype=np.int32)
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    w_g = np.ascontiguousarray(w_g, dtype=np.float32)
+    b_a = None if b_g is None else np.ascontiguousarray(b_g, dtype=np.float32)
+    sel_a = None if sel_in is None else np.ascontiguousarray(sel_in, dtype=np.int32)
+    grp = None if groups is None else np.ascontiguousarray(groups, dtype=np.int64)
+    out = {name: np.full((rows, H, d), np.nan) for name in ("O", "O_ball", "O_cmp", "O_slc")}
+    out["gates"] = np.full((rows, H, 3), np.nan)
+    out["sel"] = np.full((nb, H, topk), -2, np.int32)
+    out["scores"] = np.full((nb, H, nb), np.nan)
+    rc = _load().orc_bsa(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(perm_a), npad, rows, m, H, d, _ptr(x),
+                         x.shape[1], _ptr(w_g), _ptr(b_a), topk, int(mask_own), _ptr(sel_a), _ptr(grp),
+                         0 if grp is None else len(grp), _ptr(out["O"]),
+                         _ptr(out["O_ball"]), _ptr(out["O_cmp"]), _ptr(out["O_slc"]), _ptr(out["gates"]),
+                         _ptr(out["sel"]), _ptr(out["scores"]))
+    if rc != 0:
+        raise OracleError(f"orc_bsa failed with status {rc}")
+    return out if branches else out["O"]

@@ -258,3 +258,180 @@ void orc_compose(const int32_t *invA, const int32_t *permB, int64_t npad, int32_
 {
     for (int64_t s = 0; s < npad; ++s) map[s] = permB[s] >= 0 ? invA[permB[s]] : -1;
 }
+
+/*
+ * Ball Sparse Attention (page: Pith review of "BSA: Ball Sparse Attention for
+ * Large-scale Geometries" - reading notes and referee report).  Three
+ * branches per query, mixed by learned sigmoid gates:
+ *   ball        - attention inside the query's own ball (as above);
+ *   compression - attention over one coarse token per ball: the mean of the
+ *                 ball's K and V rows (mean pooling, one token per ball);
+ *   selection   - the queries of one group (= one ball of m slots) share one
+ *                 set of blocks: the group's pooled query (mean of its q rows)
+ *                 is scored against every coarse key, q_bar . k_bar / sqrt(d),
+ *                 the group's own ball is masked, and the top-k balls (ties to
+ *                 the lower ball index) are attended at full resolution.
+ *   gates       - g[i, h, br] = sigmoid(b[3h+br] + sum_c X[i,c] W[c, 3h+br]),
+ *                 br = 0 ball, 1 compression, 2 selection.
+ *   O = g0 O_ball + g1 O_cmp + g2 O_slc   (per head).
+ * Everything in double from the widened inputs.  A ball with no real point
+ * gives no coarse token and cannot be selected.
+ *
+ * sel_in (optional, [nb, H, topk]): use this selection instead of computing it
+ * (the tests use it where two blocks tie within rounding).  groups (optional):
+ * compute output rows only for these groups.  All outputs except O may be
+ * NULL.  Rows are [rows, H, d] in original order; scores [nb, H, nb].
+ */
+static void attend_vec(const double *q, const double *keys, const double *vals, const unsigned char *valid,
+                       int64_t n, int32_t d, double *logit, double *o)
+{
+    double scale = 1.0 / sqrt((double)d), mx = -INFINITY, den = 0.0;
+    int any = 0;
+    for (int k = 0; k < d; ++k) o[k] = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+        if (valid && !valid[j]) continue;
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) acc += q[k] * keys[j * d + k];
+        logit[j] = acc * scale;
+        if (logit[j] > mx) mx = logit[j];
+        any = 1;
+    }
+    if (!any) return;
+    for (int64_t j = 0; j < n; ++j) {
+        if (valid && !valid[j]) continue;
+        double w = exp(logit[j] - mx);
+        den += w;
+        for (int k = 0; k < d; ++k) o[k] += w * vals[j * d + k];
+    }
+    for (int k = 0; k < d; ++k) o[k] /= den;
+}
+
+int orc_bsa(const void *Q, const void *K, const void *V, int dtype, const int32_t *perm, int64_t npad, int64_t rows,
+            int32_t m, int32_t H, int32_t d, const float *X, int32_t C, const float *Wg, const float *bg, int32_t topk,
+            int32_t mask_own, const int32_t *sel_in, const int64_t *groups, int64_t n_groups, double *O,
+            double *O_ball, double *O_cmp, double *O_slc, double *gates, int32_t *sel_out, double *scores_out)
+{
+    if (!Q || !K || !V || !O || !X || !Wg || m < 1 || H < 1 || d < 1 || C < 1 || topk < 0 || npad % m) return ORC_ERR_ARG;
+    int64_t nb = npad / m;
+    double *qbar = (double *)calloc((size_t)(nb * H * d), sizeof(double));
+    double *kbar = (double *)calloc((size_t)(nb * H * d), sizeof(double));
+    double *vbar = (double *)calloc((size_t)(nb * H * d), sizeof(double));
+    unsigned char *tok = (unsigned char *)calloc((size_t)nb, 1);
+    double *logit = (double *)malloc((size_t)((nb > m * (int64_t)(topk + 1) ? nb : m * (int64_t)(topk + 1)) * sizeof(double)));
+    double *keys = (double *)malloc((size_t)(m * (int64_t)(topk + 1) * d) * sizeof(double));
+    double *vals = (double *)malloc((size_t)(m * (int64_t)(topk + 1) * d) * sizeof(double));
+    double *kc = (double *)malloc((size_t)(nb * d) * sizeof(double));
+    double *vc = (double *)malloc((size_t)(nb * d) * sizeof(double));
+    double *sc = (double *)malloc((size_t)nb * sizeof(double));
+    int32_t *sel = (int32_t *)malloc((size_t)(nb * H * (topk > 0 ? topk : 1)) * sizeof(int32_t));
+    int64_t *krows = (int64_t *)malloc((size_t)m * sizeof(int64_t));
+    double *ob = (double *)malloc((size_t)d * sizeof(double)), *oc = (double *)malloc((size_t)d * sizeof(double));
+    double *os = (double *)malloc((size_t)d * sizeof(double)), *qv = (double *)malloc((size_t)d * sizeof(double));
+    if (!qbar || !kbar || !vbar || !tok || !logit || !keys || !vals || !kc || !vc || !sc || !sel || !krows || !ob || !oc ||
+        !os || !qv)
+        return ORC_ERR_ARG;
+    /* coarse tokens and pooled queries: means over the real rows of each ball */
+    for (int64_t b = 0; b < nb; ++b) {
+        int64_t cnt = 0;
+        for (int64_t j = 0; j < m; ++j) {
+            int64_t r = perm ? perm[b * m + j] : b * m + j;
+            if (r < 0) continue;
+            ++cnt;
+            for (int32_t h = 0; h < H; ++h)
+                for (int k = 0; k < d; ++k) {
+                    int64_t idx = (r * H + h) * d + k, o = (b * H + h) * d + k;
+                    qbar[o] += widen(Q, dtype, idx);
+                    kbar[o] += widen(K, dtype, idx);
+                    vbar[o] += widen(V, dtype, idx);
+                }
+        }
+        tok[b] = cnt > 0;
+        if (cnt)
+            for (int64_t o = b * H * d; o < (b + 1) * H * d; ++o) {
+                qbar[o] /= (double)cnt;
+                kbar[o] /= (double)cnt;
+                vbar[o] /= (double)cnt;
+            }
+    }
+    /* group scores and top-k per (group, head) */
+    for (int64_t g = 0; g < nb; ++g)
+        for (int32_t h = 0; h < H; ++h) {
+            for (int64_t b = 0; b < nb; ++b) {
+                double acc = 0.0;
+                for (int k = 0; k < d; ++k) acc += qbar[(g * H + h) * d + k] * kbar[(b * H + h) * d + k];
+                sc[b] = (tok[b] && tok[g] && !(mask_own && b == g)) ? acc / sqrt((double)d) : -INFINITY;
+                if (scores_out) scores_out[(g * H + h) * nb + b] = sc[b];
+            }
+            int32_t *s = sel + (g * H + h) * topk;
+            for (int t = 0; t < topk; ++t) {
+                int64_t best = -1;
+                for (int64_t b = 0; b < nb; ++b) {
+                    if (sc[b] == -INFINITY) continue;
+                    int taken = 0;
+                    for (int u = 0; u < t; ++u) taken |= s[u] == b;
+                    if (taken) continue;
+                    if (best < 0 || sc[b] > sc[best]) best = b;  /* strict: the lower index wins ties */
+                }
+                s[t] = (int32_t)best;
+            }
+            if (sel_in)
+                for (int t = 0; t < topk; ++t) s[t] = sel_in[(g * H + h) * topk + t];
+            if (sel_out)
+                for (int t = 0; t < topk; ++t) sel_out[(g * H + h) * topk + t] = s[t];
+        }
+    /* branches, gates and the gated sum for every real query row (of the listed groups) */
+    for (int64_t gi = 0; gi < (groups ? n_groups : nb); ++gi) {
+        int64_t g = groups ? groups[gi] : gi;
+        int64_t nk = 0;
+        for (int64_t j = 0; j < m; ++j) {
+            int64_t r = perm ? perm[g * m + j] : g * m + j;
+            if (r >= 0) krows[nk++] = r;
+        }
+        for (int32_t h = 0; h < H; ++h) {
+            for (int64_t b = 0; b < nb; ++b)
+                for (int k = 0; k < d; ++k) {
+                    kc[b * d + k] = kbar[(b * H + h) * d + k];
+                    vc[b * d + k] = vbar[(b * H + h) * d + k];
+                }
+            int64_t ns = 0;
+            const int32_t *s = sel + (g * H + h) * topk;
+            for (int t = 0; t < topk; ++t) {
+                if (s[t] < 0) continue;
+                for (int64_t j = 0; j < m; ++j) {
+                    int64_t r = perm ? perm[(int64_t)s[t] * m + j] : (int64_t)s[t] * m + j;
+                    if (r < 0) continue;
+                    for (int k = 0; k < d; ++k) {
+                        keys[ns * d + k] = widen(K, dtype, (r * H + h) * d + k);
+                        vals[ns * d + k] = widen(V, dtype, (r * H + h) * d + k);
+                    }
+                    ++ns;
+                }
+            }
+            for (int64_t i = 0; i < nk; ++i) {
+                int64_t r = krows[i];
+                for (int k = 0; k < d; ++k) qv[k] = widen(Q, dtype, (r * H + h) * d + k);
+                attend(Q, K, V, dtype, H, d, h, r, krows, nk, logit, ob);
+                attend_vec(qv, kc, vc, tok, nb, d, logit, oc);
+                attend_vec(qv, keys, vals, NULL, ns, d, logit, os);
+                double gv[3];
+                for (int br = 0; br < 3; ++br) {
+                    double z = bg ? (double)bg[3 * h + br] : 0.0;
+                    for (int c = 0; c < C; ++c) z += (double)X[r * C + c] * (double)Wg[(int64_t)c * 3 * H + 3 * h + br];
+                    gv[br] = 1.0 / (1.0 + exp(-z));
+                    if (gates) gates[(r * H + h) * 3 + br] = gv[br];
+                }
+                for (int k = 0; k < d; ++k) {
+                    int64_t o = (r * H + h) * d + k;
+                    O[o] = gv[0] * ob[k] + gv[1] * oc[k] + gv[2] * os[k];
+                    if (O_ball) O_ball[o] = ob[k];
+                    if (O_cmp) O_cmp[o] = oc[k];
+                    if (O_slc) O_slc[o] = os[k];
+                }
+            }
+        }
+    }
+    (void)rows;
+    free(qbar); free(kbar); free(vbar); free(tok); free(logit); free(keys); free(vals); free(kc); free(vc); free(sc);
+    free(sel); free(krows); free(ob); free(oc); free(os); free(qv);
+    return ORC_OK;
+}
