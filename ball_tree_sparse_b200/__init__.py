@@ -44,7 +44,17 @@ _SIGS = {
     "bt_scatter": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
     "bt_ball_attention": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
     "bt_attention_device_status": ([_P], ctypes.c_int),
+    "bsa_workspace_size": ([_i64, _i64, _i32, _i32, _i32, _i32], _sz),
+    "bsa_forward": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _i32, _P, _P, None, _P, _P,
+                     _P, _sz, _P], ctypes.c_int),
 }
+
+
+class bsa_params(ctypes.Structure):
+    _fields_ = [("topk", ctypes.c_int32), ("mask_own_ball", ctypes.c_int32)]
+
+
+_SIGS["bsa_forward"][0][14] = bsa_params
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
     _f.argtypes = _args
@@ -214,3 +224,32 @@ def bt_ball_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: t
 
 def bt_attention_device_status(stream=None) -> int:
     return int(_lib.bt_attention_device_status(_stream(stream)))
+
+
+def bsa_workspace_size(npad: int, rows: int, m: int, H: int, d: int, topk: int) -> int:
+    return int(_lib.bsa_workspace_size(npad, rows, m, H, d, topk))
+
+
+def bsa_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.Tensor | None, m: int,
+                X: torch.Tensor, Wg: torch.Tensor, bg: torch.Tensor | None = None, topk: int = 8,
+                mask_own_ball: bool = True, out: torch.Tensor | None = None, sel: torch.Tensor | None = None,
+                ws: torch.Tensor | None = None, npad: int | None = None, stream=None) -> torch.Tensor:
+    """Ball Sparse Attention: ball + compression + top-k selection branches mixed by sigmoid gates.
+    Q/K/V/O bf16 [rows, H, d] in original row order; X float [rows, C]; Wg float [C, 3H]."""
+    rows, H, d = Q.shape
+    if Q.dtype != torch.bfloat16:
+        raise TypeError("bsa_forward takes bfloat16 Q/K/V")
+    if npad is None:
+        npad = perm.numel() if perm is not None else rows
+    if out is None:
+        out = torch.empty_like(Q)
+    if ws is None:
+        n = bsa_workspace_size(npad, rows, m, H, d, topk)
+        if n == 0:
+            raise BtsError("bsa_workspace_size", 2)
+        ws = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    _check("bsa_forward",
+           _lib.bsa_forward(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, rows, m, H, d, BT_BF16, _dptr(X),
+                            X.shape[1], _dptr(Wg), _dptr(bg), bsa_params(topk, int(mask_own_ball)), _dptr(out),
+                            _dptr(sel), _dptr(ws), ws.numel(), _stream(stream)))
+    return out

@@ -194,6 +194,47 @@ bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const i
                             int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream);
 
 /*
+ * Ball Sparse Attention ("BSA: Ball Sparse Attention for Large-scale
+ * Geometries", as reviewed on Pith: reading notes and referee report).  Three
+ * branches per query row i and head h, mixed by sigmoid gates:
+ *   ball        O_ball  attention inside the query's own ball (as above);
+ *   compression O_cmp   attention over one coarse token per ball: the mean of
+ *                       the ball's real K rows and V rows;
+ *   selection   O_slc   the queries of one ball form a group; the group's
+ *                       pooled query (mean of its Q rows) is scored against
+ *                       every coarse key, s_b = q_bar . k_bar_b / sqrt(d), the
+ *                       own ball masked if p.mask_own_ball, and the p.topk best
+ *                       balls (ties to the lower ball) are attended at full
+ *                       resolution;
+ *   O[i,h] = g0 O_ball + g1 O_cmp + g2 O_slc,
+ *   g_br = sigmoid(bg[3h+br] + sum_c X[i,c] Wg[c, 3h+br]), br 0 ball,
+ *   1 compression, 2 selection.
+ *   Q, K, V, perm, npad, rows  as for bt_ball_attention (bf16 only)
+ *   m        128 (the ball, the query group and one selected block)
+ *   d        32 or 64;  H <= 64;  npad / m <= 2048 balls;  0 <= topk <= 32
+ *   X        float [rows, C] gate features (original row order), C <= 2048
+ *   Wg       float [C, 3H] gate weights;  bg  float [3H] or NULL (zero)
+ *   O        bf16 [rows, H, d] out
+ *   sel_out  int32 [npad/m, H, topk] out (may be NULL): the selected balls per
+ *            (group, head), -1 where fewer than topk balls can be selected
+ *   ws       workspace of bsa_workspace_size() bytes, 256-byte aligned
+ * Coarse tokens and scores are float; attention accumulates in float with
+ * P rounded to bf16 for the tensor cores.  A ball with no real point gives
+ * no coarse token and is never selected.
+ */
+typedef struct {
+    int32_t topk;          /* blocks selected per (group, head) */
+    int32_t mask_own_ball; /* nonzero: a group never selects its own ball */
+} bsa_params;
+
+size_t bsa_workspace_size(int64_t npad, int64_t rows, int32_t m, int32_t H, int32_t d, int32_t topk);
+
+bt_status bsa_forward(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
+                      int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, const float *X, int32_t C,
+                      const float *Wg, const float *bg, bsa_params p, void *O, int32_t *sel_out, void *ws,
+                      size_t ws_bytes, void *stream);
+
+/*
  * Device-side status of the attention kernels on the current device:
  * synchronises `stream`, returns BT_OK, BT_ERR_TIMEOUT (a tensor-core
  * completion wait that gave up) or BT_ERR_INTERNAL (a perm entry >= rows),

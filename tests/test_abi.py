@@ -13,7 +13,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _declared():
     text = open(os.path.join(ROOT, "include", "bts.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bt_[a-z_0-9]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b((?:bt|bsa)_[a-z_0-9]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
