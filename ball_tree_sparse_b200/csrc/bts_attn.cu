@@ -361,6 +361,324 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Two heads per work item (d = 32, even H).  The rows of Q, K and V are gathered by TMA
+// (tile::gather4 through perm) as 128-byte pieces: the two heads of a row side by side, 128-byte
+// swizzled, so each gather moves enough bytes per request to keep HBM busy.  Warpgroup j of the CTA
+// owns head j of the pair: its S in TMEM columns [128j, 128j+128), P written back over the first 64 of
+// them, O at +64 and the row sums at +96.  The two heads share one K-major swizzle row, so head j's
+// operands start 64 bytes into it; V is read MN-major from the same rows.
+// ---------------------------------------------------------------------------
+struct PairPipe {
+    static constexpr int NS = 2;
+    static constexpr uint32_t RB = 128;                 // bytes of one row of a head pair
+    static constexpr uint32_t TILE = 128 * RB;          // Q, K or V of one item (16 KB)
+    static constexpr uint32_t STAGE = 3 * TILE;
+    static constexpr uint32_t ONES_OFF = NS * STAGE;
+    static constexpr uint32_t BYTES = ONES_OFF + 16 * 128 * 2 + 1024;
+    static constexpr uint32_t COLS = 256;
+    static constexpr int THREADS = 256;
+    static constexpr int PER_SM = 2;
+};
+
+__global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
+    k_ball_attn_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ perm, int64_t npad,
+                     int64_t rows, int lm, int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O)
+{
+    using L = PairPipe;
+    constexpr int NS = L::NS;
+    constexpr int D = 32;
+    constexpr uint32_t SBO8 = 8 * L::RB, ONES_SBO = 16 * 128, SW128 = 2;
+    constexpr uint32_t IDESC_S = idesc_bf16(128, false);
+    constexpr uint32_t IDESC_O = idesc_bf16(D, true);
+    constexpr uint32_t IDESC_SUM = idesc_bf16(16, false);
+    extern __shared__ __align__(1024) uint8_t psm[];
+    __shared__ uint32_t sKeyMask[4];
+    __shared__ __align__(8) uint64_t sBarS, sBarO, sFull[NS];
+    __shared__ uint32_t sTmem;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int hj = warp >> 2;          // head of the pair this warpgroup owns
+    const int r = tid & 127;           // query row (TMEM lane) this thread owns
+    const int m = 1 << lm;
+    const int HP = H >> 1;
+    const uint32_t base = (smem_u32(psm) + 1023u) & ~1023u;  // swizzled tiles need 1024-byte alignment
+    uint8_t *gbase = psm + (base - smem_u32(psm));
+
+    for (int i = tid; i < 16 * 128 * 2 / 16; i += L::THREADS) {
+        const int c = i >> 4, rr = i & 15;
+        const uint32_t off = (rr >> 3) * ONES_SBO + c * 128 + (rr & 7) * 16;
+        const uint32_t one = (rr == 0) ? 0x3F803F80u : 0u;
+        *reinterpret_cast<uint4 *>(gbase + L::ONES_OFF + off) = make_uint4(one, one, one, one);
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sTmem)),
+                     "r"(L::COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarS)) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarO)) : "memory");
+        for (int s0 = 0; s0 < NS; ++s0)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sFull[s0])) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sTmem;
+    const uint32_t tS = tmem + 128 * hj, tO = tS + 64, tSum = tS + 96;  // this warpgroup's columns
+    const uint32_t barS = smem_u32(&sBarS), barO = smem_u32(&sBarO);
+    const uint32_t lanebase = uint32_t((warp & 3) * 32) << 16;
+    const int32_t oob = rows < 0x7FFFFFFF ? int32_t(rows) : -1;  // a row outside the tensor reads zeros
+
+    auto raw_row = [&](int64_t item, int rr) -> int32_t {  // items < 2^31: 32-bit index arithmetic
+        if (item >= items) return -1;
+        const int64_t slot = int64_t(uint32_t(item) / uint32_t(HP)) * 128 + rr;
+        if (slot >= npad) return -1;
+        return perm ? __ldg(perm + slot) : int32_t(slot);
+    };
+    auto check = [&](int32_t row) -> int32_t {
+        if (row >= rows) {  // not a row of Q/K/V: never read or write it
+            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            return -1;
+        }
+        return row;
+    };
+    // all eight warps share the gathers of an item: lane l < 4 of warp w takes rows 4g..4g+3, g = 4w + l, of
+    // Q, K and V (both heads).  The transaction count is armed once, before any of them can complete.
+    auto issue = [&](int64_t item, int stage, const int32_t (&rw)[4]) {
+        if (item >= items) return;  // uniform across the CTA
+        const uint32_t bar = smem_u32(&sFull[stage]);
+        if (tid == 0) mbar_expect_tx(bar, L::STAGE);
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (lane >= 4) return;
+        int32_t rr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int32_t x = check(rw[i]);
+            rr[i] = x >= 0 ? x : oob;
+        }
+        const int32_t col = int32_t(uint32_t(item) % uint32_t(HP)) * 2 * D;
+        const uint32_t dq = base + stage * L::STAGE + (4 * warp + lane) * 4 * L::RB;
+        tma_gather4(dq, &tmQ, col, rr[0], rr[1], rr[2], rr[3], bar);
+        tma_gather4(dq + L::TILE, &tmK, col, rr[0], rr[1], rr[2], rr[3], bar);
+        tma_gather4(dq + 2 * L::TILE, &tmV, col, rr[0], rr[1], rr[2], rr[3], bar);
+    };
+    auto load_rows = [&](int64_t item, int32_t (&rr)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rr[i] = lane < 4 ? raw_row(item, 4 * (4 * warp + lane) + i) : -1;
+    };
+
+    const int64_t first = blockIdx.x, stride = gridDim.x;
+    int32_t nrows[4];
+    load_rows(first, nrows);
+    issue(first, 0, nrows);
+    load_rows(first + stride, nrows);
+    int32_t qcur = check(raw_row(first, r)), qnext = raw_row(first + stride, r);
+    bool ok = true;
+    int it = 0;
+    for (int64_t item = first; item < items; item += stride, ++it) {
+        const int stage = it & 1;
+        issue(item + stride, stage ^ 1, nrows);
+        load_rows(item + 2 * stride, nrows);  // consumed one iteration later
+        const int32_t qafter = raw_row(item + 2 * stride, r);
+        if (warp < 4) {
+            const uint32_t kb = __ballot_sync(0xffffffffu, qcur >= 0);
+            if (lane == 0) sKeyMask[warp] = kb;
+        }
+        ok = ok && mbar_wait(smem_u32(&sFull[stage]), (it >> 1) & 1);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        const uint32_t sq = base + stage * L::STAGE, sk = sq + L::TILE, sv = sk + L::TILE;
+        if (tid == 0 && ok) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16(tmem + 128 * j, smem_desc_sw(sq + 64 * j + 32 * kk, 16, SBO8, SW128),
+                             smem_desc_sw(sk + 64 * j + 32 * kk, 16, SBO8, SW128), IDESC_S, kk > 0);
+            mma_commit(barS);
+        }
+        ok = ok && mbar_wait(barS, it & 1);
+        tc_fence_after();
+
+        // softmax of row r of head hj; keys outside its ball or dummy get weight 0
+        const int ball0 = (r >> lm) << lm;
+        uint32_t cmask[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t bm;
+            if (m >= 32)
+                bm = (c * 32 >= ball0 && c * 32 < ball0 + m) ? 0xffffffffu : 0u;
+            else
+                bm = (c * 32 <= ball0 && ball0 < c * 32 + 32) ? (((1u << m) - 1u) << (ball0 - c * 32)) : 0u;
+            cmask[c] = bm & sKeyMask[c];
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
+                uint32_t v[32];
+                tmem_ld32(tS + lanebase + c * 32, v);
+                if (cmask[c] == 0xffffffffu) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) mx = fmax3(mx, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if ((cmask[c] >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]));
+                }
+            }
+        }
+        const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+            if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
+                uint32_t v[32];
+                tmem_ld32(tS + lanebase + c * 32, v);
+                const uint32_t cm = cmask[c];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+                    float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
+                    if (cm != 0xffffffffu) {
+                        p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
+                        p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                    }
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                    pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) pk[j] = 0u;
+            }
+            tmem_st16(tS + lanebase + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && ok) {
+            const uint32_t so1 = base + L::ONES_OFF;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t tp = tmem + 128 * j + kk * 8;
+                    mma_bf16_ts(tmem + 128 * j + 64, tp, smem_desc_sw(sv + 64 * j + kk * 16 * L::RB, 16, SBO8, SW128),
+                                IDESC_O, kk > 0);
+                    mma_bf16_ts(tmem + 128 * j + 96, tp, smem_desc(so1 + kk * 256, 128, ONES_SBO), IDESC_SUM, kk > 0);
+                }
+            mma_commit(barO);
+        }
+        ok = ok && mbar_wait(barO, it & 1);
+        tc_fence_after();
+        if (ok) {
+            uint32_t sum_bits, o[32];
+            tmem_ld1_nowait(tSum + lanebase, sum_bits);
+            tmem_ld32_nowait(tO + lanebase, o);
+            tmem_wait_ld();
+            const float sum = __uint_as_float(sum_bits);
+            const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+            const int h = int(uint32_t(item) % uint32_t(HP)) * 2 + hj;
+            if (qcur >= 0) {
+                uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qcur) * H + h) * D);
+#pragma unroll
+                for (int t = 0; t < D / 8; ++t) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * t + 2 * e]) * inv,
+                                                                        __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                    }
+                    dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        }
+        qcur = check(qnext);
+        qnext = qafter;
+        tc_fence_before();
+        __syncthreads();  // every read of S/P, O and of this stage is done before they are reused
+        tc_fence_after();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::COLS) : "memory");
+    }
+}
+
+// Tensor maps that view a [rows, H, d] bf16 tensor as rows of H*d elements with a `box`-element window
+// per row (the gather unit of the attention kernels), 128-byte swizzled to match the tcgen05 operands.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+static bool row_map(CUtensorMap *map, const void *base, int64_t rows, int hd, int box)
+{
+    const EncodeTiledFn fn = encode_tiled();
+    if (!fn || rows < 1 || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(hd), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(hd) * 2};
+    const cuuint32_t bx[2] = {cuuint32_t(box), 1};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, bx, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bt_status launch_pair(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
+                             int64_t rows, int lm, int H, void *O, cudaStream_t st)
+{
+    static bool set[64] = {false};
+    static int sms[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
+    if (dev >= 64 || !set[dev]) {
+        if (cudaFuncSetAttribute(k_ball_attn_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(PairPipe::BYTES)))
+            return BT_ERR_CUDA;
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BT_ERR_CUDA;
+        if (dev < 64) {
+            sms[dev] = n;
+            set[dev] = true;
+        }
+    }
+    CUtensorMap mq, mk, mv;
+    if (!row_map(&mq, Q, rows, H * 32, 64) || !row_map(&mk, K, rows, H * 32, 64) || !row_map(&mv, V, rows, H * 32, 64))
+        return BT_ERR_CUDA;
+    const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
+    const int64_t items = (npad + 127) / 128 * (H / 2);
+    if (items > 0x7FFFFFFF) return BT_ERR_UNSUPPORTED;
+    const int64_t grid = items < int64_t(nsm) * PairPipe::PER_SM ? items : int64_t(nsm) * PairPipe::PER_SM;
+    const float sl2 = 1.4426950408889634f / sqrtf(32.0f);
+    k_ball_attn_pair<<<unsigned(grid), PairPipe::THREADS, PairPipe::BYTES, st>>>(
+        mq, mk, mv, perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O));
+    return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
+}
+
 template <typename T, int D>
 static bt_status launch_simt(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
                              int64_t rows, int m, int H, void *O, cudaStream_t st)
@@ -429,6 +747,7 @@ extern "C" bt_status bt_ball_attention(const void *Q, const void *K, const void 
     if (dt == BT_BF16 && (m == 16 || m == 32 || m == 64 || m == 128)) {
         if (al % 16) return BT_ERR_ARG;
         const int lm = m == 16 ? 4 : m == 32 ? 5 : m == 64 ? 6 : 7;
+        if (d == 32 && H % 2 == 0 && rows < 0x7FFFFFFF) return launch_pair(Q, K, V, perm, npad, rows, lm, H, O, st);
         return d == 32 ? launch_tc<32>(Q, K, V, perm, npad, rows, lm, H, O, st)
                        : launch_tc<64>(Q, K, V, perm, npad, rows, lm, H, O, st);
     }

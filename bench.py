@@ -51,6 +51,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-suite", action="store_true", help="skip the other workloads")
+    p.add_argument("--suite-steps", type=int, default=20)
     return p.parse_args()
 
 
@@ -287,6 +289,116 @@ def run_reference(args, wl):
 
 
 # ---------------------------------------------------------------------------
+def timed_graph(fn, steps, warmup, flush):
+    """Capture fn() as a CUDA graph; return the per-replay device times (ms), L2 flushed between replays."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(warmup):
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        e0.record()
+        g.replay()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    del g
+    return ts
+
+
+def _bf16_dev(a, dev):
+    return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def suite(bts, dev, steps, flush, peak):
+    """The other synthetic workloads, each timed on its own (layer = tree build + ball attention)."""
+    res = {}
+    # tiny: fp32, one layer
+    wl = workloads.tiny()
+    c = torch.from_numpy(wl.coords).to(dev)
+    L = wl.layers[0]
+    q, k, v = (torch.from_numpy(t).to(dev) for t in (L.q, L.k, L.v))
+    perm = torch.empty(wl.n_total, dtype=torch.int32, device=dev)
+    ws = bts.workspace([0, wl.n_total], wl.m, dev)
+    out = torch.empty_like(q)
+
+    def tiny_step():
+        bts.bt_build(c, wl.m, perm=perm, ws=ws)
+        bts.bt_ball_attention(q, k, v, perm, wl.m, out=out)
+    ms = statistics.mean(timed_graph(tiny_step, steps, 3, flush))
+    res["tiny"] = {"points": wl.n_total, "layers": 1, "dtype": "f32", "ms_per_step": ms,
+                   "points_per_s_per_layer": wl.n_total / (ms / 1e3)}
+
+    # ellipsoid: one layer of tree build + BSA (ball, compression, top-8 selection, gates)
+    wl = workloads.ellipsoid()
+    L = wl.layers[0]
+    c = torch.from_numpy(wl.coords).to(dev)
+    q, k, v = (_bf16_dev(t, dev) for t in (L.q, L.k, L.v))
+    x = torch.from_numpy(wl.extra["x"]).to(dev)
+    wg = torch.from_numpy(wl.extra["w_g"]).to(dev)
+    perm = torch.empty(wl.n_total, dtype=torch.int32, device=dev)
+    ws = bts.workspace([0, wl.n_total], wl.m, dev)
+    bws = torch.empty(bts.bsa_workspace_size(wl.n_total, wl.n_total, wl.m, wl.H, wl.d, 8), dtype=torch.uint8,
+                      device=dev)
+    out = torch.empty_like(q)
+    bts.bt_build(c, wl.m, perm=perm, ws=ws)
+
+    def bsa_only():
+        bts.bsa_forward(q, k, v, perm, wl.m, x, wg, topk=8, out=out, ws=bws)
+
+    def ell_step():
+        bts.bt_build(c, wl.m, perm=perm, ws=ws)
+        bsa_only()
+    ms = statistics.mean(timed_graph(ell_step, steps, 3, flush))
+    ms_bsa = statistics.mean(timed_graph(bsa_only, steps, 3, flush))
+    flop = 4 * wl.d * wl.H * (wl.m + wl.n_total // wl.m + 8 * wl.m) * wl.n_total
+    res["ellipsoid_bsa"] = {"points": wl.n_total, "layers": 1, "ms_per_step": ms,
+                            "points_per_s_per_layer": wl.n_total / (ms / 1e3), "bsa_ms": ms_bsa,
+                            "bsa_gflop": flop / 1e9, "bsa_tflops": flop / (ms_bsa / 1e3) / 1e12,
+                            "note": "BSA = ball + compression over 512 ball means + top-8 selection, gated"}
+    del q, k, v, x, out, bws
+
+    # box + cluster, 1,048,576 points: two layers (original and rotated tree), as the headline step
+    wl = workloads.box_cluster()
+    st = Step(bts, wl, dev)
+    ms = statistics.mean(timed_graph(lambda: st.body(), steps, 3, flush))
+    a_ms = statistics.mean(timed_graph(
+        lambda: bts.bt_ball_attention(*st.qkv[1], st.perm[1], wl.m, out=st.out[1]), steps, 3, flush))
+    nbytes = 4 * wl.n_total * wl.H * wl.d * 2 + 4 * st.npad
+    res["box_cluster"] = {"points": wl.n_total, "layers": 2, "ms_per_step": ms,
+                          "points_per_s_per_layer": 2 * wl.n_total / (ms / 1e3), "attention_ms": a_ms,
+                          "attention_gbs": nbytes / (a_ms / 1e3) / 1e9,
+                          "attention_frac_of_measured_hbm": nbytes / (a_ms / 1e3) / 1e9 / peak}
+    del st
+
+    # ragged batch of 8 clouds, padded with dummies: segmented build + masked ball attention
+    wl = workloads.ragged()
+    L = wl.layers[0]
+    c = torch.from_numpy(wl.coords).to(dev)
+    q, k, v = (_bf16_dev(t, dev) for t in (L.q, L.k, L.v))
+    npad = int(wl.pad_offsets()[-1])
+    perm = torch.empty(npad, dtype=torch.int32, device=dev)
+    ws = bts.workspace(wl.offsets, wl.m, dev)
+    out = torch.empty_like(q)
+
+    def rag_step():
+        bts.bt_build_segmented(c, wl.offsets, wl.m, perm=perm, ws=ws)
+        bts.bt_ball_attention(q, k, v, perm, wl.m, out=out, npad=npad)
+    ms = statistics.mean(timed_graph(rag_step, steps, 3, flush))
+    res["ragged"] = {"points": wl.n_total, "padded_slots": npad, "clouds": wl.batch, "layers": 1, "ms_per_step": ms,
+                     "points_per_s_per_layer": wl.n_total / (ms / 1e3)}
+    return res
+
+
+# ---------------------------------------------------------------------------
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -395,11 +507,13 @@ def main():
         "gpu_launches": kernels_per_step(wl) * args.steps,
         "clocks": clocks.summary(),
     }
+    if rank == 0 and not args.no_suite:
+        del st
+        line["workloads"] = suite(bts, dev, args.suite_steps, flush, peak)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del st
     if dist:
         dist.destroy_process_group()
 
