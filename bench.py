@@ -196,6 +196,20 @@ class Step:
                 "join_b_and_maps": e["a2"].elapsed_time(e["b1"]), "attn_b": e["b1"].elapsed_time(e["b2"])}
 
 
+def reduce_max(x: float, dist=None, device="cpu") -> float:
+    """Max over ranks of a per-rank device time (every rank takes the same collective step)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_value(world: int, layers: int, points: int, steps: int, total_ms: float) -> float:
+    """Whole-job points per second per layer: every rank processed `points` per layer per step."""
+    return world * layers * points * steps / (total_ms / 1e3)
+
+
 def kernels_per_step(wl) -> int:
     """Launches of this library's kernels in one step (memsets excluded)."""
     m = wl.m
@@ -451,13 +465,9 @@ def main():
     if dist:
         dist.barrier()
     clocks.stop()
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
-    value = world * LAYERS * wl.n_total * args.steps / (total_ms / 1e3)
+    value = aggregate_value(world, LAYERS, wl.n_total, args.steps, total_ms)
 
     # end to end through the public API: pinned host inputs in, outputs back to pinned host memory
     host_in = [torch.from_numpy(wl.coords).pin_memory()]
@@ -480,12 +490,8 @@ def main():
         s1.record()
         s1.synchronize()
         e_ms.append(s0.elapsed_time(s1))
-    e_total = sum(e_ms)
-    if dist:
-        t = torch.tensor([e_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_total = float(t.item())
-    e2e_value = world * LAYERS * wl.n_total * e2e_steps / (e_total / 1e3)
+    e_total = reduce_max(sum(e_ms), dist, dev)
+    e2e_value = aggregate_value(world, LAYERS, wl.n_total, e2e_steps, e_total)
 
     peak, peak_kind = _peaks()
     attn_bytes = 4 * wl.n_total * wl.H * wl.d * 2 + 4 * st.npad  # Q, K, V read + O written, perm read
