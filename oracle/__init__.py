@@ -55,7 +55,7 @@ def _load():
         lib.orc_invert.restype = None
         lib.orc_compose.argtypes = [P, P, i64, P]
         lib.orc_compose.restype = None
-        lib.orc_bsa.argtypes = [P, P, P, ctypes.c_int, P, i64, i64, i32, i32, i32, P, i32, P, P, i32, i32, P,
+        lib.orc_bsa.argtypes = [P, P, P, ctypes.c_int, P, i64, i64, i32, i32, i32, P, i32, P, P, i32, i32, i32, P,
                                 P, i64, P, P, P, P, P, P, P]
         lib.orc_bsa.restype = ctypes.c_int
         _lib = lib
@@ -152,9 +152,10 @@ def compose(invA: np.ndarray, permB: np.ndarray) -> np.ndarray:
 
 
 def bsa(q, k, v, m: int, perm, x, w_g, b_g=None, topk: int = 8, mask_own: bool = True, sel_in=None,
-        branches: bool = False, groups=None):
+        branches: bool = False, groups=None, coarsen: bool = False):
     """Ball Sparse Attention in float64 (see oracle.c, orc_bsa).  Returns O [rows, H, d]; with branches=True
-    a dict with O, O_ball, O_cmp, O_slc, gates [rows, H, 3], sel [nb, H, topk] and scores [nb, H, nb]."""
+    a dict with O, O_ball, O_cmp, O_slc, gates [rows, H, 3], sel [nb, H, topk] and scores [nb, H, nb].
+    coarsen=True is the query-coarsening variant: compression and selection use the group's pooled query."""
     q, k, v = (np.ascontiguousarray(t) for t in (q, k, v))
     rows, H, d = q.shape
     npad = rows if perm is None else len(perm)
@@ -170,7 +171,7 @@ def bsa(q, k, v, m: int, perm, x, w_g, b_g=None, topk: int = 8, mask_own: bool =
     out["sel"] = np.full((nb, H, topk), -2, np.int32)
     out["scores"] = np.full((nb, H, nb), np.nan)
     rc = _load().orc_bsa(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(perm_a), npad, rows, m, H, d, _ptr(x),
-                         x.shape[1], _ptr(w_g), _ptr(b_a), topk, int(mask_own), _ptr(sel_a), _ptr(grp),
+                         x.shape[1], _ptr(w_g), _ptr(b_a), topk, int(mask_own), int(coarsen), _ptr(sel_a), _ptr(grp),
                          0 if grp is None else len(grp), _ptr(out["O"]),
                          _ptr(out["O_ball"]), _ptr(out["O_cmp"]), _ptr(out["O_slc"]), _ptr(out["gates"]),
                          _ptr(out["sel"]), _ptr(out["scores"]))

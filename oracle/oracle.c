@@ -277,6 +277,12 @@ void orc_compose(const int32_t *invA, const int32_t *permB, int64_t npad, int32_
  * Everything in double from the widened inputs.  A ball with no real point
  * gives no coarse token and cannot be selected.
  *
+ * coarsen_q: the optional query-coarsening step (BSA with group compression):
+ * the compression and selection branches take the group's pooled query q_bar
+ * (the mean of its real q rows) in place of each query, so every query of a
+ * group gets the same O_cmp and O_slc; the ball branch and the gates stay per
+ * query.
+ *
  * sel_in (optional, [nb, H, topk]): use this selection instead of computing it
  * (the tests use it where two blocks tie within rounding).  groups (optional):
  * compute output rows only for these groups.  All outputs except O may be
@@ -308,7 +314,7 @@ static void attend_vec(const double *q, const double *keys, const double *vals, 
 
 int orc_bsa(const void *Q, const void *K, const void *V, int dtype, const int32_t *perm, int64_t npad, int64_t rows,
             int32_t m, int32_t H, int32_t d, const float *X, int32_t C, const float *Wg, const float *bg, int32_t topk,
-            int32_t mask_own, const int32_t *sel_in, const int64_t *groups, int64_t n_groups, double *O,
+            int32_t mask_own, int32_t coarsen_q, const int32_t *sel_in, const int64_t *groups, int64_t n_groups, double *O,
             double *O_ball, double *O_cmp, double *O_slc, double *gates, int32_t *sel_out, double *scores_out)
 {
     if (!Q || !K || !V || !O || !X || !Wg || m < 1 || H < 1 || d < 1 || C < 1 || topk < 0 || npad % m) return ORC_ERR_ARG;
@@ -409,7 +415,7 @@ int orc_bsa(const void *Q, const void *K, const void *V, int dtype, const int32_
             }
             for (int64_t i = 0; i < nk; ++i) {
                 int64_t r = krows[i];
-                for (int k = 0; k < d; ++k) qv[k] = widen(Q, dtype, (r * H + h) * d + k);
+                for (int k = 0; k < d; ++k) qv[k] = coarsen_q ? qbar[(g * H + h) * d + k] : widen(Q, dtype, (r * H + h) * d + k);
                 attend(Q, K, V, dtype, H, d, h, r, krows, nk, logit, ob);
                 attend_vec(qv, kc, vc, tok, nb, d, logit, oc);
                 attend_vec(qv, keys, vals, NULL, ns, d, logit, os);

@@ -191,3 +191,60 @@ def test_exact_score_ties_pick_the_lower_ball(orc):
         want = [b for b in range(8) if b != g][:3]
         for h in range(c["H"]):
             assert r["sel"][g, h].tolist() == want
+
+
+# --- query coarsening (BSA with group compression): compression and selection take the group's pooled query ---
+
+@pytest.mark.parametrize("ragged", [False, True])
+def test_coarsened_branches_vs_sdpa_of_pooled_query(orc, ragged):
+    c = _case(ragged=ragged, seed=12, topk=3)
+    perm, r = _run(orc, c, coarsen=True)
+    _, r0 = _run(orc, c)
+    assert np.array_equal(r["sel"], r0["sel"])  # the selection already uses the pooled query
+    qb, kb, vb, valid = _means(c, perm)
+    m = c["m"]
+    K, V = _widen(c["k"]), _widen(c["v"])
+    for g in range(len(perm) // m):
+        qrows = perm[g * m:(g + 1) * m]
+        qrows = qrows[qrows >= 0]
+        if not len(qrows):
+            continue
+        for h in range(c["H"]):
+            cmp = _sdpa_rows(qb[g, h][None], kb[valid, h], vb[valid, h])[0]
+            krows = np.concatenate([perm[b * m:(b + 1) * m] for b in r["sel"][g, h] if b >= 0])
+            krows = krows[krows >= 0]
+            slc = _sdpa_rows(qb[g, h][None], K[krows, h], V[krows, h])[0]
+            np.testing.assert_allclose(r["O_cmp"][qrows, h], np.broadcast_to(cmp, (len(qrows), c["d"])),
+                                       rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(r["O_slc"][qrows, h], np.broadcast_to(slc, (len(qrows), c["d"])),
+                                       rtol=1e-11, atol=1e-12)
+    # the ball branch and the gates are per query and do not change
+    np.testing.assert_array_equal(r["O_ball"], r0["O_ball"])
+    np.testing.assert_array_equal(r["gates"], r0["gates"])
+    np.testing.assert_allclose(r["O"], (r["gates"][..., :1] * r["O_ball"] + r["gates"][..., 1:2] * r["O_cmp"]
+                                        + r["gates"][..., 2:] * r["O_slc"]), rtol=1e-13, atol=1e-14)
+
+
+def test_coarsening_single_point_balls_changes_nothing(orc):
+    # with one point per ball the pooled query is the query itself
+    c = _case(n=256, m=1, seed=13, topk=4)
+    _, r = _run(orc, c, coarsen=True)
+    _, r0 = _run(orc, c)
+    for key in ("O", "O_cmp", "O_slc"):
+        np.testing.assert_allclose(r[key], r0[key], rtol=1e-14, atol=1e-15)
+
+
+def test_coarsening_with_identical_group_queries_changes_nothing(orc):
+    # every query of a ball equal: the pooled query equals each of them
+    c = _case(n=1024, m=64, seed=14, topk=3)
+    perm, _ = orc.build(c["pts"], c["m"], None)
+    q = c["q"].copy()
+    for b in range(len(perm) // 64):
+        rows = perm[b * 64:(b + 1) * 64]
+        q[rows] = q[rows[0]]
+    c["q"] = q
+    _, r = _run(orc, c, coarsen=True)
+    _, r0 = _run(orc, c)
+    assert np.array_equal(r["sel"], r0["sel"])
+    for key in ("O", "O_cmp", "O_slc"):
+        np.testing.assert_allclose(r[key], r0[key], rtol=1e-12, atol=1e-13)
