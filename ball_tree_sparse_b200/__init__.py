@@ -51,7 +51,7 @@ _SIGS = {
 
 
 class bsa_params(ctypes.Structure):
-    _fields_ = [("topk", ctypes.c_int32), ("mask_own_ball", ctypes.c_int32)]
+    _fields_ = [("topk", ctypes.c_int32), ("mask_own_ball", ctypes.c_int32), ("coarsen_queries", ctypes.c_int32)]
 
 
 _SIGS["bsa_forward"][0][14] = bsa_params
@@ -233,9 +233,11 @@ def bsa_workspace_size(npad: int, rows: int, m: int, H: int, d: int, topk: int) 
 def bsa_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.Tensor | None, m: int,
                 X: torch.Tensor, Wg: torch.Tensor, bg: torch.Tensor | None = None, topk: int = 8,
                 mask_own_ball: bool = True, out: torch.Tensor | None = None, sel: torch.Tensor | None = None,
-                ws: torch.Tensor | None = None, npad: int | None = None, stream=None) -> torch.Tensor:
+                ws: torch.Tensor | None = None, npad: int | None = None, stream=None,
+                coarsen_queries: bool = False) -> torch.Tensor:
     """Ball Sparse Attention: ball + compression + top-k selection branches mixed by sigmoid gates.
-    Q/K/V/O bf16 [rows, H, d] in original row order; X float [rows, C]; Wg float [C, 3H]."""
+    Q/K/V/O bf16 [rows, H, d] in original row order; X float [rows, C]; Wg float [C, 3H].
+    coarsen_queries=True: compression and selection attend with each group's pooled query."""
     rows, H, d = Q.shape
     if Q.dtype != torch.bfloat16:
         raise TypeError("bsa_forward takes bfloat16 Q/K/V")
@@ -250,6 +252,7 @@ def bsa_forward(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.T
         ws = torch.empty(n, dtype=torch.uint8, device=Q.device)
     _check("bsa_forward",
            _lib.bsa_forward(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, rows, m, H, d, BT_BF16, _dptr(X),
-                            X.shape[1], _dptr(Wg), _dptr(bg), bsa_params(topk, int(mask_own_ball)), _dptr(out),
+                            X.shape[1], _dptr(Wg), _dptr(bg), bsa_params(topk, int(mask_own_ball), int(coarsen_queries)),
+                            _dptr(out),
                             _dptr(sel), _dptr(ws), ws.numel(), _stream(stream)))
     return out

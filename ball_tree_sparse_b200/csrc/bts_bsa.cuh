@@ -434,6 +434,185 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
 }
 
 // ---------------------------------------------------------------------------
+// Query coarsening ("BSA with group compression"): the compression and
+// selection branches take the group's pooled query, so each (group, head)
+// item is one query vector against the coarse tokens and then against the
+// selected balls - matrix-vector work, on the CUDA cores.  One warp per item.
+// Lanes form groups of D/8; a lane group takes one key per half-step, each lane
+// 8 of its elements (16 bytes of the bf16 row), and keeps its own online
+// softmax (log2 domain); the lane groups merge at the end of each branch.  The
+// gated sum over the group's query rows follows in the same warp.
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&f)[8])
+{
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[e]));
+        f[2 * e] = t.x;
+        f[2 * e + 1] = t.y;
+    }
+}
+
+template <int G>
+__device__ __forceinline__ float lane_group_sum(float s)
+{
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
+
+// Two keys into one lane group's running softmax (m, l, acc); s0/s1 are the
+// scaled logits (log2 domain), -inf for a missing key (its value row is zero).
+__device__ __forceinline__ void softmax_push2(float s0, float s1, const float (&v0)[8], const float (&v1)[8], float &m,
+                                              float &l, float (&acc)[8])
+{
+    const float mn = fmaxf(m, fmaxf(s0, s1));
+    if (mn == -INFINITY) return;
+    const float alpha = ex2(m - mn), p0 = ex2(s0 - mn), p1 = ex2(s1 - mn);
+    l = fmaf(l, alpha, p0 + p1);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = fmaf(acc[k], alpha, fmaf(p0, v0[k], p1 * v1[k]));
+    m = mn;
+}
+
+// Merge the lane groups' softmax states (lanes with the same element slice)
+// and normalise: out = sum p v / sum p, zero when no key was valid.
+template <int G>
+__device__ __forceinline__ void softmax_merge(float m, float l, const float (&acc)[8], float (&out)[8])
+{
+    float M = m;
+#pragma unroll
+    for (int o = G; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float f = M == -INFINITY ? 0.0f : ex2(m - M);
+    float L = l * f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) out[k] = acc[k] * f;
+#pragma unroll
+    for (int o = G; o < 32; o <<= 1) {
+        L += __shfl_xor_sync(0xffffffffu, L, o);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) out[k] += __shfl_xor_sync(0xffffffffu, out[k], o);
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) out[k] *= inv;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) k_bsa_coarse(const __nv_bfloat16 *__restrict__ K,
+                                                    const __nv_bfloat16 *__restrict__ V,
+                                                    const int32_t *__restrict__ perm, int64_t rows, int H, int nb,
+                                                    const float *__restrict__ qbar,
+                                                    const __nv_bfloat16 *__restrict__ kc,
+                                                    const __nv_bfloat16 *__restrict__ vc,
+                                                    const int32_t *__restrict__ cnt, const int32_t *__restrict__ sel,
+                                                    int topk, const float *__restrict__ gates,
+                                                    const __nv_bfloat16 *__restrict__ Oball, float sl2,
+                                                    __nv_bfloat16 *__restrict__ O)
+{
+    constexpr int G = D / 8, KPS = 32 / G;  // lanes per key, keys per half-step
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t item = int64_t(blockIdx.x) * 4 + warp;
+    if (item >= int64_t(nb) * H) return;  // no block-wide synchronisation below
+    const int g = int(item / H), h = int(item - int64_t(g) * H);
+    const int sub = lane % G, kslot = lane / G;
+    const size_t hoff = size_t(h) * D + sub * 8, rstride = size_t(H) * D;
+    float q[8];
+    {
+        const float4 *qp = reinterpret_cast<const float4 *>(qbar + size_t(g) * rstride + hoff);
+        const float4 a = qp[0], b = qp[1];
+        q[0] = a.x; q[1] = a.y; q[2] = a.z; q[3] = a.w;
+        q[4] = b.x; q[5] = b.y; q[6] = b.z; q[7] = b.w;
+    }
+    auto logit = [&](const uint4 kw, bool valid) -> float {
+        float kf[8];
+        bf16x8_to_f32(kw, kf);
+        float s = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s = fmaf(q[k], kf[k], s);
+        s = lane_group_sum<G>(s);  // every lane takes part: no early exit before this
+        return valid ? s * sl2 : -INFINITY;
+    };
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+
+    // compression branch: every coarse token of a ball with a real point
+    float ocmp[8], oslc[8];
+    {
+        float m = -INFINITY, l = 0.0f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int b0 = kslot; b0 - kslot < nb; b0 += 2 * KPS) {
+            const int b1 = b0 + KPS;
+            const bool ok0 = b0 < nb && cnt[b0] > 0, ok1 = b1 < nb && cnt[b1] > 0;
+            const uint4 k0 = ok0 ? *reinterpret_cast<const uint4 *>(kc + size_t(b0) * rstride + hoff) : zero;
+            const uint4 k1 = ok1 ? *reinterpret_cast<const uint4 *>(kc + size_t(b1) * rstride + hoff) : zero;
+            const uint4 w0 = ok0 ? *reinterpret_cast<const uint4 *>(vc + size_t(b0) * rstride + hoff) : zero;
+            const uint4 w1 = ok1 ? *reinterpret_cast<const uint4 *>(vc + size_t(b1) * rstride + hoff) : zero;
+            const float s0 = logit(k0, ok0), s1 = logit(k1, ok1);
+            float v0[8], v1[8];
+            bf16x8_to_f32(w0, v0);
+            bf16x8_to_f32(w1, v1);
+            softmax_push2(s0, s1, v0, v1, m, l, acc);
+        }
+        softmax_merge<G>(m, l, acc, ocmp);
+    }
+    // selection branch: the real rows of the selected balls, at full resolution
+    {
+        float m = -INFINITY, l = 0.0f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int t = 0; t < topk; ++t) {
+            const int s = sel[(size_t(g) * H + h) * topk + t];
+            if (s < 0) continue;  // uniform across the warp
+            if (s >= nb) {
+                record_error(&g_attn_status, BT_ERR_INTERNAL);
+                continue;
+            }
+#pragma unroll 2
+            for (int r0 = kslot; r0 < 128; r0 += 2 * KPS) {
+                const int64_t j0 = int64_t(s) * 128 + r0, j1 = j0 + KPS;
+                int32_t row0 = perm ? perm[j0] : int32_t(j0), row1 = perm ? perm[j1] : int32_t(j1);
+                if (row0 >= rows || row1 >= rows) {
+                    record_error(&g_attn_status, BT_ERR_INTERNAL);
+                    row0 = row0 >= rows ? -1 : row0;
+                    row1 = row1 >= rows ? -1 : row1;
+                }
+                const bool ok0 = row0 >= 0, ok1 = row1 >= 0;
+                const uint4 k0 = ok0 ? *reinterpret_cast<const uint4 *>(K + size_t(row0) * rstride + hoff) : zero;
+                const uint4 k1 = ok1 ? *reinterpret_cast<const uint4 *>(K + size_t(row1) * rstride + hoff) : zero;
+                const uint4 w0 = ok0 ? *reinterpret_cast<const uint4 *>(V + size_t(row0) * rstride + hoff) : zero;
+                const uint4 w1 = ok1 ? *reinterpret_cast<const uint4 *>(V + size_t(row1) * rstride + hoff) : zero;
+                const float s0 = logit(k0, ok0), s1 = logit(k1, ok1);
+                float v0[8], v1[8];
+                bf16x8_to_f32(w0, v0);
+                bf16x8_to_f32(w1, v1);
+                softmax_push2(s0, s1, v0, v1, m, l, acc);
+            }
+        }
+        softmax_merge<G>(m, l, acc, oslc);
+    }
+    // gated sum with the ball branch for every real query row of the group
+    for (int r = kslot; r < 128; r += KPS) {
+        int32_t qrow = perm ? perm[int64_t(g) * 128 + r] : int32_t(int64_t(g) * 128 + r);
+        if (qrow >= rows) {
+            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            qrow = -1;
+        }
+        if (qrow < 0) continue;
+        const float *gp = gates + (size_t(qrow) * H + h) * 3;
+        const float g0 = gp[0], g1 = gp[1], g2 = gp[2];
+        float ob[8];
+        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Oball + size_t(qrow) * rstride + hoff), ob);
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int k = 2 * e;
+            const float y0 = g0 * ob[k] + g1 * ocmp[k] + g2 * oslc[k];
+            const float y1 = g0 * ob[k + 1] + g1 * ocmp[k + 1] + g2 * oslc[k + 1];
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(y0, y1);
+            w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+        }
+        *reinterpret_cast<uint4 *>(O + size_t(qrow) * rstride + hoff) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
 struct BsaLayout {
     size_t qbar, kbar, kc, vc, cnt, sel, gates, oball, total;
 };
@@ -518,6 +697,12 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
     bt_status s = launch_tc<D>(Q, K, V, perm, npad, rows, 7, H, oball, st);
     if (s != BT_OK) return s;
     const int64_t items = int64_t(nb) * H;
+    if (p.coarsen_queries) {
+        k_bsa_coarse<D><<<unsigned((items + 3) / 4), 128, 0, st>>>(
+            k, v, perm, rows, H, nb, qbar, kc, vc, cnt, sel, p.topk, gates, oball,
+            1.4426950408889634f / sqrtf(float(D)), static_cast<__nv_bfloat16 *>(O));
+        return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
+    }
     const int64_t grid = items < int64_t(nsm) * BsaPipe<D>::PER_SM ? items : int64_t(nsm) * BsaPipe<D>::PER_SM;
     k_bsa_attn_tc<D><<<unsigned(grid), kTcThreads, BsaPipe<D>::BYTES, st>>>(
         q, k, v, perm, rows, H, nb, kc, vc, cnt, sel, p.topk, gates, oball, 1.4426950408889634f / sqrtf(float(D)),

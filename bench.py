@@ -371,13 +371,19 @@ def suite(bts, dev, steps, flush, peak):
     def ell_step():
         bts.bt_build(c, wl.m, perm=perm, ws=ws)
         bsa_only()
+    def bsa_coarsened():
+        bts.bsa_forward(q, k, v, perm, wl.m, x, wg, topk=8, out=out, ws=bws, coarsen_queries=True)
+
     ms = statistics.mean(timed_graph(ell_step, steps, 3, flush))
     ms_bsa = statistics.mean(timed_graph(bsa_only, steps, 3, flush))
+    ms_coarse = statistics.mean(timed_graph(bsa_coarsened, steps, 3, flush))
     flop = 4 * wl.d * wl.H * (wl.m + wl.n_total // wl.m + 8 * wl.m) * wl.n_total
     res["ellipsoid_bsa"] = {"points": wl.n_total, "layers": 1, "ms_per_step": ms,
                             "points_per_s_per_layer": wl.n_total / (ms / 1e3), "bsa_ms": ms_bsa,
                             "bsa_gflop": flop / 1e9, "bsa_tflops": flop / (ms_bsa / 1e3) / 1e12,
-                            "note": "BSA = ball + compression over 512 ball means + top-8 selection, gated"}
+                            "bsa_query_coarsened_ms": ms_coarse,
+                            "note": "BSA = ball + compression over 512 ball means + top-8 selection, gated; "
+                                    "query-coarsened: compression and selection with each group's pooled query"}
     del q, k, v, x, out, bws
 
     # box + cluster, 1,048,576 points: two layers (original and rotated tree), as the headline step

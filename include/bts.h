@@ -221,10 +221,17 @@ bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const i
  * Coarse tokens and scores are float; attention accumulates in float with
  * P rounded to bf16 for the tensor cores.  A ball with no real point gives
  * no coarse token and is never selected.
+ * p.coarsen_queries: the optional query-coarsening step of the same paper
+ * ("BSA with group compression"): the compression and selection branches
+ * attend with the group's pooled query instead of each query, so all rows of
+ * a group share O_cmp and O_slc (computed once per group and head on the CUDA
+ * cores, softmax in float from the bf16 coarse tokens and K/V rows); the ball
+ * branch and the gates stay per row.
  */
 typedef struct {
     int32_t topk;          /* blocks selected per (group, head) */
     int32_t mask_own_ball; /* nonzero: a group never selects its own ball */
+    int32_t coarsen_queries; /* nonzero: query coarsening, see above */
 } bsa_params;
 
 size_t bsa_workspace_size(int64_t npad, int64_t rows, int32_t m, int32_t H, int32_t d, int32_t topk);

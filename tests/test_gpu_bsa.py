@@ -4,7 +4,9 @@ The block selection is a discrete decision taken from float scores: the GPU
 scores in float32, the oracle in float64.  Selected sets must be equal, except
 where the blocks that differ tie with the k-th best block to within 1e-4 in the
 oracle's own scores; the outputs are then compared with the oracle recomputed
-on the GPU's selection (max-abs 2e-2, bf16 inputs and outputs).
+on the GPU's selection (max-abs 2e-2, bf16 inputs and outputs).  The
+query-coarsening variant (compression and selection with each group's pooled
+query) is compared with the oracle's coarsened BSA the same way.
 """
 import numpy as np
 import pytest
@@ -28,11 +30,12 @@ def _bf(a):
     return _dev(a.view(np.int16)).view(torch.bfloat16)
 
 
-def _run_gpu(q, k, v, perm, x, w, b, topk, mask_own=True):
+def _run_gpu(q, k, v, perm, x, w, b, topk, mask_own=True, coarsen=False):
     nb, H = len(perm) // 128, q.shape[1]
     sel = torch.full((nb, H, max(topk, 1)), -7, dtype=torch.int32, device="cuda")
     o = bts.bsa_forward(_bf(q), _bf(k), _bf(v), _dev(perm), 128, _dev(x), _dev(w),
-                        None if b is None else _dev(b), topk=topk, mask_own_ball=mask_own, sel=sel)
+                        None if b is None else _dev(b), topk=topk, mask_own_ball=mask_own, sel=sel,
+                        coarsen_queries=coarsen)
     assert bts.bt_attention_device_status() == 0
     return o.float().cpu().numpy().astype(np.float64), sel.cpu().numpy()[:, :, :topk]
 
@@ -53,11 +56,11 @@ def _check_selection(gpu_sel, ref, topk):
     return mism
 
 
-def _case(sizes, H, C, seed, topk, mask_own=True, bias=True):
+def _case(sizes, H, C, seed, topk, mask_own=True, bias=True, d=32):
     pts = np.concatenate([workloads.uniform_cloud(s, seed + i) for i, s in enumerate(sizes)])
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
     n = len(pts)
-    q, k, v = workloads.random_qkv(n, H, 32, workloads.BF16, seed)
+    q, k, v = workloads.random_qkv(n, H, d, workloads.BF16, seed)
     g = np.random.Generator(np.random.PCG64(seed))
     x = g.standard_normal((n, C)).astype(np.float32)
     w = (g.standard_normal((C, 3 * H)) / np.sqrt(C)).astype(np.float32)
@@ -66,16 +69,19 @@ def _case(sizes, H, C, seed, topk, mask_own=True, bias=True):
     return q, k, v, perm.cpu().numpy(), x, w, b
 
 
-@pytest.mark.parametrize("sizes,H,topk,mask_own", [([2048], 2, 4, True), ([1500, 700, 2100], 3, 3, True),
-                                                   ([4096], 1, 8, False), ([1024], 2, 0, True),
-                                                   ([300, 40], 2, 5, True)])
-def test_bsa_matches_oracle(orc, sizes, H, topk, mask_own):
-    q, k, v, perm, x, w, b = _case(sizes, H, 24, sum(sizes) + H, topk, mask_own)
-    got, sel = _run_gpu(q, k, v, perm, x, w, b, topk, mask_own)
-    ref = orc.bsa(q, k, v, 128, perm, x, w, b, topk=topk, mask_own=mask_own, branches=True)
+@pytest.mark.parametrize("coarsen", [False, True])
+@pytest.mark.parametrize("sizes,H,topk,mask_own,d", [([2048], 2, 4, True, 32), ([1500, 700, 2100], 3, 3, True, 32),
+                                                     ([4096], 1, 8, False, 32), ([1024], 2, 0, True, 32),
+                                                     ([300, 40], 2, 5, True, 32), ([1500, 900], 2, 3, True, 64),
+                                                     ([2048], 1, 0, False, 64)])
+def test_bsa_matches_oracle(orc, sizes, H, topk, mask_own, d, coarsen):
+    q, k, v, perm, x, w, b = _case(sizes, H, 24, sum(sizes) + H, topk, mask_own, d=d)
+    got, sel = _run_gpu(q, k, v, perm, x, w, b, topk, mask_own, coarsen)
+    ref = orc.bsa(q, k, v, 128, perm, x, w, b, topk=topk, mask_own=mask_own, branches=True, coarsen=coarsen)
     if topk:
         _check_selection(sel, ref, topk)
-        ref = orc.bsa(q, k, v, 128, perm, x, w, b, topk=topk, mask_own=mask_own, sel_in=sel, branches=True)
+        ref = orc.bsa(q, k, v, 128, perm, x, w, b, topk=topk, mask_own=mask_own, sel_in=sel, branches=True,
+                      coarsen=coarsen)
     real = perm[perm >= 0]
     err = np.abs(got[real] - ref["O"][real]).max()
     assert err <= TOL, f"max abs err {err}"
@@ -90,16 +96,19 @@ def test_bsa_selection_pinned_by_exact_ties(orc):
         assert sel[g, 0].tolist() == [blk for blk in range(8) if blk != g][:3]
 
 
-def test_bsa_ellipsoid_full_size_sampled_groups(orc):
+@pytest.mark.parametrize("coarsen", [False, True])
+def test_bsa_ellipsoid_full_size_sampled_groups(orc, coarsen):
     wl = workloads.ellipsoid()
     L = wl.layers[0]
     perm = bts.bt_build(_dev(wl.coords), wl.m).cpu().numpy()
-    got, sel = _run_gpu(L.q, L.k, L.v, perm, wl.extra["x"], wl.extra["w_g"], None, 8)
+    got, sel = _run_gpu(L.q, L.k, L.v, perm, wl.extra["x"], wl.extra["w_g"], None, 8, coarsen=coarsen)
     nb = len(perm) // 128
     groups = np.random.Generator(np.random.PCG64(4)).choice(nb, 12, replace=False)
-    ref = orc.bsa(L.q, L.k, L.v, 128, perm, wl.extra["x"], wl.extra["w_g"], topk=8, branches=True, groups=groups)
+    ref = orc.bsa(L.q, L.k, L.v, 128, perm, wl.extra["x"], wl.extra["w_g"], topk=8, branches=True, groups=groups,
+                  coarsen=coarsen)
     _check_selection(sel, ref, 8)
-    ref = orc.bsa(L.q, L.k, L.v, 128, perm, wl.extra["x"], wl.extra["w_g"], topk=8, sel_in=sel, groups=groups)
+    ref = orc.bsa(L.q, L.k, L.v, 128, perm, wl.extra["x"], wl.extra["w_g"], topk=8, sel_in=sel, groups=groups,
+                  coarsen=coarsen)
     rows = np.concatenate([perm[gi * 128:(gi + 1) * 128] for gi in groups])
     err = np.abs(got[rows] - ref[rows]).max()
     assert err <= TOL, f"max abs err {err}"
