@@ -58,6 +58,10 @@ def _load():
         lib.orc_bsa.argtypes = [P, P, P, ctypes.c_int, P, i64, i64, i32, i32, i32, P, i32, P, P, i32, i32, i32, P,
                                 P, i64, P, P, P, P, P, P, P]
         lib.orc_bsa.restype = ctypes.c_int
+        lib.orc_pool_mean.argtypes = [P, ctypes.c_int, P, i64, i64, i32, i32, P, P]
+        lib.orc_pool_mean.restype = ctypes.c_int
+        lib.orc_unpool.argtypes = [P, P, i64, i64, i32, i32, P]
+        lib.orc_unpool.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -103,7 +107,9 @@ def _dtype_code(a: np.ndarray) -> int:
         return 0
     if a.dtype == np.uint16:
         return 1
-    raise TypeError("Q/K/V must be float32 or raw bfloat16 bits (uint16)")
+    if a.dtype == np.float64:
+        return 2
+    raise TypeError("Q/K/V must be float32, float64 or raw bfloat16 bits (uint16)")
 
 
 def ball_attention(q, k, v, m: int, perm=None, balls=None, out=None):
@@ -178,3 +184,46 @@ def bsa(q, k, v, m: int, perm, x, w_g, b_g=None, topk: int = 8, mask_own: bool =
     if rc != 0:
         raise OracleError(f"orc_bsa failed with status {rc}")
     return out if branches else out["O"]
+
+
+def pool_mean(x, perm, stride: int, npad: int | None = None):
+    """Mean over the real slots of each node `stride` slots wide (see oracle.c, orc_pool_mean).
+    x [rows, ...] float32 / float64 / bf16 bits in original row order.  Returns (xc float64
+    [npad/stride, ...] in coarse slot order, cperm int32 [npad/stride])."""
+    x = np.ascontiguousarray(x)
+    rows = x.shape[0]
+    C = int(np.prod(x.shape[1:]))
+    npad = (rows if perm is None else len(perm)) if npad is None else npad
+    perm_a = None if perm is None else np.ascontiguousarray(perm, dtype=np.int32)
+    xc = np.full((npad // stride,) + x.shape[1:], np.nan)
+    cperm = np.full(npad // stride, -2, np.int32)
+    rc = _load().orc_pool_mean(_ptr(x), _dtype_code(x), _ptr(perm_a), npad, rows, C, stride, _ptr(xc), _ptr(cperm))
+    if rc != 0:
+        raise OracleError(f"orc_pool_mean failed with status {rc}")
+    return xc, cperm
+
+
+def unpool(xc, perm, stride: int, rows: int, out=None):
+    """Copy each node's value back to its real slots' rows (see oracle.c, orc_unpool).  Returns
+    float64 [rows, ...]; rows no slot names stay NaN (or as in ``out``)."""
+    xc = np.ascontiguousarray(xc, dtype=np.float64)
+    C = int(np.prod(xc.shape[1:]))
+    npad = xc.shape[0] * stride if perm is None else len(perm)
+    perm_a = None if perm is None else np.ascontiguousarray(perm, dtype=np.int32)
+    o = np.full((rows,) + xc.shape[1:], np.nan) if out is None else out
+    rc = _load().orc_unpool(_ptr(xc), _ptr(perm_a), npad, rows, C, stride, _ptr(o))
+    if rc != 0:
+        raise OracleError(f"orc_unpool failed with status {rc}")
+    return o
+
+
+def coarse_ball_attention(q, k, v, m: int, perm, stride: int):
+    """Ball attention `log2(stride)` levels up the tree: Q/K/V mean-pooled over nodes of `stride` slots,
+    attention inside balls of m coarse tokens (m*stride slots), and the result copied back to every real
+    row of the node.  Returns float64 [rows, H, d]."""
+    rows = q.shape[0]
+    qc, cperm = pool_mean(q, perm, stride)
+    kc, _ = pool_mean(k, perm, stride)
+    vc, _ = pool_mean(v, perm, stride)
+    oc = ball_attention(qc, kc, vc, m, cperm)
+    return unpool(oc, perm, stride, rows)

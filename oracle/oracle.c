@@ -20,6 +20,10 @@
  *  - thread post on cross-partition exchange (the tree is rotated where Swin
  *    would shift its windows): the rotated layer rebuilds the tree on rotated
  *    coordinates (45 degrees about +z here).
+ *  - same thread, posts 8/N and 9/N: coarsening and refinement of the tree
+ *    keep the ball size of attention fixed; because the points of a node are
+ *    contiguous at every level, pooling to the parent level is a mean over
+ *    consecutive slots and refinement copies a parent back to its children.
  */
 #include <math.h>
 #include <stdint.h>
@@ -158,10 +162,12 @@ void orc_rotate_z(const float *in, int64_t n, float *out)
     }
 }
 
-/* element (row, head, k) of a [rows, H, d] tensor, widened to double */
+/* element (row, head, k) of a [rows, H, d] tensor, widened to double
+   (dtype 0 float, 1 bf16 bits, 2 double) */
 static double widen(const void *p, int dtype, int64_t idx)
 {
     if (dtype == 0) return (double)((const float *)p)[idx];
+    if (dtype == 2) return ((const double *)p)[idx];
     uint32_t u = (uint32_t)((const uint16_t *)p)[idx] << 16;
     float f;
     memcpy(&f, &u, 4);
@@ -439,5 +445,54 @@ int orc_bsa(const void *Q, const void *K, const void *V, int dtype, const int32_
     (void)rows;
     free(qbar); free(kbar); free(vbar); free(tok); free(logit); free(keys); free(vals); free(kc); free(vc); free(sc);
     free(sel); free(krows); free(ob); free(oc); free(os); free(qv);
+    return ORC_OK;
+}
+
+/*
+ * Coarsening to a higher tree level ("Erwin" thread, posts 8/N and 9/N): the
+ * nodes `s` levels up (s = stride, a power of two) hold `stride` consecutive
+ * slots each.  Xc[j, c] = mean of X[perm[slot], c] over the real slots of node
+ * j (slots j*stride .. j*stride+stride-1 with perm >= 0); a node without a real
+ * slot is 0 and gets cperm[j] = -1, otherwise cperm[j] = j.  X is [rows, C] in
+ * original row order (dtype as widen()), Xc [npad/stride, C] in coarse slot
+ * order, cperm may be NULL.  cperm is a valid perm for the coarse level (rows =
+ * npad/stride), so levels chain.
+ */
+int orc_pool_mean(const void *X, int dtype, const int32_t *perm, int64_t npad, int64_t rows, int32_t C,
+                  int32_t stride, double *Xc, int32_t *cperm)
+{
+    if (!X || !Xc || C < 1 || stride < 1 || npad < 1 || npad % stride) return ORC_ERR_ARG;
+    for (int64_t j = 0; j < npad / stride; ++j) {
+        int64_t cnt = 0;
+        for (int32_t c = 0; c < C; ++c) Xc[j * C + c] = 0.0;
+        for (int32_t t = 0; t < stride; ++t) {
+            int64_t slot = j * stride + t, r = perm ? perm[slot] : slot;
+            if (r < 0) continue;
+            if (r >= rows) return ORC_ERR_ARG;
+            ++cnt;
+            for (int32_t c = 0; c < C; ++c) Xc[j * C + c] += widen(X, dtype, r * C + c);
+        }
+        if (cnt)
+            for (int32_t c = 0; c < C; ++c) Xc[j * C + c] /= (double)cnt;
+        if (cperm) cperm[j] = cnt ? (int32_t)j : -1;
+    }
+    return ORC_OK;
+}
+
+/*
+ * Refinement back to the finer level (same posts): every real slot takes the
+ * value of its node `stride` slots wide: X[perm[slot], c] = Xc[slot / stride, c].
+ * Rows that no slot names are left as they are.
+ */
+int orc_unpool(const double *Xc, const int32_t *perm, int64_t npad, int64_t rows, int32_t C, int32_t stride,
+               double *X)
+{
+    if (!X || !Xc || C < 1 || stride < 1 || npad < 1 || npad % stride) return ORC_ERR_ARG;
+    for (int64_t slot = 0; slot < npad; ++slot) {
+        int64_t r = perm ? perm[slot] : slot;
+        if (r < 0) continue;
+        if (r >= rows) return ORC_ERR_ARG;
+        for (int32_t c = 0; c < C; ++c) X[r * C + c] = Xc[(slot / stride) * C + c];
+    }
     return ORC_OK;
 }
