@@ -47,6 +47,11 @@ _SIGS = {
     "bsa_workspace_size": ([_i64, _i64, _i32, _i32, _i32, _i32], _sz),
     "bsa_forward": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _i32, _P, _P, None, _P, _P,
                      _P, _sz, _P], ctypes.c_int),
+    "bt_pool_mean": ([_P, _P, _i64, _i64, _i32, _i32, ctypes.c_int, _P, _P, _P], ctypes.c_int),
+    "bt_unpool": ([_P, _P, _i64, _i64, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
+    "bt_coarse_workspace_size": ([_i64, _i32, _i32, _i32, ctypes.c_int], _sz),
+    "bt_coarse_ball_attention": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _i32, _P, _P, _sz,
+                                  _P], ctypes.c_int),
 }
 
 
@@ -219,6 +224,71 @@ def bt_ball_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: t
     _check("bt_ball_attention",
            _lib.bt_ball_attention(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, rows, m, H, d, dt,
                                   _dptr(out), _stream(stream)))
+    return out
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BT_F32
+    if t.dtype == torch.bfloat16:
+        return BT_BF16
+    raise TypeError("tensors must be float32 or bfloat16")
+
+
+def bt_pool_mean(X: torch.Tensor, perm: torch.Tensor | None, stride: int, out: torch.Tensor | None = None,
+                 cperm: torch.Tensor | None = None, npad: int | None = None, stream=None):
+    """Mean over the real slots of every node `stride` slots wide.  X [rows, ...] in original row order; returns
+    (Xc [npad/stride, ...] in coarse slot order, cperm int32 [npad/stride]: j, or -1 for a node of dummies)."""
+    rows = X.shape[0]
+    C = X[0].numel() if rows else 1
+    if npad is None:
+        npad = perm.numel() if perm is not None else rows
+    nc = npad // stride
+    if out is None:
+        out = torch.empty((nc, *X.shape[1:]), dtype=X.dtype, device=X.device)
+    if cperm is None:
+        cperm = torch.empty(nc, dtype=torch.int32, device=X.device)
+    _check("bt_pool_mean", _lib.bt_pool_mean(_dptr(X), _dptr(perm), npad, rows, C, stride, _dt(X), _dptr(out),
+                                             _dptr(cperm), _stream(stream)))
+    return out, cperm
+
+
+def bt_unpool(Xc: torch.Tensor, perm: torch.Tensor | None, stride: int, X: torch.Tensor, npad: int | None = None,
+              stream=None) -> torch.Tensor:
+    """X[perm[s]] = Xc[s // stride] for every real slot s; X [rows, ...] original row order (written in place)."""
+    rows = X.shape[0]
+    C = X[0].numel() if rows else 1
+    if npad is None:
+        npad = perm.numel() if perm is not None else Xc.shape[0] * stride
+    _check("bt_unpool", _lib.bt_unpool(_dptr(Xc), _dptr(perm), npad, rows, C, stride, _dt(X), _dptr(X),
+                                       _stream(stream)))
+    return X
+
+
+def bt_coarse_workspace_size(npad: int, H: int, d: int, stride: int, dtype: torch.dtype) -> int:
+    return int(_lib.bt_coarse_workspace_size(npad, H, d, stride, BT_F32 if dtype == torch.float32 else BT_BF16))
+
+
+def bt_coarse_ball_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, perm: torch.Tensor | None, m: int,
+                             stride: int, out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                             npad: int | None = None, stream=None) -> torch.Tensor:
+    """Ball attention log2(stride) levels up the tree: Q/K/V pooled to nodes of `stride` slots, attention in balls
+    of m coarse tokens, each node's output copied back to its real rows.  Q/K/V/O [rows, H, d]."""
+    rows, H, d = Q.shape
+    if not (K.dtype == V.dtype == Q.dtype):
+        raise TypeError("Q, K and V must share one dtype")
+    if npad is None:
+        npad = perm.numel() if perm is not None else rows
+    if out is None:
+        out = torch.empty_like(Q)
+    if ws is None:
+        n = bt_coarse_workspace_size(npad, H, d, stride, Q.dtype)
+        if n == 0:
+            raise BtsError("bt_coarse_workspace_size", 1)
+        ws = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    _check("bt_coarse_ball_attention",
+           _lib.bt_coarse_ball_attention(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, rows, m, H, d, _dt(Q),
+                                         stride, _dptr(out), _dptr(ws), ws.numel(), _stream(stream)))
     return out
 
 

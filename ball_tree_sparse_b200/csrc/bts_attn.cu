@@ -3,20 +3,25 @@
 // scaled dot-product attention restricted to every ball of m consecutive
 // tree slots, all balls and heads in parallel.
 //
-// Two kernels:
-//  - k_ball_attn_tc2  bf16, m dividing 128: persistent CTAs over work items
-//                     (128-slot tile, head).  Q/K/V rows are gathered through
-//                     perm with cp.async into the no-swizzle canonical
-//                     tensor-core layouts, a few items ahead; S = QK^T runs on
-//                     tcgen05 (M=128, N=128) into TMEM, the softmax reads S back
-//                     with tcgen05.ld (one row per thread) and writes P (bf16,
-//                     unnormalised) to shared memory, O = PV and the row sums
-//                     (P times a ones column) run on tcgen05 into TMEM, and the
-//                     epilogue scales by 1/rowsum and scatters O through perm.
-//                     Balls smaller than 128 share a tile; keys of other balls
-//                     and dummy keys get weight 0.
+// Three kernels:
+//  - k_ball_attn_pair bf16, m dividing 128, d = 32, even H: one work item is a
+//                     128-slot tile and a pair of heads, one warpgroup per head.
+//                     Q/K/V rows are gathered through perm by TMA (tile::gather4,
+//                     128-byte pieces holding both heads of a row, 128-byte
+//                     swizzle), two stages deep, issued by all eight warps.
+//  - k_ball_attn_tc2  bf16, m dividing 128, any d in {32, 64} and H: persistent
+//                     CTAs over work items (128-slot tile, head), rows gathered
+//                     with cp.async into the canonical no-swizzle layouts.
+//    Both tensor-core kernels run S = QK^T on tcgen05 (M=128, N=128) into
+//    TMEM, read S back with tcgen05.ld (one row per thread), write P (bf16,
+//    unnormalised) back over S in TMEM with tcgen05.st, run O = PV with P as
+//    the TMEM A operand and the row sums as P times a ones column, and scale by
+//    1/rowsum in the epilogue, which scatters O through perm.  Balls smaller
+//    than 128 share a tile; keys of other balls and dummy keys get weight 0.
 //  - k_ball_attn_simt fp32 (and any other shape): one CTA per (ball, head) on
 //                     the CUDA cores, exact two-pass softmax.
+// The BSA kernels (bts_bsa.cuh) and the coarse-level pooling kernels
+// (bts_coarse.cuh) are included into this translation unit.
 #include <cuda_bf16.h>
 
 #include "bts_internal.cuh"
@@ -768,3 +773,5 @@ extern "C" bt_status bt_attention_device_status(void *stream)
     if (h && cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(zero)) != cudaSuccess) return BT_ERR_CUDA;
     return static_cast<bt_status>(h);
 }
+
+#include "bts_coarse.cuh"

@@ -22,6 +22,8 @@
 //                  softmax over chunks of 128 keys (S and P in TMEM, P V and
 //                  the row sums on the tensor core), then the gated sum with
 //                  the ball branch, scattered through perm.
+//   k_bsa_coarse   the query-coarsening variant of the two branches: one warp
+//                  per (group, head) with the pooled query, then the gated sum.
 // This file is included by bts_attn.cu (one translation unit with the ball
 // attention kernel and the attention status word).
 #pragma once

@@ -399,6 +399,38 @@ def suite(bts, dev, steps, flush, peak):
                           "attention_frac_of_measured_hbm": nbytes / (a_ms / 1e3) / 1e9 / peak}
     del st
 
+    # coarser levels: gauss_mix 4 x 16384 on a tree of leaf size 1 (every power-of-two stride is a tree level);
+    # attention one and two levels up: Q/K/V pooled to nodes of 2 or 4 slots, balls of 128 nodes, copied back
+    wl = workloads.gauss_mix()
+    L = wl.layers[0]
+    c = torch.from_numpy(wl.coords).to(dev)
+    q, k, v = (_bf16_dev(t, dev) for t in (L.q, L.k, L.v))
+    ws1 = bts.workspace(wl.offsets, 1, dev)
+    npad = int(sum(bts._padded(int(wl.offsets[i + 1] - wl.offsets[i]), 1) for i in range(wl.batch)))
+    perm1 = torch.empty(npad, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    bts.bt_build_segmented(c, wl.offsets, 1, perm=perm1, ws=ws1)
+    ms_b1 = statistics.mean(timed_graph(lambda: bts.bt_build_segmented(c, wl.offsets, 1, perm=perm1, ws=ws1),
+                                        steps, 3, flush))
+    entry = {"points": wl.n_total, "H": wl.H, "d": wl.d, "m": wl.m, "build_leaf1_ms": ms_b1}
+    hd2 = wl.H * wl.d * 2
+    for stride in (2, 4):
+        cws = torch.empty(bts.bt_coarse_workspace_size(npad, wl.H, wl.d, stride, torch.bfloat16), dtype=torch.uint8,
+                          device=dev)
+
+        def coarse_step(stride=stride, cws=cws):
+            bts.bt_coarse_ball_attention(q, k, v, perm1, wl.m, stride, out=out, ws=cws)
+        cms = statistics.mean(timed_graph(coarse_step, steps, 3, flush))
+        nc = npad // stride
+        # pool: read Q/K/V rows + perm, write 3 coarse tensors + map; coarse attention: read 3, write 1, map;
+        # unpool: read coarse O + perm, write O
+        nbytes = (3 * wl.n_total * hd2 + 4 * npad + 3 * nc * hd2 + 4 * nc) + (4 * nc * hd2 + 4 * nc) + \
+                 (nc * hd2 + 4 * npad + wl.n_total * hd2)
+        entry[f"stride{stride}_ms"] = cms
+        entry[f"stride{stride}_gbs"] = nbytes / (cms / 1e3) / 1e9
+    res["gauss_mix_coarse_levels"] = entry
+    del q, k, v, out, perm1, ws1
+
     # ragged batch of 8 clouds, padded with dummies: segmented build + masked ball attention
     wl = workloads.ragged()
     L = wl.layers[0]

@@ -242,6 +242,55 @@ bt_status bsa_forward(const void *Q, const void *K, const void *V, const int32_t
                       size_t ws_bytes, void *stream);
 
 /*
+ * Coarser tree levels (author's thread on Erwin, posts 8/N and 9/N: the tree
+ * is coarsened and refined while the attention ball keeps its size; the points
+ * of every node are contiguous at every level, so pooling is a mean over
+ * consecutive slots).  A node `stride` slots wide is a tree node when the
+ * tree was built with a leaf size that divides stride (leaf size 1 makes
+ * every power-of-two stride a tree level).
+ *
+ * bt_pool_mean: Xc[j, :] = mean of X[perm[s], :] over the real slots s of
+ * node j (s = j*stride .. j*stride+stride-1, perm[s] >= 0), accumulated in
+ * float and rounded to dt; a node without a real slot gets zeros and
+ * cperm[j] = -1, every other node cperm[j] = j.  cperm is a perm of the
+ * coarse level (rows = npad/stride), so levels chain.
+ *   X      dt [rows, C] device, original row order (perm NULL: slot order,
+ *          rows >= npad)
+ *   perm   int32 [npad] device (slot -> row, -1 dummy) or NULL
+ *   stride power of two dividing npad;  C >= 1 elements per row
+ *   Xc     dt [npad/stride, C] device out, coarse slot order
+ *   cperm  int32 [npad/stride] device out, or NULL
+ * A perm entry >= rows is skipped and recorded as BT_ERR_INTERNAL in the
+ * attention status word (bt_attention_device_status).
+ */
+bt_status bt_pool_mean(const void *X, const int32_t *perm, int64_t npad, int64_t rows, int32_t C, int32_t stride,
+                       bt_dtype dt, void *Xc, int32_t *cperm, void *stream);
+
+/*
+ * bt_unpool: refinement by copy, X[perm[s], :] = Xc[s / stride, :] for every
+ * real slot s.  Rows no slot names are not written.  Arguments as for
+ * bt_pool_mean, with Xc the input and X the output.
+ */
+bt_status bt_unpool(const void *Xc, const int32_t *perm, int64_t npad, int64_t rows, int32_t C, int32_t stride,
+                    bt_dtype dt, void *X, void *stream);
+
+/*
+ * Ball attention log2(stride) levels up the tree: Q, K and V are mean-pooled
+ * to nodes of `stride` slots (one launch), ball attention runs over balls of
+ * m coarse tokens (m*stride slots) with the coarse slot map as perm, and each
+ * node's output is copied back to its real rows of O ([rows, H, d], original
+ * order).  Mean pooling commutes with a linear Q/K/V projection, so this is
+ * the attention of the coarse level's pooled features.  (npad/stride) % m == 0.
+ * ws: bt_coarse_workspace_size() bytes, 256-byte aligned (coarse Q, K, V, O
+ * and the coarse slot map).
+ */
+size_t bt_coarse_workspace_size(int64_t npad, int32_t H, int32_t d, int32_t stride, bt_dtype dt);
+
+bt_status bt_coarse_ball_attention(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
+                                   int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, int32_t stride, void *O,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Device-side status of the attention kernels on the current device:
  * synchronises `stream`, returns BT_OK, BT_ERR_TIMEOUT (a tensor-core
  * completion wait that gave up) or BT_ERR_INTERNAL (a perm entry >= rows),

@@ -63,3 +63,19 @@ def test_argument_errors_before_any_launch(lib):
     assert lib.bt_ball_attention(one, one, one, None, 128, 64, 32, 2, 32, 1, one, None) == 1  # rows < npad
     lib.bt_gather.argtypes = [P, P, ctypes.c_int64, ctypes.c_int32, P, P]
     assert lib.bt_gather(one, one, 10, 0, one, None) == 1                   # row_bytes < 1
+    i64, i32 = ctypes.c_int64, ctypes.c_int32
+    lib.bt_pool_mean.argtypes = [P, P, i64, i64, i32, i32, ctypes.c_int, P, P, P]
+    assert lib.bt_pool_mean(one, one, 96, 96, 8, 3, 1, one, None, None) == 2   # stride not a power of two
+    assert lib.bt_pool_mean(one, one, 96, 96, 8, 64, 1, one, None, None) == 2  # stride does not divide npad
+    assert lib.bt_pool_mean(one, None, 128, 100, 8, 2, 1, one, None, None) == 1  # no perm, rows < npad
+    assert lib.bt_pool_mean(None, one, 128, 128, 8, 2, 1, one, None, None) == 1
+    lib.bt_coarse_workspace_size.argtypes = [i64, i32, i32, i32, ctypes.c_int]
+    lib.bt_coarse_workspace_size.restype = ctypes.c_size_t
+    assert lib.bt_coarse_workspace_size(1024, 2, 32, 4, 1) >= 4 * 256 * 2 * 32 * 2 + 256 * 4
+    assert lib.bt_coarse_workspace_size(1024, 2, 32, 3, 1) == 0
+    lib.bt_coarse_ball_attention.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, ctypes.c_int, i32, P, P,
+                                             ctypes.c_size_t, P]
+    assert lib.bt_coarse_ball_attention(one, one, one, one, 1024, 1024, 128, 2, 32, 1, 16, one, one, 1 << 30,
+                                        None) == 2                          # 64 coarse tokens, ball of 128
+    assert lib.bt_coarse_ball_attention(one, one, one, one, 1024, 1024, 32, 2, 32, 1, 4, one, None, 0,
+                                        None) == 4                          # no workspace

@@ -108,3 +108,20 @@ def test_one_coarse_ball_is_sdpa_over_node_means(orc):
     node_of[perm[perm >= 0]] = np.nonzero(perm >= 0)[0] // stride
     idx = np.cumsum(valid) - 1  # node -> position among valid nodes
     np.testing.assert_allclose(got, oc[idx[node_of]], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("m", [4, 16, 128])
+def test_leaf_size_one_tree_has_the_same_nodes(orc, m):
+    # the split rule above size m does not depend on the leaf size: the nodes of m slots hold the same points,
+    # so ball attention on the deeper tree equals ball attention on the leaf-size-m tree
+    sizes = [1000, 333, 2048]
+    pts = np.concatenate([workloads.uniform_cloud(s, 50 + i) for i, s in enumerate(sizes)])
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    p1, _ = orc.build(pts, 1, offsets)
+    pm, _ = orc.build(pts, m, offsets)
+    assert len(p1) == len(pm)
+    for b in range(len(pm) // m):
+        assert sorted(p1[b * m:(b + 1) * m]) == sorted(pm[b * m:(b + 1) * m])
+    q, k, v = workloads.random_qkv(len(pts), 1, 8, workloads.F32, 51)
+    np.testing.assert_allclose(orc.ball_attention(q, k, v, m, p1), orc.ball_attention(q, k, v, m, pm),
+                               rtol=1e-13, atol=1e-14)
