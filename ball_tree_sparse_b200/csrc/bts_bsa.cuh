@@ -1,7 +1,8 @@
 // Ball Sparse Attention (page: Pith review of "BSA: Ball Sparse Attention for
 // Large-scale Geometries": reading notes and referee report; figure 1 caption).
 // Three branches per query, mixed by per-head sigmoid gates:
-//   ball        - attention inside the query's own ball (k_ball_attn_tc2);
+//   ball        - attention inside the query's own ball (the ball attention
+//                 kernels, into the workspace);
 //   compression - attention over one coarse token per ball, the mean of the
 //                 ball's K and V rows;
 //   selection   - the queries of one group (one ball of 128 slots) share one
@@ -14,15 +15,16 @@
 // Kernels (all on the caller's stream):
 //   k_bsa_means    one CTA per ball: pooled query, coarse key (f32 and bf16)
 //                  and coarse value (bf16), number of real points.
-//   k_bsa_gates    32 rows per CTA, W and the X tile in shared memory.
-//   k_bsa_topk     one warp per (group, head): scores from the pooled query and
-//                  the f32 coarse keys, own ball and empty balls masked, top-k.
+//   k_bsa_gates    one thread per row, W and an X tile in shared memory.
+//   k_bsa_topk     one CTA per (head, 8 groups), one warp per group: scores
+//                  from the pooled query and the f32 coarse keys, own ball and
+//                  empty balls masked, top-k.
 //   k_bsa_attn_tc  persistent tcgen05 kernel over (group, head) items: the
 //                  compression and selection branches as flash-style online
 //                  softmax over chunks of 128 keys (S and P in TMEM, P V and
 //                  the row sums on the tensor core), then the gated sum with
 //                  the ball branch, scattered through perm.
-//   k_bsa_coarse   the query-coarsening variant of the two branches: one warp
+//   k_bsa_coarse   the query-coarsening variant of the two branches: one CTA
 //                  per (group, head) with the pooled query, then the gated sum.
 // This file is included by bts_attn.cu (one translation unit with the ball
 // attention kernel and the attention status word).
@@ -33,24 +35,44 @@ namespace bts {
 constexpr int kBsaMaxTopk = 32;
 constexpr int64_t kBsaMaxBalls = 2048;
 
+// eight bf16 values (one 16-byte load) widened to float
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&f)[8])
+{
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[e]));
+        f[2 * e] = t.x;
+        f[2 * e + 1] = t.y;
+    }
+}
+
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128) k_bsa_means(const __nv_bfloat16 *__restrict__ Q,
-                                                   const __nv_bfloat16 *__restrict__ K,
-                                                   const __nv_bfloat16 *__restrict__ V,
-                                                   const int32_t *__restrict__ perm, int64_t rows, int H,
-                                                   float *__restrict__ qbar, float *__restrict__ kbar,
-                                                   __nv_bfloat16 *__restrict__ kc, __nv_bfloat16 *__restrict__ vc,
-                                                   int32_t *__restrict__ cnt)
+// Ball means: one CTA of 8 warps per ball.  Warp w sums rows w, w+8, ... of
+// the ball; each lane owns 8 consecutive channels (16-byte loads of Q, K and
+// V), so one warp covers 256 channels per row.  The 8 partial sums meet in
+// shared memory.
+constexpr int kMeanWarps = 8;
+
+__global__ void __launch_bounds__(kMeanWarps * 32) k_bsa_means(const __nv_bfloat16 *__restrict__ Q,
+                                                              const __nv_bfloat16 *__restrict__ K,
+                                                              const __nv_bfloat16 *__restrict__ V,
+                                                              const int32_t *__restrict__ perm, int64_t rows,
+                                                              int HD, float *__restrict__ qbar,
+                                                              float *__restrict__ kbar,
+                                                              __nv_bfloat16 *__restrict__ kc,
+                                                              __nv_bfloat16 *__restrict__ vc,
+                                                              int32_t *__restrict__ cnt)
 {
     constexpr int M = 128;
     __shared__ int32_t srow[M];
     __shared__ int s_cnt;
-    const int tid = threadIdx.x;
+    __shared__ float sred[kMeanWarps][3][256];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t b = blockIdx.x;
     if (tid == 0) s_cnt = 0;
     __syncthreads();
-    {
+    if (tid < M) {
         int32_t r = perm ? perm[b * M + tid] : int32_t(b * M + tid);
         if (r >= rows) {
             record_error(&g_attn_status, BT_ERR_INTERNAL);
@@ -58,89 +80,220 @@ __global__ void __launch_bounds__(128) k_bsa_means(const __nv_bfloat16 *__restri
         }
         srow[tid] = r;
         const uint32_t vb = __ballot_sync(0xffffffffu, r >= 0);
-        if ((tid & 31) == 0) atomicAdd(&s_cnt, __popc(vb));
+        if (lane == 0) atomicAdd(&s_cnt, __popc(vb));
     }
     __syncthreads();
     const int n = s_cnt;
-    const int HD = H * D;
     const float inv = n > 0 ? 1.0f / float(n) : 0.0f;
-    for (int t = 2 * tid; t < HD; t += 2 * M) {
-        float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+    for (int c0 = 0; c0 < HD; c0 += 256) {
+        const int ch = c0 + 8 * lane;  // this lane's 8 channels
+        float aq[8], ak[8], av[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) aq[k] = ak[k] = av[k] = 0.0f;
+        if (ch < HD) {
 #pragma unroll 4
-        for (int j = 0; j < M; ++j) {
-            const int32_t r = srow[j];
-            if (r < 0) continue;
-            const size_t off = size_t(r) * HD + t;
-            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(Q + off));
-            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(K + off));
-            const float2 vf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(V + off));
-            q0 += qf.x; q1 += qf.y; k0 += kf.x; k1 += kf.y; v0 += vf.x; v1 += vf.y;
+            for (int j = warp; j < M; j += kMeanWarps) {
+                const int32_t r = srow[j];
+                if (r < 0) continue;
+                const size_t off = size_t(r) * HD + ch;
+                float f[8];
+                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Q + off), f);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) aq[k] += f[k];
+                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(K + off), f);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) ak[k] += f[k];
+                bf16x8_to_f32(*reinterpret_cast<const uint4 *>(V + off), f);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) av[k] += f[k];
+            }
         }
-        const size_t o = size_t(b) * HD + t;
-        qbar[o] = q0 * inv; qbar[o + 1] = q1 * inv;
-        kbar[o] = k0 * inv; kbar[o + 1] = k1 * inv;
-        *reinterpret_cast<__nv_bfloat162 *>(kc + o) = __floats2bfloat162_rn(k0 * inv, k1 * inv);
-        *reinterpret_cast<__nv_bfloat162 *>(vc + o) = __floats2bfloat162_rn(v0 * inv, v1 * inv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            sred[warp][0][8 * lane + k] = aq[k];
+            sred[warp][1][8 * lane + k] = ak[k];
+            sred[warp][2][8 * lane + k] = av[k];
+        }
+        __syncthreads();
+        {
+            const int c = c0 + tid;  // one channel per thread (256 threads)
+            if (c < HD) {
+                float sq = 0.f, sk = 0.f, sv = 0.f;
+#pragma unroll
+                for (int w = 0; w < kMeanWarps; ++w) {
+                    sq += sred[w][0][tid];
+                    sk += sred[w][1][tid];
+                    sv += sred[w][2][tid];
+                }
+                const size_t o = size_t(b) * HD + c;
+                qbar[o] = sq * inv;
+                kbar[o] = sk * inv;
+                kc[o] = __float2bfloat16_rn(sk * inv);
+                vc[o] = __float2bfloat16_rn(sv * inv);
+            }
+        }
+        __syncthreads();  // sred is reused by the next channel block
     }
     if (tid == 0) cnt[b] = n;
 }
 
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_bsa_gates(const float *__restrict__ X, int64_t rows, int C,
-                                                   const float *__restrict__ W, const float *__restrict__ bg, int H,
-                                                   float *__restrict__ gates)
+// Gates: one thread per row, kGateOut outputs at a time in registers.  W is
+// staged once per CTA with its rows padded to a multiple of kGateOut (zeros),
+// so the inner loop is one X value (conflict-free, rows padded by one word)
+// and kGateOut/4 broadcast float4 reads of W per kGateOut FMAs.  X is staged
+// kGateCols columns at a time with coalesced loads.
+constexpr int kGateRows = 128, kGateCols = 64, kGateOut = 24;
+
+static int gate_out_padded(int H) { return (3 * H + kGateOut - 1) / kGateOut * kGateOut; }
+
+static size_t gate_smem_bytes(int C, int H)
+{
+    return (size_t(C) * gate_out_padded(H) + size_t(kGateRows) * (kGateCols + 1)) * 4;
+}
+
+__global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict__ X, int64_t rows, int C,
+                                                         const float *__restrict__ W, const float *__restrict__ bg,
+                                                         int H, int NOP, float *__restrict__ gates)
 {
     extern __shared__ __align__(16) float gsm[];
-    const int NO = 3 * H, CP = C + 1;  // X rows padded by one word against bank conflicts
-    float *sW = gsm, *sX = gsm + C * NO;
+    constexpr int XP = kGateCols + 1;
+    const int NO = 3 * H;
+    float *sW = gsm, *sX = gsm + size_t(C) * NOP;
     const int tid = threadIdx.x;
-    for (int i = tid; i < C * NO; i += 256) sW[i] = W[i];
-    const int64_t r0 = int64_t(blockIdx.x) * 32;
-    for (int i = tid; i < 32 * C; i += 256) {
-        const int rr = i / C, c = i - rr * C;
-        sX[rr * CP + c] = (r0 + rr < rows) ? X[(r0 + rr) * C + c] : 0.0f;
+    {
+        // W rows padded to NOP columns with zeros; loads batched 8 per thread ahead of their stores
+        const int total = C * NO, pad = NOP - NO;
+        for (int i0 = 0; i0 < total; i0 += 8 * kGateRows) {
+            float t[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * kGateRows + tid;
+                t[u] = i < total ? W[i] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * kGateRows + tid;
+                if (i < total) {
+                    const int c = i / NO, j = i - c * NO;
+                    sW[c * NOP + j] = t[u];
+                }
+            }
+        }
+        for (int i = tid; i < C * pad; i += kGateRows) {
+            const int c = i / pad, j = NO + (i - c * pad);
+            sW[c * NOP + j] = 0.0f;
+        }
     }
-    __syncthreads();
-    const int rr = tid >> 3;
-    if (r0 + rr >= rows) return;
-    for (int j = tid & 7; j < NO; j += 8) {
-        float acc = bg ? bg[j] : 0.0f;
-        for (int c = 0; c < C; ++c) acc = fmaf(sX[rr * CP + c], sW[c * NO + j], acc);
-        gates[(r0 + rr) * NO + j] = 1.0f / (1.0f + expf(-acc));
+    const int64_t r0 = int64_t(blockIdx.x) * kGateRows, r = r0 + tid;
+    const bool vec4 = (C % 4) == 0 && (reinterpret_cast<uintptr_t>(X) % 16) == 0;
+    for (int j0 = 0; j0 < NO; j0 += kGateOut) {
+        float acc[kGateOut];
+#pragma unroll
+        for (int j = 0; j < kGateOut; ++j) acc[j] = (bg && j0 + j < NO) ? bg[j0 + j] : 0.0f;
+        for (int c0 = 0; c0 < C; c0 += kGateCols) {
+            const int cw = C - c0 < kGateCols ? C - c0 : kGateCols;
+            __syncthreads();  // W is staged / the previous X tile is consumed
+            if (cw == kGateCols && vec4) {
+                // full tile, float4 loads, all issued before the first store
+                constexpr int U = kGateRows * kGateCols / 4 / kGateRows;  // float4 per thread
+                float4 t[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+                    t[u] = (r0 + rr < rows) ? *reinterpret_cast<const float4 *>(X + (r0 + rr) * C + c0 + 4 * c4)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+                    float *d = sX + rr * XP + 4 * c4;
+                    d[0] = t[u].x; d[1] = t[u].y; d[2] = t[u].z; d[3] = t[u].w;
+                }
+            } else {
+                for (int i = tid; i < kGateRows * cw; i += kGateRows) {
+                    const int rr = i / cw, cc = i - rr * cw;
+                    sX[rr * XP + cc] = (r0 + rr < rows) ? X[(r0 + rr) * C + c0 + cc] : 0.0f;
+                }
+            }
+            __syncthreads();
+            for (int cc = 0; cc < cw; ++cc) {
+                const float x = sX[tid * XP + cc];
+                const float4 *w4 = reinterpret_cast<const float4 *>(sW + size_t(c0 + cc) * NOP + j0);
+#pragma unroll
+                for (int j4 = 0; j4 < kGateOut / 4; ++j4) {
+                    const float4 w = w4[j4];
+                    acc[4 * j4] = fmaf(x, w.x, acc[4 * j4]);
+                    acc[4 * j4 + 1] = fmaf(x, w.y, acc[4 * j4 + 1]);
+                    acc[4 * j4 + 2] = fmaf(x, w.z, acc[4 * j4 + 2]);
+                    acc[4 * j4 + 3] = fmaf(x, w.w, acc[4 * j4 + 3]);
+                }
+            }
+        }
+        if (r < rows) {
+#pragma unroll
+            for (int j = 0; j < kGateOut; ++j)
+                if (j0 + j < NO) gates[r * NO + j0 + j] = 1.0f / (1.0f + expf(-acc[j]));
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(128) k_bsa_topk(const float *__restrict__ qbar, const float *__restrict__ kbar,
-                                                  const int32_t *__restrict__ cnt, int nb, int H, int topk,
-                                                  int mask_own, float scale, int32_t *__restrict__ sel)
+// Group scores and top-k: one CTA of 8 warps per (head, 8 consecutive
+// groups), one warp per group.  The head's coarse keys are staged through
+// shared memory kTopkKeys at a time (rows padded by one word: the lanes read
+// different keys at the same element without bank conflicts) and shared by
+// the 8 groups; each warp keeps its group's nb scores in shared memory and
+// takes the top k by repeated warp argmax.
+constexpr int kTopkWarps = 8, kTopkKeys = 256;
+
+static size_t topk_smem_bytes(int D, int nb)
 {
-    extern __shared__ float ssc[];
+    return (size_t(kTopkKeys) * (D + 1) + size_t(kTopkWarps) * nb) * 4;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTopkWarps * 32) k_bsa_topk(const float *__restrict__ qbar,
+                                                             const float *__restrict__ kbar,
+                                                             const int32_t *__restrict__ cnt, int nb, int H, int topk,
+                                                             int mask_own, float scale, int32_t *__restrict__ sel)
+{
+    extern __shared__ __align__(16) float bsa_tsm[];
+    constexpr int KP = D + 1;
+    float *sK = bsa_tsm, *ssc = bsa_tsm + kTopkKeys * KP;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t item = int64_t(blockIdx.x) * 4 + warp;
-    if (item >= int64_t(nb) * H) return;  // no block-wide synchronisation below
-    const int g = int(item / H), h = int(item - int64_t(g) * H);
+    const int ngb = (nb + kTopkWarps - 1) / kTopkWarps;
+    const int h = int(blockIdx.x) / ngb, g = (int(blockIdx.x) - h * ngb) * kTopkWarps + warp;
+    const bool active = g < nb;
     float *sc = ssc + warp * nb;
     float q[D];
 #pragma unroll
-    for (int k = 0; k < D; ++k) q[k] = qbar[(size_t(g) * H + h) * D + k];
-    const bool gvalid = cnt[g] > 0;
-    for (int b = lane; b < nb; b += 32) {
-        const float4 *kp = reinterpret_cast<const float4 *>(kbar + (size_t(b) * H + h) * D);
-        float acc = 0.0f;
-#pragma unroll
-        for (int k4 = 0; k4 < D / 4; ++k4) {
-            const float4 kv = kp[k4];
-            acc = fmaf(q[4 * k4], kv.x, acc);
-            acc = fmaf(q[4 * k4 + 1], kv.y, acc);
-            acc = fmaf(q[4 * k4 + 2], kv.z, acc);
-            acc = fmaf(q[4 * k4 + 3], kv.w, acc);
+    for (int k = 0; k < D; ++k) q[k] = active ? qbar[(size_t(g) * H + h) * D + k] : 0.0f;
+    const bool gvalid = active && cnt[g] > 0;
+    for (int b0 = 0; b0 < nb; b0 += kTopkKeys) {
+        const int nk = nb - b0 < kTopkKeys ? nb - b0 : kTopkKeys;
+        __syncthreads();  // the previous key tile is consumed
+        for (int i = threadIdx.x; i < nk * (D / 4); i += kTopkWarps * 32) {
+            const int kk = i / (D / 4), u = i - kk * (D / 4);
+            const float4 v = *reinterpret_cast<const float4 *>(kbar + (size_t(b0 + kk) * H + h) * D + 4 * u);
+            float *dst = sK + kk * KP + 4 * u;
+            dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
         }
-        const bool ok = gvalid && cnt[b] > 0 && !(mask_own && b == g);
-        sc[b] = ok ? acc * scale : -INFINITY;
+        __syncthreads();
+        if (active) {
+            for (int kk = lane; kk < nk; kk += 32) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int k = 0; k < D; ++k) acc = fmaf(q[k], sK[kk * KP + k], acc);
+                const int b = b0 + kk;
+                const bool ok = gvalid && cnt[b] > 0 && !(mask_own && b == g);
+                sc[b] = ok ? acc * scale : -INFINITY;
+            }
+        }
     }
+    if (!active) return;  // no block-wide synchronisation below
     __syncwarp();
+    const int64_t item = int64_t(g) * H + h;
     for (int t = 0; t < topk; ++t) {
         float bv = -INFINITY;
         int bi = 0x7fffffff;
@@ -444,17 +597,6 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
 // 8 of its elements (16 bytes of the bf16 row), and keeps its own online
 // softmax (log2 domain); the lane groups merge at the end of each branch.  The
 // gated sum over the group's query rows follows in the same warp.
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 w, float (&f)[8])
-{
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u[e]));
-        f[2 * e] = t.x;
-        f[2 * e + 1] = t.y;
-    }
-}
-
 template <int G>
 __device__ __forceinline__ float lane_group_sum(float s)
 {
@@ -477,47 +619,56 @@ __device__ __forceinline__ void softmax_push2(float s0, float s1, const float (&
     m = mn;
 }
 
-// Merge the lane groups' softmax states (lanes with the same element slice)
-// and normalise: out = sum p v / sum p, zero when no key was valid.
+// Merge the lane groups' softmax states (lanes with the same element slice):
+// afterwards every lane holds the warp's max M, its sum L and its un-normalised
+// accumulator for the lane's element slice, all relative to M.
 template <int G>
-__device__ __forceinline__ void softmax_merge(float m, float l, const float (&acc)[8], float (&out)[8])
+__device__ __forceinline__ void softmax_warp_merge(float &m, float &l, float (&acc)[8])
 {
     float M = m;
 #pragma unroll
     for (int o = G; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const float f = M == -INFINITY ? 0.0f : ex2(m - M);
-    float L = l * f;
+    l *= f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) out[k] = acc[k] * f;
+    for (int k = 0; k < 8; ++k) acc[k] *= f;
 #pragma unroll
     for (int o = G; o < 32; o <<= 1) {
-        L += __shfl_xor_sync(0xffffffffu, L, o);
+        l += __shfl_xor_sync(0xffffffffu, l, o);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) out[k] += __shfl_xor_sync(0xffffffffu, out[k], o);
+        for (int k = 0; k < 8; ++k) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
     }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) out[k] *= inv;
+    m = M;
 }
 
+// One CTA of kCoarseWarps warps per (group, head) item.  The warps split the
+// coarse tokens (by half-steps) and the selected balls (one ball at a time),
+// merge their softmax states through shared memory, and split the group's
+// query rows for the gated sum.
+constexpr int kCoarseWarps = 4;
+
 template <int D>
-__global__ void __launch_bounds__(128) k_bsa_coarse(const __nv_bfloat16 *__restrict__ K,
-                                                    const __nv_bfloat16 *__restrict__ V,
-                                                    const int32_t *__restrict__ perm, int64_t rows, int H, int nb,
-                                                    const float *__restrict__ qbar,
-                                                    const __nv_bfloat16 *__restrict__ kc,
-                                                    const __nv_bfloat16 *__restrict__ vc,
-                                                    const int32_t *__restrict__ cnt, const int32_t *__restrict__ sel,
-                                                    int topk, const float *__restrict__ gates,
-                                                    const __nv_bfloat16 *__restrict__ Oball, float sl2,
-                                                    __nv_bfloat16 *__restrict__ O)
+__global__ void __launch_bounds__(kCoarseWarps * 32) k_bsa_coarse(const __nv_bfloat16 *__restrict__ K,
+                                                                  const __nv_bfloat16 *__restrict__ V,
+                                                                  const int32_t *__restrict__ perm, int64_t rows,
+                                                                  int H, int nb, const float *__restrict__ qbar,
+                                                                  const __nv_bfloat16 *__restrict__ kc,
+                                                                  const __nv_bfloat16 *__restrict__ vc,
+                                                                  const int32_t *__restrict__ cnt,
+                                                                  const int32_t *__restrict__ sel, int topk,
+                                                                  const float *__restrict__ gates,
+                                                                  const __nv_bfloat16 *__restrict__ Oball, float sl2,
+                                                                  __nv_bfloat16 *__restrict__ O)
 {
     constexpr int G = D / 8, KPS = 32 / G;  // lanes per key, keys per half-step
+    constexpr int NW = kCoarseWarps;
+    __shared__ float sM[2][NW], sL[2][NW];
+    __shared__ __align__(16) float sAcc[2][NW][D];
+    __shared__ __align__(16) float sOut[2][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t item = int64_t(blockIdx.x) * 4 + warp;
-    if (item >= int64_t(nb) * H) return;  // no block-wide synchronisation below
+    const int64_t item = blockIdx.x;
     const int g = int(item / H), h = int(item - int64_t(g) * H);
-    const int sub = lane % G, kslot = lane / G;
+    const int sub = lane % G, kslot = lane / G;  // elements [8 sub, 8 sub + 8) of key kslot of each half-step
     const size_t hoff = size_t(h) * D + sub * 8, rstride = size_t(H) * D;
     float q[8];
     {
@@ -532,70 +683,132 @@ __global__ void __launch_bounds__(128) k_bsa_coarse(const __nv_bfloat16 *__restr
         float s = 0.0f;
 #pragma unroll
         for (int k = 0; k < 8; ++k) s = fmaf(q[k], kf[k], s);
-        s = lane_group_sum<G>(s);  // every lane takes part: no early exit before this
+        s = lane_group_sum<G>(s);  // every lane of the warp takes part
         return valid ? s * sl2 : -INFINITY;
+    };
+    auto publish = [&](int br, float m, float l, float (&acc)[8]) {
+        softmax_warp_merge<G>(m, l, acc);
+        if (kslot == 0) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) sAcc[br][warp][sub * 8 + k] = acc[k];
+        }
+        if (lane == 0) {
+            sM[br][warp] = m;
+            sL[br][warp] = l;
+        }
     };
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
 
-    // compression branch: every coarse token of a ball with a real point
-    float ocmp[8], oslc[8];
+    // Loads are batched: BI half-step pairs (2*BI keys per lane) are fetched before any is used, and the
+    // row indices of a batch before its K/V rows, so a batch costs two round trips to memory.
+    constexpr int BI = 2;
+    // compression branch: the coarse tokens of balls with a real point; warp w takes half-step pairs w, w+NW, ...
     {
         float m = -INFINITY, l = 0.0f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int b0 = kslot; b0 - kslot < nb; b0 += 2 * KPS) {
-            const int b1 = b0 + KPS;
-            const bool ok0 = b0 < nb && cnt[b0] > 0, ok1 = b1 < nb && cnt[b1] > 0;
-            const uint4 k0 = ok0 ? *reinterpret_cast<const uint4 *>(kc + size_t(b0) * rstride + hoff) : zero;
-            const uint4 k1 = ok1 ? *reinterpret_cast<const uint4 *>(kc + size_t(b1) * rstride + hoff) : zero;
-            const uint4 w0 = ok0 ? *reinterpret_cast<const uint4 *>(vc + size_t(b0) * rstride + hoff) : zero;
-            const uint4 w1 = ok1 ? *reinterpret_cast<const uint4 *>(vc + size_t(b1) * rstride + hoff) : zero;
-            const float s0 = logit(k0, ok0), s1 = logit(k1, ok1);
-            float v0[8], v1[8];
-            bf16x8_to_f32(w0, v0);
-            bf16x8_to_f32(w1, v1);
-            softmax_push2(s0, s1, v0, v1, m, l, acc);
+        for (int base = 2 * warp * KPS; base < nb; base += BI * 2 * NW * KPS) {
+            uint4 kk[2 * BI], vv[2 * BI];
+            bool ok[2 * BI];
+#pragma unroll
+            for (int u = 0; u < 2 * BI; ++u) {
+                const int b = base + (u >> 1) * 2 * NW * KPS + (u & 1) * KPS + kslot;
+                const bool in = b < nb;
+                ok[u] = in && cnt[b] > 0;  // the coarse rows exist for every ball: loaded regardless
+                kk[u] = in ? *reinterpret_cast<const uint4 *>(kc + size_t(b) * rstride + hoff) : zero;
+                vv[u] = in ? *reinterpret_cast<const uint4 *>(vc + size_t(b) * rstride + hoff) : zero;
+            }
+#pragma unroll
+            for (int u = 0; u < BI; ++u) {
+                const float s0 = logit(kk[2 * u], ok[2 * u]), s1 = logit(kk[2 * u + 1], ok[2 * u + 1]);
+                float v0[8], v1[8];
+                bf16x8_to_f32(vv[2 * u], v0);
+                bf16x8_to_f32(vv[2 * u + 1], v1);
+                softmax_push2(s0, s1, v0, v1, m, l, acc);
+            }
         }
-        softmax_merge<G>(m, l, acc, ocmp);
+        publish(0, m, l, acc);
     }
-    // selection branch: the real rows of the selected balls, at full resolution
+    // selection branch: the real rows of the selected balls; warp w takes balls w, w+NW, ...
     {
+        constexpr int RPL = 128 / KPS;  // rows of a ball per lane
         float m = -INFINITY, l = 0.0f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int t = 0; t < topk; ++t) {
+        for (int t = warp; t < topk; t += NW) {
             const int s = sel[(size_t(g) * H + h) * topk + t];
             if (s < 0) continue;  // uniform across the warp
             if (s >= nb) {
                 record_error(&g_attn_status, BT_ERR_INTERNAL);
                 continue;
             }
-#pragma unroll 2
-            for (int r0 = kslot; r0 < 128; r0 += 2 * KPS) {
-                const int64_t j0 = int64_t(s) * 128 + r0, j1 = j0 + KPS;
-                int32_t row0 = perm ? perm[j0] : int32_t(j0), row1 = perm ? perm[j1] : int32_t(j1);
-                if (row0 >= rows || row1 >= rows) {
-                    record_error(&g_attn_status, BT_ERR_INTERNAL);
-                    row0 = row0 >= rows ? -1 : row0;
-                    row1 = row1 >= rows ? -1 : row1;
+            for (int i0 = 0; i0 < RPL; i0 += 2 * BI) {
+                int32_t rw[2 * BI];
+#pragma unroll
+                for (int u = 0; u < 2 * BI; ++u) {
+                    const int64_t j = int64_t(s) * 128 + kslot + KPS * (i0 + u);
+                    int32_t row = perm ? perm[j] : int32_t(j);
+                    if (row >= rows) {
+                        record_error(&g_attn_status, BT_ERR_INTERNAL);
+                        row = -1;
+                    }
+                    rw[u] = row;
                 }
-                const bool ok0 = row0 >= 0, ok1 = row1 >= 0;
-                const uint4 k0 = ok0 ? *reinterpret_cast<const uint4 *>(K + size_t(row0) * rstride + hoff) : zero;
-                const uint4 k1 = ok1 ? *reinterpret_cast<const uint4 *>(K + size_t(row1) * rstride + hoff) : zero;
-                const uint4 w0 = ok0 ? *reinterpret_cast<const uint4 *>(V + size_t(row0) * rstride + hoff) : zero;
-                const uint4 w1 = ok1 ? *reinterpret_cast<const uint4 *>(V + size_t(row1) * rstride + hoff) : zero;
-                const float s0 = logit(k0, ok0), s1 = logit(k1, ok1);
-                float v0[8], v1[8];
-                bf16x8_to_f32(w0, v0);
-                bf16x8_to_f32(w1, v1);
-                softmax_push2(s0, s1, v0, v1, m, l, acc);
+                uint4 kk[2 * BI], vv[2 * BI];
+#pragma unroll
+                for (int u = 0; u < 2 * BI; ++u) {
+                    kk[u] = rw[u] >= 0 ? *reinterpret_cast<const uint4 *>(K + size_t(rw[u]) * rstride + hoff) : zero;
+                    vv[u] = rw[u] >= 0 ? *reinterpret_cast<const uint4 *>(V + size_t(rw[u]) * rstride + hoff) : zero;
+                }
+#pragma unroll
+                for (int u = 0; u < BI; ++u) {
+                    const float s0 = logit(kk[2 * u], rw[2 * u] >= 0), s1 = logit(kk[2 * u + 1], rw[2 * u + 1] >= 0);
+                    float v0[8], v1[8];
+                    bf16x8_to_f32(vv[2 * u], v0);
+                    bf16x8_to_f32(vv[2 * u + 1], v1);
+                    softmax_push2(s0, s1, v0, v1, m, l, acc);
+                }
             }
         }
-        softmax_merge<G>(m, l, acc, oslc);
+        publish(1, m, l, acc);
     }
-    // gated sum with the ball branch for every real query row of the group
-    for (int r = kslot; r < 128; r += KPS) {
+    __syncthreads();
+    // merge the warps: one thread per (branch, element)
+    if (threadIdx.x < 2 * D) {
+        const int br = threadIdx.x / D, k = threadIdx.x - br * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, sM[br][w]);
+        float L = 0.0f, A = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float f = ex2(sM[br][w] - M);  // a warp without keys has M_w = -inf: weight 0
+                L = fmaf(sL[br][w], f, L);
+                A = fmaf(sAcc[br][w][k], f, A);
+            }
+        }
+        sOut[br][k] = L > 0.0f ? A / L : 0.0f;
+    }
+    __syncthreads();
+    float ocmp[8], oslc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        ocmp[k] = sOut[0][sub * 8 + k];
+        oslc[k] = sOut[1][sub * 8 + k];
+    }
+    // gated sum with the ball branch for every real query row of the group; warp w takes rows w*KPS + kslot, ...
+    constexpr int ITE = 128 / (NW * KPS);
+    int32_t qr[ITE];
+#pragma unroll
+    for (int it = 0; it < ITE; ++it) {
+        const int r = it * NW * KPS + warp * KPS + kslot;
         int32_t qrow = perm ? perm[int64_t(g) * 128 + r] : int32_t(int64_t(g) * 128 + r);
         if (qrow >= rows) {
             record_error(&g_attn_status, BT_ERR_INTERNAL);
             qrow = -1;
         }
+        qr[it] = qrow;
+    }
+#pragma unroll
+    for (int it = 0; it < ITE; ++it) {
+        const int32_t qrow = qr[it];
         if (qrow < 0) continue;
         const float *gp = gates + (size_t(qrow) * H + h) * 3;
         const float g0 = gp[0], g1 = gp[1], g2 = gp[2];
@@ -642,7 +855,7 @@ static bt_status bsa_check(int64_t npad, int64_t rows, int32_t m, int32_t H, int
     if (npad < 1 || rows < 1 || H < 1 || C < 1) return BT_ERR_ARG;
     if (m != 128 || npad % m || (d != 32 && d != 64)) return BT_ERR_SHAPE;
     if (topk < 0 || topk > kBsaMaxTopk || npad / m > kBsaMaxBalls || H > 64 || C > 2048) return BT_ERR_UNSUPPORTED;
-    if (size_t(C) * 3 * H * 4 + size_t(32) * (C + 1) * 4 > 200 * 1024) return BT_ERR_UNSUPPORTED;
+    if (gate_smem_bytes(C, H) > 200 * 1024) return BT_ERR_UNSUPPORTED;
     return BT_OK;
 }
 
@@ -680,7 +893,7 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
                                  int(BsaPipe<D>::BYTES)) ||
             cudaFuncSetAttribute(k_bsa_gates, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ||
             cudaFuncSetAttribute(k_bsa_topk<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(4 * kBsaMaxBalls * 4)))
+                                 int(topk_smem_bytes(D, int(kBsaMaxBalls)))))
             return BT_ERR_CUDA;
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BT_ERR_CUDA;
@@ -690,17 +903,19 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
         }
     }
     const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
-    k_bsa_means<D><<<nb, 128, 0, st>>>(q, k, v, perm, rows, H, qbar, kbar, kc, vc, cnt);
-    const size_t gsmem = (size_t(C) * 3 * H + size_t(32) * (C + 1)) * 4;
-    k_bsa_gates<<<unsigned((rows + 31) / 32), 256, gsmem, st>>>(X, rows, C, Wg, bg, H, gates);
+    k_bsa_means<<<nb, kMeanWarps * 32, 0, st>>>(q, k, v, perm, rows, H * D, qbar, kbar, kc, vc, cnt);
+    k_bsa_gates<<<unsigned((rows + kGateRows - 1) / kGateRows), kGateRows, gate_smem_bytes(C, H), st>>>(
+        X, rows, C, Wg, bg, H, gate_out_padded(H), gates);
     if (p.topk > 0)
-        k_bsa_topk<D><<<unsigned((int64_t(nb) * H + 3) / 4), 128, size_t(4) * nb * 4, st>>>(
+        k_bsa_topk<D><<<unsigned(int64_t(H) * ((nb + kTopkWarps - 1) / kTopkWarps)), kTopkWarps * 32,
+                        topk_smem_bytes(D, nb), st>>>(
             qbar, kbar, cnt, nb, H, p.topk, p.mask_own_ball, 1.0f / sqrtf(float(D)), sel);
-    bt_status s = launch_tc<D>(Q, K, V, perm, npad, rows, 7, H, oball, st);
+    bt_status s = (D == 32 && H % 2 == 0 && rows < 0x7FFFFFFF) ? launch_pair(Q, K, V, perm, npad, rows, 7, H, oball, st)
+                                                               : launch_tc<D>(Q, K, V, perm, npad, rows, 7, H, oball, st);
     if (s != BT_OK) return s;
     const int64_t items = int64_t(nb) * H;
     if (p.coarsen_queries) {
-        k_bsa_coarse<D><<<unsigned((items + 3) / 4), 128, 0, st>>>(
+        k_bsa_coarse<D><<<unsigned(items), kCoarseWarps * 32, 0, st>>>(
             k, v, perm, rows, H, nb, qbar, kc, vc, cnt, sel, p.topk, gates, oball,
             1.4426950408889634f / sqrtf(float(D)), static_cast<__nv_bfloat16 *>(O));
         return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;

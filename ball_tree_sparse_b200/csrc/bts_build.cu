@@ -378,8 +378,24 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
         s_cand[tid] = pp;
         s_ckey[tid] = keys[tid * np + pp];
     }
-    for (int l = 0; l < 4; ++l)
-        for (int i = tid; i < TP; i += NT) sl[l][i] = lin[l * np + tile0 + i];
+    {
+        // the tile's slots of all four lists: every load issued before the first store
+        uint32_t t[4][EPT];
+#pragma unroll
+        for (int l = 0; l < 4; ++l)
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int i = tid + q * NT;
+                t[l][q] = i < TP ? lin[l * np + tile0 + i] : 0u;
+            }
+#pragma unroll
+        for (int l = 0; l < 4; ++l)
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int i = tid + q * NT;
+                if (i < TP) sl[l][i] = t[l][q];
+            }
+    }
     __syncthreads();
     if (tid == 0) {
         int ax = 0;
@@ -463,7 +479,8 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
 // 4. the remaining levels of one node of at most T slots, in shared memory.
 //    Points are renamed to local indices 0..sT-1 in ascending id order (the
 //    node's index list), so the index list itself is the identity and every
-//    list fits in 16 bits.  `loc` is a global scratch array pid -> local index.
+//    list fits in 16 bits.  An id's local index is its rank in the node's
+//    ascending id list, found by binary search in shared memory.
 // ---------------------------------------------------------------------------
 // A local index read from a tail list; out of range only after an invariant broke (then recorded)
 __device__ __forceinline__ uint32_t local_ok(uint32_t v, int sT, uint32_t *status)
@@ -475,8 +492,8 @@ __device__ __forceinline__ uint32_t local_ok(uint32_t v, int sT, uint32_t *statu
 
 template <int NT>
 __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict__ keys,
-                                             const uint32_t *__restrict__ lists, uint32_t *__restrict__ loc,
-                                             int32_t *__restrict__ perm, uint32_t *status)
+                                             const uint32_t *__restrict__ lists, int32_t *__restrict__ perm,
+                                             uint32_t *status)
 {
     constexpr int EPT = 4;  // slots per thread: T <= 1024 runs with 256 threads, T <= 4096 with 1024
     static_assert(kTailMax <= 1024 * EPT && 1024 <= 256 * EPT, "tail slots per thread");
@@ -504,30 +521,54 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
     const int m = P.m;
 
     const uint32_t id_lo = uint32_t(P.pad[b]), id_hi = uint32_t(P.pad[b + 1]);  // ids of this cloud
-    for (int e = tid; e < sT; e += NT) {
-        uint32_t pid = lin[3 * np + seg + e];
-        if (pid < id_lo || pid >= id_hi) {  // never index with a foreign id
-            record_error(status, BT_ERR_INTERNAL);
-            pid = id_lo;
-        } else {
-            loc[pid] = uint32_t(e);
+    {
+        // all list loads of this thread's slots first, then the keys of its ids: two round trips
+        uint32_t pI[EPT], pA[3][EPT], kk[3][EPT];
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = tid + q * NT;
+            const bool ok = e < sT;
+            pI[q] = ok ? lin[3 * np + seg + e] : id_lo;
+#pragma unroll
+            for (int a = 0; a < 3; ++a) pA[a][q] = ok ? lin[a * np + seg + e] : id_lo;
         }
-        ps[e] = pid;
 #pragma unroll
-        for (int a = 0; a < 3; ++a) k3[a * T + e] = keys[a * np + pid];
-        lst[3 * T + e] = uint16_t(e);
-    }
-    __syncthreads();  // loc[] of this node is written (block-wide visibility of global stores)
-    for (int e = tid; e < sT; e += NT) {
-#pragma unroll
-        for (int a = 0; a < 3; ++a) {
-            const uint32_t pid = lin[a * np + seg + e];
-            const uint32_t l = (pid >= id_lo && pid < id_hi) ? loc[pid] : 0xFFFFFFFFu;
-            if (l >= uint32_t(sT) || ps[l] != pid) {  // lists disagree on the node's points
+        for (int q = 0; q < EPT; ++q) {
+            if (pI[q] < id_lo || pI[q] >= id_hi) {  // never index with a foreign id
                 record_error(status, BT_ERR_INTERNAL);
-                lst[a * T + e] = 0;
-            } else {
-                lst[a * T + e] = uint16_t(l);
+                pI[q] = id_lo;
+            }
+#pragma unroll
+            for (int a = 0; a < 3; ++a) kk[a][q] = tid + q * NT < sT ? keys[a * np + pI[q]] : 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = tid + q * NT;
+            if (e < sT) {
+                ps[e] = pI[q];
+#pragma unroll
+                for (int a = 0; a < 3; ++a) k3[a * T + e] = kk[a][q];
+                lst[3 * T + e] = uint16_t(e);
+            }
+        }
+        __syncthreads();  // ps[] holds the node's ids in ascending order
+        // local index of an id = its rank in ps[]: a fixed-length binary search in shared memory
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = tid + q * NT;
+            if (e >= sT) continue;
+#pragma unroll
+            for (int a = 0; a < 3; ++a) {
+                const uint32_t pid = pA[a][q];
+                int lo = 0;
+#pragma unroll
+                for (int step = kTailMax / 2; step > 0; step >>= 1)
+                    if (lo + step < sT && ps[lo + step] <= pid) lo += step;
+                if (ps[lo] != pid) {  // lists disagree on the node's points
+                    record_error(status, BT_ERR_INTERNAL);
+                    lo = 0;
+                }
+                lst[a * T + e] = uint16_t(lo);
             }
         }
     }
@@ -704,11 +745,10 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
         uint32_t *lout = lists + size_t((lev + 1) & 1) * 4 * np;
         k_level<<<unsigned(tiles), kLevelThreads, 0, st>>>(P, lev, keys, lin, lout, lstat, counters, status);
     }
-    // the sort buffers are dead after the last radix pass: reuse one as the pid -> local index map
     if (P.T <= 1024)
-        k_tail<256><<<P.tail0[P.B], 256, tail_smem, st>>>(P, keys, lists, sk, perm, status);
+        k_tail<256><<<P.tail0[P.B], 256, tail_smem, st>>>(P, keys, lists, perm, status);
     else
-        k_tail<1024><<<P.tail0[P.B], 1024, tail_smem, st>>>(P, keys, lists, sk, perm, status);
+        k_tail<1024><<<P.tail0[P.B], 1024, tail_smem, st>>>(P, keys, lists, perm, status);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 

@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import hashlib
 import json
 import math
 import os
@@ -41,6 +42,31 @@ import workloads  # noqa: E402
 METRIC = "points/sec per layer (tree build + ball attention) at N=65,536; % roofline"
 UNIT = "points/s"
 LAYERS = 2
+
+# DRAM traffic of one launch of the dominant kernel on this workload (ncu dram__bytes_read.sum +
+# dram__bytes_write.sum, profiles/k_ball_attn_pair_gauss_mix.md) and the hash of the attention source it was
+# taken on (code lines only).  Reported only while that source is unchanged; null otherwise.
+ROOF_KERNEL = "k_ball_attn_pair"
+ROOF_TRAFFIC = {"bytes": 109482496,
+                "source_sha256": "984c47dc54783ed8e9c64cbf8d740c4c0f819f23ad821c6ce4e909e609924a47"}
+_ATTN_SOURCES = ("ball_tree_sparse_b200/csrc/bts_attn.cu", "ball_tree_sparse_b200/csrc/bts_tc.cuh")
+
+
+def attention_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in _ATTN_SOURCES:
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), rel)) as f:
+            for line in f:
+                t = line.strip()
+                if t and not t.startswith("//"):
+                    h.update(t.encode())
+    return h.hexdigest()
+
+
+def roof_traffic():
+    if ROOF_TRAFFIC["bytes"] is None or ROOF_TRAFFIC["source_sha256"] != attention_source_hash():
+        return None
+    return ROOF_TRAFFIC["bytes"]
 
 
 def parse():
@@ -185,9 +211,11 @@ class Step:
         for _ in range(3):
             self.body()
         torch.cuda.synchronize()
-        self.graph = torch.cuda.CUDAGraph()
+        self.graph = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(self.graph):
             self.body(capturing=True)
+        self.graph.instantiate()
+        self.launches = graph_kernel_nodes(self.rt, self.graph)
         torch.cuda.synchronize()
 
     def times(self):
@@ -210,15 +238,43 @@ def aggregate_value(world: int, layers: int, points: int, steps: int, total_ms: 
     return world * layers * points * steps / (total_ms / 1e3)
 
 
+def graph_kernel_nodes(rt, graph) -> int | None:
+    """Kernel nodes (cudaGraphNodeTypeKernel) of a captured step graph: every one is a launch of this
+    library's kernels (the step calls nothing else; memset and event nodes are not kernels)."""
+    try:
+        h = ctypes.c_void_p(graph.raw_cuda_graph())
+        rt.cudaGraphGetNodes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_size_t)]
+        rt.cudaGraphNodeGetType.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]
+        n = ctypes.c_size_t(0)
+        if rt.cudaGraphGetNodes(h, None, ctypes.byref(n)) != 0:
+            return None
+        nodes = (ctypes.c_void_p * n.value)()
+        if rt.cudaGraphGetNodes(h, nodes, ctypes.byref(n)) != 0:
+            return None
+        count = 0
+        for nd in nodes[:n.value]:
+            t = ctypes.c_int(-1)
+            if rt.cudaGraphNodeGetType(ctypes.c_void_p(nd), ctypes.byref(t)) != 0:
+                return None
+            count += t.value == 0
+        return count
+    except (AttributeError, RuntimeError, OSError):
+        return None
+
+
 def kernels_per_step(wl) -> int:
-    """Launches of this library's kernels in one step (memsets excluded)."""
+    """Launches of this library's kernels in one step (memsets excluded), from the build plan's rule for the
+    tail size T: m * 2^t with t = log2(Npad_all / (296 m)) clamped to [max(2, log2(512/m)), log2(4096/m)]."""
     m = wl.m
-    T = m << int(math.floor(math.log2(4096 // m)))
-    t = int(math.log2(T // m))
-    nlev = 0
-    for b in range(wl.batch):
-        npad = workloads.padded_size(int(wl.offsets[b + 1] - wl.offsets[b]), m)
-        nlev = max(nlev, int(math.log2(npad // m)) - t)
+
+    def ilog2(v):
+        return max(0, int(v).bit_length() - 1)
+    npads = [workloads.padded_size(int(wl.offsets[b + 1] - wl.offsets[b]), m) for b in range(wl.batch)]
+    tmax = ilog2(4096 // m)
+    tmin = min(tmax, max(2, ilog2(512 // m) if m <= 512 else 0))
+    t = ilog2(sum(npads) // (296 * m)) if sum(npads) >= 296 * m else 0
+    t = max(min(t, tmax), tmin)
+    nlev = max(max(0, ilog2(npad // m) - t) for npad in npads)
     build = 1 + 4 + nlev + 1
     return 2 * build + 2 + 3
 
@@ -542,13 +598,13 @@ def main():
         "config": {"workload": "gauss_mix 4x16384 (m=128, H=8, d=32), layers: original + rotated tree",
                    "global_batch": 4 * world, "seq_len": 16384, "parallelism": f"replicas{world}",
                    "l2": "256 MB write between timed steps", "graph": "one CUDA graph per step"},
-        "roofline": {"bound": "hbm", "kernel": "k_ball_attn_tc2<32>", "achieved": achieved, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": ROOF_KERNEL, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
-                     "bytes_per_launch": attn_bytes, "avg_launch_ms": attn_avg_ms, "traffic": None},
+                     "bytes_per_launch": attn_bytes, "avg_launch_ms": attn_avg_ms, "traffic": roof_traffic()},
         "breakdown_ms_per_step": {k: v / args.steps for k, v in parts.items()},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": kernels_per_step(wl) * args.steps,
+        "gpu_launches": (st.launches if st.launches is not None else kernels_per_step(wl)) * args.steps,
         "clocks": clocks.summary(),
     }
     if rank == 0 and not args.no_suite:

@@ -212,8 +212,10 @@ bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const i
  *   Q, K, V, perm, npad, rows  as for bt_ball_attention (bf16 only)
  *   m        128 (the ball, the query group and one selected block)
  *   d        32 or 64;  H <= 64;  npad / m <= 2048 balls;  0 <= topk <= 32
- *   X        float [rows, C] gate features (original row order), C <= 2048
- *   Wg       float [C, 3H] gate weights;  bg  float [3H] or NULL (zero)
+ *   X        float [rows, C] gate features (original row order)
+ *   Wg       float [C, 3H] gate weights;  bg  float [3H] or NULL (zero);
+ *            W is staged in shared memory: C * (3H rounded up to 24) * 4
+ *            bytes + 33,280 must not exceed 200 KiB (BT_ERR_UNSUPPORTED)
  *   O        bf16 [rows, H, d] out
  *   sel_out  int32 [npad/m, H, topk] out (may be NULL): the selected balls per
  *            (group, head), -1 where fewer than topk balls can be selected
