@@ -382,10 +382,27 @@ struct PairPipe {
     static constexpr uint32_t ONES_OFF = NS * STAGE;
     static constexpr uint32_t BYTES = ONES_OFF + 16 * 128 * 2 + 1024;
     static constexpr uint32_t COLS = 256;
-    static constexpr int THREADS = 256;
+    static constexpr int CONSUMERS = 256;               // two warpgroups, one per head of the pair
+    static constexpr int PRODUCERS = 64;                // two warps that gather the next item's rows
+    static constexpr int THREADS = CONSUMERS + PRODUCERS;
     static constexpr int PER_SM = 2;
 };
 
+// Named barrier of one head's warpgroup (ids 1 and 2; 3 is the producers').
+__device__ __forceinline__ void head_sync(int hj)
+{
+    if (hj == 0)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+    else
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+}
+
+// Warps 0-7 compute: warpgroup j (warps 4j..4j+3) owns head j of the pair and runs on its own (its first
+// thread issues that head's MMAs, its own mbarriers and named barrier), so one head's MMA waits overlap
+// the other head's softmax.  Warps 8-9 only load perm and issue the TMA gathers of the next item into the
+// free stage, so the gathers' issue cost is off the compute path.  Stage s is full when its transaction
+// count completes (sFull[s]) and free again when both heads' MMAs that read it have completed (sEmpty[s],
+// two arrivals, each armed by tcgen05.commit after that head's P V product).
 __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     k_ball_attn_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ perm, int64_t npad,
@@ -399,13 +416,11 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     constexpr uint32_t IDESC_O = idesc_bf16(D, true);
     constexpr uint32_t IDESC_SUM = idesc_bf16(16, false);
     extern __shared__ __align__(1024) uint8_t psm[];
-    __shared__ uint32_t sKeyMask[4];
-    __shared__ __align__(8) uint64_t sBarS, sBarO, sFull[NS];
+    __shared__ uint32_t sKeyMask[2][4];
+    __shared__ __align__(8) uint64_t sBarS[2], sBarO[2], sFull[NS], sEmpty[NS];
     __shared__ uint32_t sTmem;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int hj = warp >> 2;          // head of the pair this warpgroup owns
-    const int r = tid & 127;           // query row (TMEM lane) this thread owns
     const int m = 1 << lm;
     const int HP = H >> 1;
     const uint32_t base = (smem_u32(psm) + 1023u) & ~1023u;  // swizzled tiles need 1024-byte alignment
@@ -424,10 +439,14 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarS)) : "memory");
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarO)) : "memory");
-        for (int s0 = 0; s0 < NS; ++s0)
+        for (int j = 0; j < 2; ++j) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarS[j])) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarO[j])) : "memory");
+        }
+        for (int s0 = 0; s0 < NS; ++s0) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sFull[s0])) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(smem_u32(&sEmpty[s0])) : "memory");
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     fence_async_smem();
@@ -435,10 +454,8 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sTmem;
-    const uint32_t tS = tmem + 128 * hj, tO = tS + 64, tSum = tS + 96;  // this warpgroup's columns
-    const uint32_t barS = smem_u32(&sBarS), barO = smem_u32(&sBarO);
-    const uint32_t lanebase = uint32_t((warp & 3) * 32) << 16;
     const int32_t oob = rows < 0x7FFFFFFF ? int32_t(rows) : -1;  // a row outside the tensor reads zeros
+    const int64_t first = blockIdx.x, stride = gridDim.x;
 
     auto raw_row = [&](int64_t item, int rr) -> int32_t {  // items < 2^31: 32-bit index arithmetic
         if (item >= items) return -1;
@@ -453,165 +470,177 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         }
         return row;
     };
-    // all eight warps share the gathers of an item: lane l < 4 of warp w takes rows 4g..4g+3, g = 4w + l, of
-    // Q, K and V (both heads).  The transaction count is armed once, before any of them can complete.
-    auto issue = [&](int64_t item, int stage, const int32_t (&rw)[4]) {
-        if (item >= items) return;  // uniform across the CTA
-        const uint32_t bar = smem_u32(&sFull[stage]);
-        if (tid == 0) mbar_expect_tx(bar, L::STAGE);
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (lane >= 4) return;
-        int32_t rr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int32_t x = check(rw[i]);
-            rr[i] = x >= 0 ? x : oob;
-        }
-        const int32_t col = int32_t(uint32_t(item) % uint32_t(HP)) * 2 * D;
-        const uint32_t dq = base + stage * L::STAGE + (4 * warp + lane) * 4 * L::RB;
-        tma_gather4(dq, &tmQ, col, rr[0], rr[1], rr[2], rr[3], bar);
-        tma_gather4(dq + L::TILE, &tmK, col, rr[0], rr[1], rr[2], rr[3], bar);
-        tma_gather4(dq + 2 * L::TILE, &tmV, col, rr[0], rr[1], rr[2], rr[3], bar);
-    };
-    auto load_rows = [&](int64_t item, int32_t (&rr)[4]) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) rr[i] = lane < 4 ? raw_row(item, 4 * (4 * warp + lane) + i) : -1;
-    };
 
-    const int64_t first = blockIdx.x, stride = gridDim.x;
-    int32_t nrows[4];
-    load_rows(first, nrows);
-    issue(first, 0, nrows);
-    load_rows(first + stride, nrows);
-    int32_t qcur = check(raw_row(first, r)), qnext = raw_row(first + stride, r);
-    bool ok = true;
-    int it = 0;
-    for (int64_t item = first; item < items; item += stride, ++it) {
-        const int stage = it & 1;
-        issue(item + stride, stage ^ 1, nrows);
-        load_rows(item + 2 * stride, nrows);  // consumed one iteration later
-        const int32_t qafter = raw_row(item + 2 * stride, r);
-        if (warp < 4) {
-            const uint32_t kb = __ballot_sync(0xffffffffu, qcur >= 0);
-            if (lane == 0) sKeyMask[warp] = kb;
-        }
-        ok = ok && mbar_wait(smem_u32(&sFull[stage]), (it >> 1) & 1);
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        const uint32_t sq = base + stage * L::STAGE, sk = sq + L::TILE, sv = sk + L::TILE;
-        if (tid == 0 && ok) {
+    if (warp >= 8) {
+        // ---------------- producers: lanes 0-15 of warp 8 + w take rows 4g..4g+3, g = 16 w + lane ----------------
+        const int pw = warp - 8, g = 16 * pw + lane;
+        auto load_rows = [&](int64_t item, int32_t (&rr)[4]) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+            for (int i = 0; i < 4; ++i) rr[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
+        };
+        int32_t nrows[4];
+        load_rows(first, nrows);
+        bool pok = true;
+        int it = 0;
+        for (int64_t item = first; item < items; item += stride, ++it) {
+            const int stage = it & (NS - 1);
+            int32_t rr[4];
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16(tmem + 128 * j, smem_desc_sw(sq + 64 * j + 32 * kk, 16, SBO8, SW128),
-                             smem_desc_sw(sk + 64 * j + 32 * kk, 16, SBO8, SW128), IDESC_S, kk > 0);
-            mma_commit(barS);
+            for (int i = 0; i < 4; ++i) {
+                const int32_t x = check(nrows[i]);
+                rr[i] = x >= 0 ? x : oob;
+            }
+            load_rows(item + stride, nrows);  // consumed by the next iteration
+            if (it >= NS) pok = pok && mbar_wait(smem_u32(&sEmpty[stage]), ((it / NS) + 1) & 1);
+            const uint32_t bar = smem_u32(&sFull[stage]);
+            if (tid == 8 * 32) mbar_expect_tx(bar, L::STAGE);
+            asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");  // armed before any gather lands
+            if (lane < 16) {
+                const int32_t col = int32_t(uint32_t(item) % uint32_t(HP)) * 2 * D;
+                const uint32_t dq = base + stage * L::STAGE + g * 4 * L::RB;
+                tma_gather4(dq, &tmQ, col, rr[0], rr[1], rr[2], rr[3], bar);
+                tma_gather4(dq + L::TILE, &tmK, col, rr[0], rr[1], rr[2], rr[3], bar);
+                tma_gather4(dq + 2 * L::TILE, &tmV, col, rr[0], rr[1], rr[2], rr[3], bar);
+            }
         }
-        ok = ok && mbar_wait(barS, it & 1);
-        tc_fence_after();
+        (void)pok;
+    } else {
+        // ---------------- consumers ----------------
+        const int hj = warp >> 2;  // head of the pair this warpgroup owns
+        const int r = tid & 127;   // query row (TMEM lane) this thread owns
+        const bool issuer = r == 0;
+        const uint32_t tS = tmem + 128 * hj, tO = tS + 64, tSum = tS + 96;  // this warpgroup's columns
+        const uint32_t barS = smem_u32(&sBarS[hj]), barO = smem_u32(&sBarO[hj]);
+        const uint32_t lanebase = uint32_t((warp & 3) * 32) << 16;
+        int32_t qcur = check(raw_row(first, r)), qnext = raw_row(first + stride, r);
+        bool ok = true;
+        int it = 0;
+        for (int64_t item = first; item < items; item += stride, ++it) {
+            const int stage = it & (NS - 1);
+            const int32_t qafter = raw_row(item + 2 * stride, r);
+            {
+                const uint32_t kb = __ballot_sync(0xffffffffu, qcur >= 0);
+                if (lane == 0) sKeyMask[hj][warp & 3] = kb;
+            }
+            ok = ok && mbar_wait(smem_u32(&sFull[stage]), (it / NS) & 1);
+            tc_fence_before();
+            head_sync(hj);
+            tc_fence_after();
+            const uint32_t sq = base + stage * L::STAGE, sk = sq + L::TILE, sv = sk + L::TILE;
+            if (issuer) {
+                if (ok) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        mma_bf16(tS, smem_desc_sw(sq + 64 * hj + 32 * kk, 16, SBO8, SW128),
+                                 smem_desc_sw(sk + 64 * hj + 32 * kk, 16, SBO8, SW128), IDESC_S, kk > 0);
+                }
+                mma_commit(barS);  // arrives at once when nothing was issued: a failed wait ends quickly
+            }
+            ok = ok && mbar_wait(barS, it & 1);
+            tc_fence_after();
 
-        // softmax of row r of head hj; keys outside its ball or dummy get weight 0
-        const int ball0 = (r >> lm) << lm;
-        uint32_t cmask[4];
+            // softmax of row r of head hj; keys outside its ball or dummy get weight 0
+            const int ball0 = (r >> lm) << lm;
+            uint32_t cmask[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t bm;
-            if (m >= 32)
-                bm = (c * 32 >= ball0 && c * 32 < ball0 + m) ? 0xffffffffu : 0u;
-            else
-                bm = (c * 32 <= ball0 && ball0 < c * 32 + 32) ? (((1u << m) - 1u) << (ball0 - c * 32)) : 0u;
-            cmask[c] = bm & sKeyMask[c];
-        }
-        float mx = -INFINITY;
+            for (int c = 0; c < 4; ++c) {
+                uint32_t bm;
+                if (m >= 32)
+                    bm = (c * 32 >= ball0 && c * 32 < ball0 + m) ? 0xffffffffu : 0u;
+                else
+                    bm = (c * 32 <= ball0 && ball0 < c * 32 + 32) ? (((1u << m) - 1u) << (ball0 - c * 32)) : 0u;
+                cmask[c] = bm & sKeyMask[hj][c];
+            }
+            float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
-                uint32_t v[32];
-                tmem_ld32(tS + lanebase + c * 32, v);
-                if (cmask[c] == 0xffffffffu) {
+            for (int c = 0; c < 4; ++c) {
+                if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
+                    uint32_t v[32];
+                    tmem_ld32(tS + lanebase + c * 32, v);
+                    if (cmask[c] == 0xffffffffu) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) mx = fmax3(mx, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                        for (int j = 0; j < 32; j += 2) mx = fmax3(mx, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if ((cmask[c] >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]));
+                    }
+                }
+            }
+            const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+                if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
+                    uint32_t v[32];
+                    tmem_ld32(tS + lanebase + c * 32, v);
+                    const uint32_t cm = cmask[c];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+                        float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
+                        if (cm != 0xffffffffu) {
+                            p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
+                            p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                        }
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                    }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if ((cmask[c] >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]));
+                    for (int j = 0; j < 16; ++j) pk[j] = 0u;
                 }
+                tmem_st16(tS + lanebase + c * 16, pk);
             }
-        }
-        const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
+            tmem_wait_st();
+            tc_fence_before();
+            head_sync(hj);
+            tc_fence_after();
+            if (issuer) {
+                if (ok) {
+                    const uint32_t so1 = base + L::ONES_OFF;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t pk[16];
-            if (__any_sync(0xffffffffu, cmask[c] != 0u)) {
-                uint32_t v[32];
-                tmem_ld32(tS + lanebase + c * 32, v);
-                const uint32_t cm = cmask[c];
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-                    float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
-                    if (cm != 0xffffffffu) {
-                        p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
-                        p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t tp = tS + kk * 8;
+                        mma_bf16_ts(tO, tp, smem_desc_sw(sv + 64 * hj + kk * 16 * L::RB, 16, SBO8, SW128), IDESC_O,
+                                    kk > 0);
+                        mma_bf16_ts(tSum, tp, smem_desc(so1 + kk * 256, 128, ONES_SBO), IDESC_SUM, kk > 0);
                     }
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
                 }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                mma_commit(barO);
+                mma_commit(smem_u32(&sEmpty[stage]));  // this head is done with the stage
             }
-            tmem_st16(tS + lanebase + c * 16, pk);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0 && ok) {
-            const uint32_t so1 = base + L::ONES_OFF;
+            ok = ok && mbar_wait(barO, it & 1);
+            tc_fence_after();
+            if (ok) {
+                uint32_t sum_bits, o[32];
+                tmem_ld1_nowait(tSum + lanebase, sum_bits);
+                tmem_ld32_nowait(tO + lanebase, o);
+                tmem_wait_ld();
+                const float sum = __uint_as_float(sum_bits);
+                const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+                const int h = int(uint32_t(item) % uint32_t(HP)) * 2 + hj;
+                if (qcur >= 0) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qcur) * H + h) * D);
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+                    for (int t = 0; t < D / 8; ++t) {
+                        uint32_t w[4];
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t tp = tmem + 128 * j + kk * 8;
-                    mma_bf16_ts(tmem + 128 * j + 64, tp, smem_desc_sw(sv + 64 * j + kk * 16 * L::RB, 16, SBO8, SW128),
-                                IDESC_O, kk > 0);
-                    mma_bf16_ts(tmem + 128 * j + 96, tp, smem_desc(so1 + kk * 256, 128, ONES_SBO), IDESC_SUM, kk > 0);
-                }
-            mma_commit(barO);
-        }
-        ok = ok && mbar_wait(barO, it & 1);
-        tc_fence_after();
-        if (ok) {
-            uint32_t sum_bits, o[32];
-            tmem_ld1_nowait(tSum + lanebase, sum_bits);
-            tmem_ld32_nowait(tO + lanebase, o);
-            tmem_wait_ld();
-            const float sum = __uint_as_float(sum_bits);
-            const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
-            const int h = int(uint32_t(item) % uint32_t(HP)) * 2 + hj;
-            if (qcur >= 0) {
-                uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qcur) * H + h) * D);
-#pragma unroll
-                for (int t = 0; t < D / 8; ++t) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * t + 2 * e]) * inv,
-                                                                        __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
-                        w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * t + 2 * e]) * inv,
+                                                                            __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
+                            w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                        }
+                        dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
+            qcur = check(qnext);
+            qnext = qafter;
+            tc_fence_before();
+            head_sync(hj);  // this head's S/P and O are free again
+            tc_fence_after();
         }
-        qcur = check(qnext);
-        qnext = qafter;
-        tc_fence_before();
-        __syncthreads();  // every read of S/P, O and of this stage is done before they are reused
-        tc_fence_after();
     }
     tc_fence_before();
     __syncthreads();
