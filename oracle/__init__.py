@@ -62,6 +62,8 @@ def _load():
         lib.orc_pool_mean.restype = ctypes.c_int
         lib.orc_unpool.argtypes = [P, P, i64, i64, i32, i32, P]
         lib.orc_unpool.restype = ctypes.c_int
+        lib.orc_project.argtypes = [P, ctypes.c_int, P, ctypes.c_int, i64, i32, i32, i32, P, P, P]
+        lib.orc_project.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -227,3 +229,22 @@ def coarse_ball_attention(q, k, v, m: int, perm, stride: int):
     vc, _ = pool_mean(v, perm, stride)
     oc = ball_attention(qc, kc, vc, m, cperm)
     return unpool(oc, perm, stride, rows)
+
+
+def project(x, w, H: int, d: int):
+    """Q, K, V = X W in float64 (see oracle.c, orc_project).  x [rows, C], w [C, 3*H*d] (float32, float64 or bf16
+    bits); returns three float64 arrays [rows, H, d]."""
+    x = np.ascontiguousarray(x)
+    w = np.ascontiguousarray(w)
+    rows, C = x.shape
+    q, k, v = (np.full((rows, H, d), np.nan) for _ in range(3))
+    rc = _load().orc_project(_ptr(x), _dtype_code(x), _ptr(w), _dtype_code(w), rows, C, H, d, _ptr(q), _ptr(k), _ptr(v))
+    if rc != 0:
+        raise OracleError(f"orc_project failed with status {rc}")
+    return q, k, v
+
+
+def projected_ball_attention(x, w, H: int, d: int, m: int, perm, balls=None):
+    """Ball attention of the projected features: Q, K, V = X W (float64), then attention inside the balls."""
+    q, k, v = project(x, w, H, d)
+    return ball_attention(q, k, v, m, perm, balls=balls)

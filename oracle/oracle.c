@@ -496,3 +496,26 @@ int orc_unpool(const double *Xc, const int32_t *perm, int64_t npad, int64_t rows
     }
     return ORC_OK;
 }
+
+/*
+ * Projection of features to queries, keys and values (the linear maps that
+ * precede ball attention in every Erwin / BSA attention block; the Erwin
+ * thread's posts 7/N-9/N apply attention to projected features of the
+ * points).  Y = X W in double: X [rows, C] (dtype as widen()), W [C, 3*H*d]
+ * (dtype as widen()), columns [0, Hd) give Q, [Hd, 2Hd) K, [2Hd, 3Hd) V, head h
+ * at h*d .. h*d+d-1 of each block.  Q, K, V out: double [rows, H, d].
+ */
+int orc_project(const void *X, int xdtype, const void *W, int wdtype, int64_t rows, int32_t C, int32_t H, int32_t d,
+                double *Q, double *K, double *V)
+{
+    if (!X || !W || !Q || !K || !V || rows < 0 || C < 1 || H < 1 || d < 1) return ORC_ERR_ARG;
+    const int64_t hd = (int64_t)H * d;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < 3 * hd; ++j) {
+            double acc = 0.0;
+            for (int32_t c = 0; c < C; ++c) acc += widen(X, xdtype, r * C + c) * widen(W, wdtype, (int64_t)c * 3 * hd + j);
+            double *dst = j < hd ? Q : (j < 2 * hd ? K : V);
+            dst[r * hd + (j % hd)] = acc;
+        }
+    return ORC_OK;
+}

@@ -125,3 +125,35 @@ def test_leaf_size_one_tree_has_the_same_nodes(orc, m):
     q, k, v = workloads.random_qkv(len(pts), 1, 8, workloads.F32, 51)
     np.testing.assert_allclose(orc.ball_attention(q, k, v, m, p1), orc.ball_attention(q, k, v, m, pm),
                                rtol=1e-13, atol=1e-14)
+
+
+# --- projection of features to Q, K, V (feeds the fused projection + attention path) ---
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_projection_matches_numpy_matmul(orc, dtype):
+    rng = np.random.Generator(np.random.PCG64(60))
+    x = rng.standard_normal((300, 24)).astype(np.float32)
+    w = (rng.standard_normal((24, 3 * 2 * 8)) / np.sqrt(24)).astype(np.float32)
+    if dtype == "bf16":
+        x, w = workloads.f32_to_bf16_bits(x), workloads.f32_to_bf16_bits(w)
+        xd, wd = workloads.bf16_bits_to_f32(x).astype(np.float64), workloads.bf16_bits_to_f32(w).astype(np.float64)
+    else:
+        xd, wd = x.astype(np.float64), w.astype(np.float64)
+    q, k, v = orc.project(x, w, 2, 8)
+    y = xd @ wd  # [300, 48]: Q heads, K heads, V heads
+    np.testing.assert_allclose(q.reshape(300, 16), y[:, :16], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(k.reshape(300, 16), y[:, 16:32], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(v.reshape(300, 16), y[:, 32:], rtol=1e-12, atol=1e-12)
+
+
+def test_projection_with_identity_blocks_returns_the_features(orc):
+    # W = [I I I]: Q = K = V = X (C = H*d), so attention of the projection is attention of X itself
+    rng = np.random.Generator(np.random.PCG64(61))
+    x = rng.standard_normal((256, 16)).astype(np.float32)
+    w = np.concatenate([np.eye(16, dtype=np.float32)] * 3, axis=1)
+    q, k, v = orc.project(x, w, 2, 8)
+    np.testing.assert_array_equal(q.reshape(256, 16), x.astype(np.float64))
+    pts, perm = _cloud([256], 32, 62)
+    xr = x.reshape(256, 2, 8)
+    np.testing.assert_array_equal(orc.projected_ball_attention(x, w, 2, 8, 32, perm),
+                                  orc.ball_attention(xr, xr, xr, 32, perm))
