@@ -29,10 +29,10 @@ namespace bts {
 
 constexpr int kSortTile = 1024;      // keys per radix tile
 constexpr int kSortThreads = 256;
-constexpr int kLevelThreads = 512;     // one slot of each list per thread (two when m > 512)
-constexpr int kLevelTileTarget = 512;  // slots per list per wide-level tile (m * 2^k, or m when m > 512)
-constexpr int kLevelTileMax = 1024;
-constexpr int kLevelEpt = kLevelTileMax / kLevelThreads;
+constexpr int kLevelThreads = 512;
+constexpr int kLevelTileMin = 512;       // smallest wide-level tile, slots per list (or m when m is larger)
+constexpr int kLevelTileMax = 4096;      // largest: eight slots of each list per thread
+constexpr int kLevelTilesWanted = 148;   // large builds: about one wide-level tile per SM
 constexpr int kTailMax = 4096;         // largest node finished in shared memory
 constexpr int kTailMin = 512;          // smallest tail node (for m <= 512)
 constexpr int kTailCtasWanted = 2 * 148;  // aim for two tail CTAs per SM
@@ -79,7 +79,16 @@ static bt_status make_plan(const int64_t *offsets, int32_t B, int32_t m, Plan &P
     std::memset(&P, 0, sizeof(P));
     P.B = B;
     P.m = m;
-    P.TP = m <= kLevelTileTarget ? (m << ilog2(kLevelTileTarget / m)) : m;
+    // wide-level tile TP = m * 2^k slots: at least kLevelTileMin, about npad / kLevelTilesWanted on large
+    // builds (fewer, larger tiles: fewer predecessors to sum), at most kLevelTileMax
+    {
+        int64_t all = 0;
+        for (int b = 0; b < B; ++b) all += padded_size(offsets[b + 1] - offsets[b], m);
+        const int64_t want = std::max<int64_t>(kLevelTileMin, all / kLevelTilesWanted);
+        int64_t tp = m;
+        while (tp < want && 2 * tp <= kLevelTileMax) tp *= 2;
+        P.TP = int32_t(tp);
+    }
     int64_t npad_all = 0;
     for (int b = 0; b < B; ++b) {
         const int64_t n = offsets[b + 1] - offsets[b];
@@ -142,7 +151,7 @@ static Layout make_layout(const Plan &P)
     L.hist = 512;
     L.sst = L.hist + size_t(3) * P.B * 4 * 256 * 4;
     L.lst = L.sst + size_t(4) * 3 * P.sort_tiles * 256 * 4;
-    L.ctrl_end = align256(L.lst + size_t(std::max(P.nlev, 1)) * (np / P.TP) * 4 * 4);
+    L.ctrl_end = align256(L.lst + size_t(std::max(P.nlev, 1)) * (np / P.TP) * 8);
     L.keys = L.ctrl_end;
     L.sk = align256(L.keys + 3 * np * 4);
     L.sv = align256(L.sk + 2 * 3 * np * 4);
@@ -321,13 +330,64 @@ __device__ __forceinline__ bool before(uint32_t key, uint32_t id, uint32_t pkey,
     return key < pkey || (key == pkey && id < pid);
 }
 
-__global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const uint32_t *__restrict__ keys,
-                                                         const uint32_t *__restrict__ lin, uint32_t *__restrict__ lout,
-                                                         uint32_t *lst, uint32_t *counters, uint32_t *status)
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p)
 {
-    constexpr int NT = kLevelThreads, EPT = kLevelEpt;
-    __shared__ uint32_t sl[4][kLevelTileMax];
-    __shared__ unsigned long long scratch[NT / 32 + 1];
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Sum of two 64-bit values over the block (every thread calls; the result is returned to all).
+template <int NT>
+__device__ __forceinline__ void block_sum2(unsigned long long &a, unsigned long long &b, unsigned long long *red)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+    }
+    if (lane == 0) {
+        red[2 * warp] = a;
+        red[2 * warp + 1] = b;
+    }
+    __syncthreads();
+    a = 0;
+    b = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        a += red[2 * w];
+        b += red[2 * w + 1];
+    }
+    __syncthreads();
+}
+
+// A wide-level tile publishes one word: bit 63 set, and the left counts of its four lists in 15-bit fields
+// (a tile holds at most kLevelTileMax = 4096 slots of each list).
+constexpr unsigned long long kAggPublished = 1ull << 63;
+static_assert(kLevelTileMax < (1 << 15), "left counts of a tile must fit 15 bits");
+
+// One launch per wide level.  Tile j of a node (EPT*NT >= TP slots of each of the four lists) loads its
+// slots, finds its node's widest axis and median from the two ends of the sorted lists, classifies every
+// slot against the median (the node's own axis list splits by position; the other three lists compare
+// keys gathered by id), and publishes its four left counts at once.  Its offsets inside the node are the
+// sums of the counts of tiles 0..j-1 of the same node, read in one round by many threads: no tile waits on
+// a chain of inclusive prefixes.  Tiles take ids from an atomic counter, so every tile a tile waits on
+// has started before it and publishes before it waits on anything.
+template <int EPT>
+__global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level(Plan P, int lev, const uint32_t *__restrict__ keys,
+                                                            const uint32_t *__restrict__ lin,
+                                                            uint32_t *__restrict__ lout, unsigned long long *agg,
+                                                            uint32_t *counters, uint32_t *status)
+{
+    constexpr int NT = kLevelThreads;
+    extern __shared__ __align__(16) uint32_t sl[];  // [4][TP]
+    __shared__ unsigned long long scratch[2 * (NT / 32) + 1];
     __shared__ uint32_t s_tile, s_excl[4], s_pkey, s_pid, s_cand[3], s_ckey[3];
     __shared__ int s_axis;
     __shared__ float s_ext[3];
@@ -348,7 +408,7 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
     }
     const int64_t s = (P.pad[b + 1] - P.pad[b]) >> lev, half = s >> 1;
     const int64_t tps = s / TP;
-    if (tps < 1) {  // cannot happen for a valid plan; never divide by zero or index out of the lists
+    if (tps < 1 || TP > EPT * NT) {  // cannot happen for a valid plan; never divide by zero or index out of the lists
         if (tid == 0) record_error(status, BT_ERR_INTERNAL);
         return;
     }
@@ -393,7 +453,7 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
 #pragma unroll
             for (int q = 0; q < EPT; ++q) {
                 const int i = tid + q * NT;
-                if (i < TP) sl[l][i] = t[l][q];
+                if (i < TP) sl[l * TP + i] = t[l][q];
             }
     }
     __syncthreads();
@@ -411,39 +471,84 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
     const uint32_t *kax = keys + ax * np;
     const int ept = (TP + NT - 1) / NT;
     const int i0 = tid * ept;
-    uint32_t v[4][EPT];
-    uint32_t lbits[4] = {0, 0, 0, 0};
-    unsigned long long packed = 0;
+    uint32_t v[4][EPT], kk[4][EPT];
+    uint32_t bad = 0;
 #pragma unroll
-    for (int l = 0; l < 4; ++l) {
+    for (int l = 0; l < 4; ++l)
 #pragma unroll
         for (int q = 0; q < EPT; ++q) {
             const int i = i0 + q;
-            v[l][q] = 0;
+            v[l][q] = (q < ept && i < TP) ? sl[l * TP + i] : 0u;
+        }
+    // key gathers of the three lists that are not the split axis' own: all issued before the first compare
+#pragma unroll
+    for (int l = 0; l < 4; ++l)
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            kk[l][q] = 0u;
+            if (l != ax && q < ept && i0 + q < TP) {
+                const uint32_t pid = v[l][q];
+                if (pid < id_lo || pid >= id_hi)
+                    bad |= 1u << (l * EPT + q);
+                else
+                    kk[l][q] = kax[pid];
+            }
+        }
+    if (bad) record_error(status, BT_ERR_INTERNAL);
+    uint32_t lbits[4] = {0, 0, 0, 0};
+    unsigned long long packed = 0;
+#pragma unroll
+    for (int l = 0; l < 4; ++l)
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int i = i0 + q;
             if (q < ept && i < TP) {
-                const uint32_t pid = sl[l][i];
-                v[l][q] = pid;
                 bool left;
-                if (l == ax) {
+                if (l == ax)
                     left = int64_t(j) * TP + i < half;
-                } else if (pid < id_lo || pid >= id_hi) {
-                    record_error(status, BT_ERR_INTERNAL);
-                    left = false;
-                } else {
-                    left = before(kax[pid], pid, pkey, ppid);
-                }
+                else
+                    left = !((bad >> (l * EPT + q)) & 1u) && before(kk[l][q], v[l][q], pkey, ppid);
                 if (left) {
                     lbits[l] |= 1u << q;
                     packed += 1ull << (16 * l);
                 }
             }
         }
-    }
     unsigned long long tot = 0;
     const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, &tot);
-    if (tid < 4)
-        s_excl[tid] = lookback<16>(&lst[(size_t(lev) * (np / TP) + id) * 4 + tid], 4, j,
-                               uint32_t((tot >> (16 * tid)) & 0xFFFFu), status);
+    unsigned long long *node_agg = agg + size_t(lev) * (np / TP) + (id - j);
+    if (tid == 0) {
+        unsigned long long w = kAggPublished;
+#pragma unroll
+        for (int l = 0; l < 4; ++l) w |= ((tot >> (16 * l)) & 0xFFFFull) << (15 * l);
+        st_relaxed_u64(node_agg + j, w);
+    }
+    {
+        // left counts of the tiles before this one in the node: two 32-bit sums per 64-bit word
+        unsigned long long a01 = 0, a23 = 0;
+        for (int t = tid; t < j; t += NT) {
+            unsigned long long w = ld_relaxed_u64(node_agg + t);
+            int spins = 0;
+            while (!(w & kAggPublished)) {
+                if (++spins > kSpinLimit) {
+                    record_error(status, BT_ERR_TIMEOUT);
+                    w = kAggPublished;
+                    break;
+                }
+                __nanosleep(32);
+                w = ld_relaxed_u64(node_agg + t);
+            }
+            a01 += (w & 0x7FFFull) | (((w >> 15) & 0x7FFFull) << 32);
+            a23 += ((w >> 30) & 0x7FFFull) | (((w >> 45) & 0x7FFFull) << 32);
+        }
+        block_sum2<NT>(a01, a23, scratch);
+        if (tid == 0) {
+            s_excl[0] = uint32_t(a01);
+            s_excl[1] = uint32_t(a01 >> 32);
+            s_excl[2] = uint32_t(a23);
+            s_excl[3] = uint32_t(a23 >> 32);
+        }
+    }
 #pragma unroll
     for (int l = 0; l < 4; ++l) {
         const int nl = int((tot >> (16 * l)) & 0xFFFFu);
@@ -455,7 +560,7 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
                 const bool left = (lbits[l] >> q) & 1u;
                 const int pos = left ? run : nl + (i - run);
                 run += left;
-                sl[l][pos] = v[l][q];
+                sl[l * TP + pos] = v[l][q];
             }
         }
     }
@@ -470,7 +575,7 @@ __global__ void __launch_bounds__(kLevelThreads) k_level(Plan P, int lev, const 
                 record_error(status, BT_ERR_INTERNAL);
                 continue;
             }
-            lout[l * np + seg + dst] = sl[l][i];
+            lout[l * np + seg + dst] = sl[l * TP + i];
         }
     }
 }
@@ -701,7 +806,7 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
     uint32_t *counters = reinterpret_cast<uint32_t *>(w + L.counters);
     uint32_t *hist = reinterpret_cast<uint32_t *>(w + L.hist);
     uint32_t *sst = reinterpret_cast<uint32_t *>(w + L.sst);
-    uint32_t *lstat = reinterpret_cast<uint32_t *>(w + L.lst);
+    unsigned long long *lagg = reinterpret_cast<unsigned long long *>(w + L.lst);
     uint32_t *keys = reinterpret_cast<uint32_t *>(w + L.keys);
     uint32_t *sk = reinterpret_cast<uint32_t *>(w + L.sk);
     uint32_t *sv = reinterpret_cast<uint32_t *>(w + L.sv);
@@ -718,6 +823,8 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
             cudaFuncSetAttribute(k_sort_pass<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
             cudaFuncSetAttribute(k_sort_pass<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
             cudaFuncSetAttribute(k_sort_pass<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
+            cudaFuncSetAttribute(k_level<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(4 * kLevelTileMax * sizeof(uint32_t))) ||
             cudaFuncSetAttribute(k_tail<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(tail_smem_bytes(1024))) ||
             cudaFuncSetAttribute(k_tail<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -743,7 +850,16 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
         }
         const uint32_t *lin = lists + size_t(lev & 1) * 4 * np;
         uint32_t *lout = lists + size_t((lev + 1) & 1) * 4 * np;
-        k_level<<<unsigned(tiles), kLevelThreads, 0, st>>>(P, lev, keys, lin, lout, lstat, counters, status);
+        const size_t lsm = size_t(4) * P.TP * sizeof(uint32_t);
+        const unsigned g = unsigned(tiles);
+        if (P.TP <= kLevelThreads)
+            k_level<1><<<g, kLevelThreads, lsm, st>>>(P, lev, keys, lin, lout, lagg, counters, status);
+        else if (P.TP <= 2 * kLevelThreads)
+            k_level<2><<<g, kLevelThreads, lsm, st>>>(P, lev, keys, lin, lout, lagg, counters, status);
+        else if (P.TP <= 4 * kLevelThreads)
+            k_level<4><<<g, kLevelThreads, lsm, st>>>(P, lev, keys, lin, lout, lagg, counters, status);
+        else
+            k_level<8><<<g, kLevelThreads, lsm, st>>>(P, lev, keys, lin, lout, lagg, counters, status);
     }
     if (P.T <= 1024)
         k_tail<256><<<P.tail0[P.B], 256, tail_smem, st>>>(P, keys, lists, perm, status);
