@@ -23,6 +23,8 @@
 #include <algorithm>
 #include <cstring>
 
+#include <cooperative_groups.h>
+
 #include "bts_internal.cuh"
 
 namespace bts {
@@ -160,6 +162,60 @@ static Layout make_layout(const Plan &P)
     return L;
 }
 
+// Lanes of the warp whose 8-bit digit equals this lane's (bit i set for lane i), among the lanes with
+// `valid` set: eight ballots, one per digit bit (the warp-level multisplit of radix-sort literature).
+__device__ __forceinline__ uint32_t digit_peers(uint32_t d, bool valid)
+{
+    uint32_t mask = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+    for (int bit = 0; bit < 8; ++bit) {
+        const bool on = (d >> bit) & 1u;
+        const uint32_t b = __ballot_sync(0xffffffffu, on);
+        mask &= on ? b : ~b;
+    }
+    return mask;
+}
+
+// Distributed shared memory of the cluster, by explicit shared::cluster addresses.
+__device__ __forceinline__ uint32_t cluster_addr(const void *local_smem, uint32_t rank)
+{
+    const uint32_t a = uint32_t(__cvta_generic_to_shared(local_smem));
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ unsigned long long ld_cluster_u64(uint32_t addr)
+{
+    unsigned long long v;
+    asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, const uint4 &v)
+{
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // 1. keys, index list, digit histograms
 // ---------------------------------------------------------------------------
@@ -269,8 +325,8 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
     // stable rank of every element among equal digits of its warp, warp counts
 #pragma unroll
     for (int q = 0; q < ROUNDS; ++q) {
-        const uint32_t peers = __match_any_sync(0xffffffffu, dig[q]);
         const bool ok = dig[q] < 256u;
+        const uint32_t peers = digit_peers(dig[q], ok);
         const uint32_t base = ok ? whist[warp][dig[q]] : 0u;
         __syncwarp();
         if (ok && (peers & lt) == 0u) whist[warp][dig[q]] = base + __popc(peers);
@@ -788,10 +844,476 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
     }
 }
 
+// ---------------------------------------------------------------------------
+// 5. whole build of clouds of at most kClusterMaxCtas * kClusterMaxChunk slots
+//    in one launch: one thread-block cluster per cloud, the cloud's lists in
+//    the distributed shared memory of its CTAs.
+//
+// Every list element is a 16-byte record (key x, key y, key z, cloud-local
+// id), so classifying an element against any axis' median needs no gather.
+// CTA r of a cluster holds slots r*C .. r*C+C-1 of each list (C = npad / NC).
+//   sort    - per axis, four stable 8-bit LSD passes over the cluster: every
+//             CTA ranks its slots locally (warp match + per-warp digit
+//             counts), the CTAs' digit counts are exchanged, and every record
+//             is stored into the CTA that holds its global position.
+//   levels  - while a node spans several CTAs: each CTA classifies its slots
+//             against the node's median (read from the node's lists in the
+//             owning CTAs), publishes its four left counts, sums those of
+//             the node's CTAs before it and stores every record at its
+//             position in the other list buffer of the owning CTA.  Below
+//             that, nodes lie inside one CTA and the levels run in its own
+//             shared memory.
+//   output  - perm from the index list (ids ascending inside every leaf).
+// Every CTA of a cluster takes the same sequence of cluster barriers.
+// ---------------------------------------------------------------------------
+constexpr int kClusterThreads = 512;
+constexpr int kClusterMaxChunk = 1024;  // slots per CTA: 8 lists x 16 B x 1024 = 128 KB of records
+constexpr int kClusterMaxCtas = 16;     // non-portable cluster size (B200 allows 16)
+constexpr int kClusterEpt = kClusterMaxChunk / kClusterThreads;     // slots per thread in a level
+constexpr int kClusterRounds = kClusterMaxChunk / kClusterThreads;  // 32-slot rounds per warp in a sort pass
+static_assert(int64_t(kClusterMaxCtas) * kClusterMaxChunk < 65536, "cluster-path positions fit 16-bit lanes");
+
+__device__ __forceinline__ uint32_t rkey(const uint4 &r, int a) { return a == 0 ? r.x : (a == 1 ? r.y : r.z); }
+
+static size_t cluster_smem_bytes(int CS)
+{
+    // records [2][4][CS] + per-warp 16-bit digit counts [3][16][256] + digit counts, starts, offsets [3][3][256]
+    return size_t(8) * CS * sizeof(uint4) + size_t(3) * (kClusterThreads / 32) * 256 * 2 + size_t(9) * 256 * 4;
+}
+
+// NC CTAs per cluster; every cloud has a power-of-two slot count npad, and CTA r holds slots r*C..r*C+C-1
+// with C = npad / NC = 2^lc.  CS (>= every cloud's C) is the list stride in shared memory.
+template <int NC>
+__global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, int CS, const float *__restrict__ coords,
+                                                                      int32_t *__restrict__ perm, uint32_t *status)
+{
+    namespace cg = cooperative_groups;
+    constexpr int NT = kClusterThreads, NW = NT / 32, EPT = kClusterEpt, RM = kClusterRounds;
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ __align__(16) uint8_t dsm[];
+    uint4 *const recs = reinterpret_cast<uint4 *>(dsm);                   // [2][4][CS]
+    uint16_t *const wh = reinterpret_cast<uint16_t *>(recs + 8 * CS);     // [3][NW][256]; local levels reuse it
+    uint32_t *const hcnt = reinterpret_cast<uint32_t *>(wh + 3 * NW * 256);  // [3][256] this CTA's digit counts
+    uint32_t *const tst = hcnt + 3 * 256;                                 // [3][256] digit starts in this CTA
+    uint32_t *const off = tst + 3 * 256;                                  // [3][256] global position - local
+    __shared__ unsigned long long scratch[NT / 32 + 1];
+    __shared__ unsigned long long s_cnt, s_excl;
+    __shared__ uint32_t s_ck[3], s_cid[3], s_pk, s_pid;
+    __shared__ float s_ext[3];
+    __shared__ int s_ax;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rank = int(cluster.block_rank());
+    const int b = int(blockIdx.x) / NC;
+    const int npad = int(P.pad[b + 1] - P.pad[b]);
+    const int lnp = 31 - __clz(npad);
+    const int lc = lnp - (31 - __clz(NC));
+    const int C = 1 << lc, cmask = C - 1;
+    const int n = int(P.n[b]);
+    const int m = P.m;
+    const int pos0 = rank << lc;  // cloud-local position of this CTA's first slot, and id of its first point
+    auto L = [&](int buf, int l) { return recs + (buf * 4 + l) * CS; };
+
+    // --- records of this CTA's points; every list starts in id order -------
+    for (int i = tid; i < C; i += NT) {
+        const int id = pos0 + i;
+        uint4 r = make_uint4(kDummyKey, kDummyKey, kDummyKey, uint32_t(id));
+        if (id < n) {
+            const float *c = coords + (P.row0[b] + id) * 3;
+            const float x = c[0], y = c[1], z = c[2];
+            if (!isfinite(x) || !isfinite(y) || !isfinite(z)) record_error(status, BT_ERR_NONFINITE);
+            r.x = float_key(x);
+            r.y = float_key(y);
+            r.z = float_key(z);
+        }
+#pragma unroll
+        for (int l = 0; l < 4; ++l) L(0, l)[i] = r;
+    }
+
+    // --- presort: lists 0..2 end sorted by (key of their axis, id) ---------
+    const int BW = C >= NW * 32 ? C / NW : 32;  // slots of one warp's contiguous block
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int sh = 8 * pass;
+        for (int i = tid; i < 3 * NW * 256 / 8; i += NT) reinterpret_cast<uint4 *>(wh)[i] = make_uint4(0, 0, 0, 0);
+        __syncthreads();
+        uint4 rec[3][RM];
+        uint32_t dig[3][RM], rnk[3][RM];
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int q = 0; q < RM; ++q) {
+                const int e = warp * BW + q * 32 + lane;
+                const bool ok = q * 32 < BW && e < C;
+                rec[a][q] = ok ? L(0, a)[e] : make_uint4(0, 0, 0, 0);
+                dig[a][q] = ok ? ((rkey(rec[a][q], a) >> sh) & 255u) : (256u + lane);
+            }
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            uint16_t *w = wh + (a * NW + warp) * 256;
+#pragma unroll
+            for (int q = 0; q < RM; ++q) {
+                const bool ok = dig[a][q] < 256u;
+                const uint32_t peers = digit_peers(dig[a][q], ok);
+                const uint32_t base = ok ? w[dig[a][q]] : 0u;
+                __syncwarp();
+                if (ok && (peers & lt) == 0u) w[dig[a][q]] = uint16_t(base + __popc(peers));
+                __syncwarp();
+                rnk[a][q] = base + __popc(peers & lt);
+            }
+        }
+        __syncthreads();
+        unsigned long long pk = 0;
+        if (tid < 256) {
+#pragma unroll
+            for (int a = 0; a < 3; ++a) {
+                uint32_t run = 0;
+                for (int w = 0; w < NW; ++w) {
+                    const uint32_t c = wh[(a * NW + w) * 256 + tid];
+                    wh[(a * NW + w) * 256 + tid] = uint16_t(run);
+                    run += c;
+                }
+                hcnt[a * 256 + tid] = run;
+                pk |= uint64_t(run) << (16 * a);
+            }
+        }
+        const unsigned long long ts = block_exclusive_scan<NT, unsigned long long>(pk, scratch, nullptr);
+        if (tid < 256) {
+#pragma unroll
+            for (int a = 0; a < 3; ++a) tst[a * 256 + tid] = uint32_t((ts >> (16 * a)) & 0xFFFFu);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            uint4 *stg = L(1, a);
+            const uint16_t *w = wh + (a * NW + warp) * 256;
+#pragma unroll
+            for (int q = 0; q < RM; ++q)
+                if (dig[a][q] < 256u) stg[tst[a * 256 + dig[a][q]] + w[dig[a][q]] + rnk[a][q]] = rec[a][q];
+        }
+        cluster.sync();  // every CTA's digit counts and locally ordered runs are ready
+        {
+            unsigned long long tot = 0;
+            uint32_t pre[3] = {0, 0, 0};
+            if (tid < 256) {
+                uint32_t v[NC][3];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    const uint32_t rh = cluster_addr(hcnt + tid, c);
+#pragma unroll
+                    for (int a = 0; a < 3; ++a) v[c][a] = ld_cluster_u32(rh + a * 256 * 4);
+                }
+                uint32_t t3[3] = {0, 0, 0};
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+#pragma unroll
+                    for (int a = 0; a < 3; ++a) {
+                        t3[a] += v[c][a];
+                        if (c < rank) pre[a] += v[c][a];
+                    }
+                tot = t3[0] | (uint64_t(t3[1]) << 16) | (uint64_t(t3[2]) << 32);
+            }
+            const unsigned long long base = block_exclusive_scan<NT, unsigned long long>(tot, scratch, nullptr);
+            if (tid < 256) {
+#pragma unroll
+                for (int a = 0; a < 3; ++a)
+                    off[a * 256 + tid] = uint32_t((base >> (16 * a)) & 0xFFFFu) + pre[a] - tst[a * 256 + tid];
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            const uint4 *stg = L(1, a);
+            for (int j = tid; j < C; j += NT) {
+                const uint4 r = stg[j];
+                const uint32_t g = off[a * 256 + ((rkey(r, a) >> sh) & 255u)] + uint32_t(j);
+                if (g >= uint32_t(npad)) {  // counts disagree: never store outside the cluster's lists
+                    record_error(status, BT_ERR_INTERNAL);
+                    continue;
+                }
+                st_cluster_v4(cluster_addr(L(0, a) + (g & cmask), g >> lc), r);
+            }
+        }
+        cluster.sync();  // every record is in place for the next pass
+    }
+
+    // --- levels whose nodes span several CTAs ------------------------------
+    int cb = 0;
+    int ls = lnp;  // log2 of the node size
+    while ((1 << ls) > m && ls > lc) {
+        const int s = 1 << ls, half = s >> 1;
+        const int lper = ls - lc;  // log2 of the CTAs per node
+        const int k = rank >> lper, j = rank & ((1 << lper) - 1);
+        const int nstart = k << ls;
+        const int nreal = max(0, min(s, n - nstart));
+        if (tid < 3) {
+            const int a = tid;
+            const uint4 *La = L(cb, a);
+            const int pm = nstart + half;
+            const uint4 med = ld_cluster_v4(cluster_addr(La + (pm & cmask), pm >> lc));
+            float e = 0.0f;
+            if (nreal > 0) {
+                const int p1 = nstart + nreal - 1;
+                const uint4 f = ld_cluster_v4(cluster_addr(La + (nstart & cmask), nstart >> lc));
+                const uint4 l = ld_cluster_v4(cluster_addr(La + (p1 & cmask), p1 >> lc));
+                e = __fsub_rn(key_float(rkey(l, a)), key_float(rkey(f, a)));
+            }
+            s_ext[a] = e;
+            s_ck[a] = rkey(med, a);
+            s_cid[a] = med.w;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int ax = 0;
+            if (s_ext[1] > s_ext[ax]) ax = 1;
+            if (s_ext[2] > s_ext[ax]) ax = 2;
+            s_ax = ax;
+            s_pk = s_ck[ax];
+            s_pid = s_cid[ax];
+        }
+        __syncthreads();
+        const int ax = s_ax;
+        const uint32_t pk = s_pk, pid = s_pid;
+        const int ept = C >= NT ? C / NT : 1;
+        const int i0 = tid * ept;
+        uint4 v[4][EPT];
+        uint32_t lbits[4] = {0, 0, 0, 0};
+        unsigned long long packed = 0;
+#pragma unroll
+        for (int l = 0; l < 4; ++l)
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int i = i0 + q;
+                v[l][q] = make_uint4(0, 0, 0, 0);
+                if (q < ept && i < C) {
+                    v[l][q] = L(cb, l)[i];
+                    const bool left = (l == ax) ? ((j << lc) + i < half)
+                                                : before(rkey(v[l][q], ax), v[l][q].w, pk, pid);
+                    if (left) {
+                        lbits[l] |= 1u << q;
+                        packed += 1ull << (16 * l);
+                    }
+                }
+            }
+        unsigned long long tot = 0;
+        const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, &tot);
+        if (tid == 0) s_cnt = tot;
+        cluster.sync();  // every CTA's left counts are published
+        if (warp == 0) {
+            unsigned long long sum = 0;
+            for (int t = lane; t < j; t += 32) sum += ld_cluster_u64(cluster_addr(&s_cnt, (k << lper) + t));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (lane == 0) s_excl = sum;
+        }
+        __syncthreads();
+        const unsigned long long exn = s_excl;
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+            const int excl = int((exn >> (16 * l)) & 0xFFFFu);
+            int run = int((ex >> (16 * l)) & 0xFFFFu);
+            uint4 *Ln = L(cb ^ 1, l);
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int i = i0 + q;
+                if (q < ept && i < C) {
+                    const bool left = (lbits[l] >> q) & 1u;
+                    const int dst = left ? excl + run : half + ((j << lc) - excl) + (i - run);
+                    run += left;
+                    if ((left && dst >= half) || dst < 0 || dst >= s) {  // never store outside the node
+                        record_error(status, BT_ERR_INTERNAL);
+                        continue;
+                    }
+                    const int pos = nstart + dst;
+                    st_cluster_v4(cluster_addr(Ln + (pos & cmask), pos >> lc), v[l][q]);
+                }
+            }
+        }
+        cluster.sync();  // the next level reads the other buffer
+        cb ^= 1;
+        --ls;
+    }
+
+    // --- levels inside this CTA --------------------------------------------
+    {
+        uint32_t *spk = reinterpret_cast<uint32_t *>(wh);                  // [C/2] pivot key per node
+        uint32_t *spid = spk + kClusterMaxChunk / 2;                        // [C/2] pivot id
+        unsigned long long *segpre = reinterpret_cast<unsigned long long *>(spid + kClusterMaxChunk / 2);  // [C/2]
+        uint8_t *sax = reinterpret_cast<uint8_t *>(segpre + kClusterMaxChunk / 2);                        // [C/2]
+        const int ept = C >= NT ? C / NT : 1;
+        const int i0 = tid * ept;
+        for (; (1 << ls) > m; --ls) {
+            const int sz = 1 << ls, half = sz >> 1, nsub = C >> ls;
+            for (int q = tid; q < nsub; q += NT) {
+                const int start = q << ls;
+                const int nr = max(0, min(sz, n - (pos0 + start)));
+                float e[3] = {0.0f, 0.0f, 0.0f};
+                if (nr > 0) {
+#pragma unroll
+                    for (int a = 0; a < 3; ++a)
+                        e[a] = __fsub_rn(key_float(rkey(L(cb, a)[start + nr - 1], a)),
+                                         key_float(rkey(L(cb, a)[start], a)));
+                }
+                int ax = 0;
+                if (e[1] > e[ax]) ax = 1;
+                if (e[2] > e[ax]) ax = 2;
+                const uint4 med = L(cb, ax)[start + half];
+                sax[q] = uint8_t(ax);
+                spk[q] = rkey(med, ax);
+                spid[q] = med.w;
+            }
+            __syncthreads();
+            uint4 v[4][EPT];
+            uint32_t lbits[4] = {0, 0, 0, 0};
+            unsigned long long packed = 0;
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int i = i0 + q;
+                if (q < ept && i < C) {
+                    const int sub = i >> ls, off_in = i & (sz - 1);
+                    const int ax = sax[sub];
+                    const uint32_t pk = spk[sub], pid = spid[sub];
+#pragma unroll
+                    for (int l = 0; l < 4; ++l) {
+                        v[l][q] = L(cb, l)[i];
+                        const bool left = (l == ax) ? off_in < half : before(rkey(v[l][q], ax), v[l][q].w, pk, pid);
+                        if (left) {
+                            lbits[l] |= 1u << q;
+                            packed += 1ull << (16 * l);
+                        }
+                    }
+                }
+            }
+            const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, nullptr);
+            {
+                unsigned long long run = ex;
+#pragma unroll
+                for (int q = 0; q < EPT; ++q) {
+                    const int i = i0 + q;
+                    if (q < ept && i < C) {
+                        if ((i & (sz - 1)) == 0) segpre[i >> ls] = run;
+#pragma unroll
+                        for (int l = 0; l < 4; ++l)
+                            if ((lbits[l] >> q) & 1u) run += 1ull << (16 * l);
+                    }
+                }
+            }
+            __syncthreads();
+            {
+                unsigned long long run = ex;
+#pragma unroll
+                for (int q = 0; q < EPT; ++q) {
+                    const int i = i0 + q;
+                    if (q < ept && i < C) {
+                        const int sub = i >> ls, start = sub << ls;
+                        const unsigned long long sp = segpre[sub];
+#pragma unroll
+                        for (int l = 0; l < 4; ++l) {
+                            const int pre = int(((run >> (16 * l)) & 0xFFFFu) - ((sp >> (16 * l)) & 0xFFFFu));
+                            const bool left = (lbits[l] >> q) & 1u;
+                            const int dst = left ? start + pre : start + half + (i - start - pre);
+                            if ((left && pre >= half) || dst < start || dst >= start + sz)
+                                record_error(status, BT_ERR_INTERNAL);  // never store outside the node
+                            else
+                                L(cb ^ 1, l)[dst] = v[l][q];
+                            if (left) run += 1ull << (16 * l);
+                        }
+                    }
+                }
+            }
+            __syncthreads();
+            cb ^= 1;
+        }
+    }
+
+    // --- perm: the index list holds every leaf's ids in ascending order ----
+    const uint4 *I = L(cb, 3);
+    for (int i = tid; i < C; i += NT) {
+        const uint32_t id = I[i].w;
+        perm[P.pad[b] + pos0 + i] = int(id) < n ? int32_t(P.row0[b] + id) : -1;
+    }
+}
+
 static size_t tail_smem_bytes(int T)
 {
     // ps + k3 (16 B) + segpre (4 B) + pivot key (2 B) + pivot index (1 B) + lists (16 B) + axis (0.5 B) per slot
     return size_t(T) * 16 + size_t(T / 2) * (8 + 4 + 2 + 1) + size_t(8) * T * 2 + 16;
+}
+
+// Cluster size and list stride for the one-launch path, or false when a cloud does not fit it: every cloud's
+// slot count must be a power of two (m a power of two) of at most kClusterMaxCtas * kClusterMaxChunk.
+static bool cluster_shape(const Plan &P, int &NC, int &CS)
+{
+    int64_t mx = 0;
+    for (int b = 0; b < P.B; ++b) {
+        const int64_t np = P.pad[b + 1] - P.pad[b];
+        if (np & (np - 1)) return false;
+        mx = std::max<int64_t>(mx, np);
+    }
+    if (mx > int64_t(kClusterMaxCtas) * kClusterMaxChunk) return false;
+    NC = 4;
+    while (NC < kClusterMaxCtas && mx > int64_t(NC) * kClusterMaxChunk) NC *= 2;
+    for (int b = 0; b < P.B; ++b)
+        if ((P.pad[b + 1] - P.pad[b]) < NC) return false;
+    CS = int(mx / NC);
+    return true;
+}
+
+template <int NC>
+static cudaError_t cluster_launch(const Plan &P, int CS, const float *coords, int32_t *perm, uint32_t *status,
+                                  cudaStream_t st, int *max_clusters)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(P.B * NC));
+    cfg.blockDim = dim3(kClusterThreads);
+    cfg.dynamicSmemBytes = cluster_smem_bytes(CS);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = unsigned(NC);
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (max_clusters) {  // set-up query: attributes, then how many such clusters fit the device
+        cudaError_t e = cudaFuncSetAttribute(k_cluster_build<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(cluster_smem_bytes(kClusterMaxChunk)));
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k_cluster_build<NC>,
+                                                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        cfg.gridDim = dim3(unsigned(NC));
+        cfg.dynamicSmemBytes = cluster_smem_bytes(kClusterMaxChunk);
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(max_clusters, k_cluster_build<NC>, &cfg);
+        return e;
+    }
+    return cudaLaunchKernelEx(&cfg, k_cluster_build<NC>, P, CS, coords, perm, status);
+}
+
+static cudaError_t cluster_dispatch(int NC, const Plan &P, int CS, const float *coords, int32_t *perm,
+                                    uint32_t *status, cudaStream_t st, int *max_clusters)
+{
+    switch (NC) {
+    case 4: return cluster_launch<4>(P, CS, coords, perm, status, st, max_clusters);
+    case 8: return cluster_launch<8>(P, CS, coords, perm, status, st, max_clusters);
+    case 16: return cluster_launch<16>(P, CS, coords, perm, status, st, max_clusters);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// Whether clusters of NC CTAs with the largest chunk's shared memory can run on this device (cached per device).
+static bool cluster_runs(int dev, int NC)
+{
+    static int cache[64][5] = {};  // 0 unknown, 1 yes, 2 no; index log2(NC)
+    int li = 0;
+    while ((1 << li) < NC) ++li;
+    if (dev < 0 || dev >= 64 || li > 4) return false;
+    if (cache[dev][li]) return cache[dev][li] == 1;
+    int nclusters = 0;
+    const bool ok = cluster_dispatch(NC, Plan{}, kClusterMaxChunk, nullptr, nullptr, nullptr, nullptr, &nclusters) ==
+                        cudaSuccess &&
+                    nclusters > 0;
+    (void)cudaGetLastError();  // a refused query is not an error of this call
+    cache[dev][li] = ok ? 1 : 2;
+    return ok;
 }
 
 static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm, void *ws, size_t ws_bytes,
@@ -831,6 +1353,13 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
                                  int(tail_smem_bytes(kTailMax))))
             return BT_ERR_CUDA;
         attrs_set[dev] = true;
+    }
+    int NC = 0, CS = 0;
+    if (cluster_shape(P, NC, CS) && cluster_runs(dev, NC)) {
+        // every cloud fits one cluster: the whole build is one launch; only the status word needs clearing
+        if (cudaMemsetAsync(ws, 0, 64, st) != cudaSuccess) return BT_ERR_CUDA;
+        if (cluster_dispatch(NC, P, CS, coords, perm, status, st, nullptr) != cudaSuccess) return BT_ERR_CUDA;
+        return BT_OK;
     }
     if (cudaMemsetAsync(ws, 0, L.ctrl_end, st) != cudaSuccess) return BT_ERR_CUDA;
     k_init<<<P.sort_tiles, kSortThreads, 0, st>>>(P, coords, keys, lists + 3 * np, hist, status);
