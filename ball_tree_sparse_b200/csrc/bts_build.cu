@@ -870,15 +870,18 @@ constexpr int kClusterThreads = 512;
 constexpr int kClusterMaxChunk = 1024;  // slots per CTA: 8 lists x 16 B x 1024 = 128 KB of records
 constexpr int kClusterMaxCtas = 16;     // non-portable cluster size (B200 allows 16)
 constexpr int kClusterEpt = kClusterMaxChunk / kClusterThreads;     // slots per thread in a level
-constexpr int kClusterRounds = kClusterMaxChunk / kClusterThreads;  // 32-slot rounds per warp in a sort pass
 static_assert(int64_t(kClusterMaxCtas) * kClusterMaxChunk < 65536, "cluster-path positions fit 16-bit lanes");
 
 __device__ __forceinline__ uint32_t rkey(const uint4 &r, int a) { return a == 0 ? r.x : (a == 1 ? r.y : r.z); }
 
+constexpr int kClusterRankWarps = 4;  // warps that rank one axis' slots in a sort pass
+
 static size_t cluster_smem_bytes(int CS)
 {
-    // records [2][4][CS] + per-warp 16-bit digit counts [3][16][256] + digit counts, starts, offsets [3][3][256]
-    return size_t(8) * CS * sizeof(uint4) + size_t(3) * (kClusterThreads / 32) * 256 * 2 + size_t(9) * 256 * 4;
+    // records [2][4][CS] + scratch (per-warp digit counts [3][4][256] u16 in the sort, node pivots in the
+    // levels: 12 KB) + received digit counts [16][3][256] u16 + digit starts and offsets [2][3][256] u32
+    return size_t(8) * CS * sizeof(uint4) + size_t(12) * 1024 + size_t(kClusterMaxCtas) * 3 * 256 * 2 +
+           size_t(6) * 256 * 4;
 }
 
 // NC CTAs per cluster; every cloud has a power-of-two slot count npad, and CTA r holds slots r*C..r*C+C-1
@@ -888,13 +891,14 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                                                                       int32_t *__restrict__ perm, uint32_t *status)
 {
     namespace cg = cooperative_groups;
-    constexpr int NT = kClusterThreads, NW = NT / 32, EPT = kClusterEpt, RM = kClusterRounds;
+    constexpr int NT = kClusterThreads, EPT = kClusterEpt;
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(16) uint8_t dsm[];
+    constexpr int RW = kClusterRankWarps;
     uint4 *const recs = reinterpret_cast<uint4 *>(dsm);                   // [2][4][CS]
-    uint16_t *const wh = reinterpret_cast<uint16_t *>(recs + 8 * CS);     // [3][NW][256]; local levels reuse it
-    uint32_t *const hcnt = reinterpret_cast<uint32_t *>(wh + 3 * NW * 256);  // [3][256] this CTA's digit counts
-    uint32_t *const tst = hcnt + 3 * 256;                                 // [3][256] digit starts in this CTA
+    uint16_t *const wh = reinterpret_cast<uint16_t *>(recs + 8 * CS);     // [3][RW][256]; local levels reuse it
+    uint16_t *const rcv = wh + 12 * 1024 / 2;                             // [NC][3][256] every CTA's digit counts
+    uint32_t *const tst = reinterpret_cast<uint32_t *>(rcv + kClusterMaxCtas * 3 * 256);  // [3][256] starts here
     uint32_t *const off = tst + 3 * 256;                                  // [3][256] global position - local
     __shared__ unsigned long long scratch[NT / 32 + 1];
     __shared__ unsigned long long s_cnt, s_excl;
@@ -931,35 +935,36 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
     }
 
     // --- presort: lists 0..2 end sorted by (key of their axis, id) ---------
-    const int BW = C >= NW * 32 ? C / NW : 32;  // slots of one warp's contiguous block
+    // Warps 4a..4a+3 rank axis a: warp 4a+w takes the w-th quarter of the CTA's slots, 32 per round.
+    constexpr int RQ = kClusterMaxChunk / RW / 32;  // rounds per ranking warp (at most)
+    const int QW = C >= RW * 32 ? C / RW : 32;      // slots of one ranking warp's contiguous block
+    const int ra = warp / RW, rw = warp % RW;       // axis and quarter of a ranking warp (ra < 3)
     const uint32_t lt = (1u << lane) - 1u;
     for (int pass = 0; pass < 4; ++pass) {
         const int sh = 8 * pass;
-        for (int i = tid; i < 3 * NW * 256 / 8; i += NT) reinterpret_cast<uint4 *>(wh)[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tid; i < 3 * RW * 256 / 8; i += NT) reinterpret_cast<uint4 *>(wh)[i] = make_uint4(0, 0, 0, 0);
         __syncthreads();
-        uint4 rec[3][RM];
-        uint32_t dig[3][RM], rnk[3][RM];
+        uint4 rec[RQ];
+        uint32_t dig[RQ], rnk[RQ];
+        if (ra < 3) {
+            const uint4 *cur = L(0, ra);
+            uint16_t *w = wh + (ra * RW + rw) * 256;
 #pragma unroll
-        for (int a = 0; a < 3; ++a)
-#pragma unroll
-            for (int q = 0; q < RM; ++q) {
-                const int e = warp * BW + q * 32 + lane;
-                const bool ok = q * 32 < BW && e < C;
-                rec[a][q] = ok ? L(0, a)[e] : make_uint4(0, 0, 0, 0);
-                dig[a][q] = ok ? ((rkey(rec[a][q], a) >> sh) & 255u) : (256u + lane);
+            for (int q = 0; q < RQ; ++q) {
+                const int e = rw * QW + q * 32 + lane;
+                const bool ok = q * 32 < QW && e < C;
+                rec[q] = ok ? cur[e] : make_uint4(0, 0, 0, 0);
+                dig[q] = ok ? ((rkey(rec[q], ra) >> sh) & 255u) : 256u;
             }
 #pragma unroll
-        for (int a = 0; a < 3; ++a) {
-            uint16_t *w = wh + (a * NW + warp) * 256;
-#pragma unroll
-            for (int q = 0; q < RM; ++q) {
-                const bool ok = dig[a][q] < 256u;
-                const uint32_t peers = digit_peers(dig[a][q], ok);
-                const uint32_t base = ok ? w[dig[a][q]] : 0u;
+            for (int q = 0; q < RQ; ++q) {
+                const bool ok = dig[q] < 256u;
+                const uint32_t peers = digit_peers(dig[q], ok);
+                const uint32_t base = ok ? w[dig[q]] : 0u;
                 __syncwarp();
-                if (ok && (peers & lt) == 0u) w[dig[a][q]] = uint16_t(base + __popc(peers));
+                if (ok && (peers & lt) == 0u) w[dig[q]] = uint16_t(base + __popc(peers));
                 __syncwarp();
-                rnk[a][q] = base + __popc(peers & lt);
+                rnk[q] = base + __popc(peers & lt);
             }
         }
         __syncthreads();
@@ -968,12 +973,13 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
 #pragma unroll
             for (int a = 0; a < 3; ++a) {
                 uint32_t run = 0;
-                for (int w = 0; w < NW; ++w) {
-                    const uint32_t c = wh[(a * NW + w) * 256 + tid];
-                    wh[(a * NW + w) * 256 + tid] = uint16_t(run);
+#pragma unroll
+                for (int w = 0; w < RW; ++w) {
+                    const uint32_t c = wh[(a * RW + w) * 256 + tid];
+                    wh[(a * RW + w) * 256 + tid] = uint16_t(run);
                     run += c;
                 }
-                hcnt[a * 256 + tid] = run;
+                rcv[(rank * 3 + a) * 256 + tid] = uint16_t(run);  // this CTA's row of the exchanged counts
                 pk |= uint64_t(run) << (16 * a);
             }
         }
@@ -983,33 +989,32 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
             for (int a = 0; a < 3; ++a) tst[a * 256 + tid] = uint32_t((ts >> (16 * a)) & 0xFFFFu);
         }
         __syncthreads();
-#pragma unroll
-        for (int a = 0; a < 3; ++a) {
-            uint4 *stg = L(1, a);
-            const uint16_t *w = wh + (a * NW + warp) * 256;
-#pragma unroll
-            for (int q = 0; q < RM; ++q)
-                if (dig[a][q] < 256u) stg[tst[a * 256 + dig[a][q]] + w[dig[a][q]] + rnk[a][q]] = rec[a][q];
+        // push this CTA's digit counts to every other CTA of the cluster (posted stores)
+        for (int i = tid; i < (NC - 1) * 96; i += NT) {
+            const int c = (rank + 1 + i / 96) % NC, part = i % 96;
+            const uint4 v = reinterpret_cast<const uint4 *>(rcv + rank * 3 * 256)[part];
+            st_cluster_v4(cluster_addr(reinterpret_cast<const uint4 *>(rcv + rank * 3 * 256) + part, c), v);
         }
-        cluster.sync();  // every CTA's digit counts and locally ordered runs are ready
+        if (ra < 3) {
+            uint4 *stg = L(1, ra);
+            const uint16_t *w = wh + (ra * RW + rw) * 256;
+#pragma unroll
+            for (int q = 0; q < RQ; ++q)
+                if (dig[q] < 256u) stg[tst[ra * 256 + dig[q]] + w[dig[q]] + rnk[q]] = rec[q];
+        }
+        cluster.sync();  // every CTA's digit counts have arrived and its locally ordered runs are ready
         {
             unsigned long long tot = 0;
             uint32_t pre[3] = {0, 0, 0};
             if (tid < 256) {
-                uint32_t v[NC][3];
-#pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    const uint32_t rh = cluster_addr(hcnt + tid, c);
-#pragma unroll
-                    for (int a = 0; a < 3; ++a) v[c][a] = ld_cluster_u32(rh + a * 256 * 4);
-                }
                 uint32_t t3[3] = {0, 0, 0};
 #pragma unroll
                 for (int c = 0; c < NC; ++c)
 #pragma unroll
                     for (int a = 0; a < 3; ++a) {
-                        t3[a] += v[c][a];
-                        if (c < rank) pre[a] += v[c][a];
+                        const uint32_t v = rcv[(c * 3 + a) * 256 + tid];
+                        t3[a] += v;
+                        if (c < rank) pre[a] += v;
                     }
                 tot = t3[0] | (uint64_t(t3[1]) << 16) | (uint64_t(t3[2]) << 32);
             }
