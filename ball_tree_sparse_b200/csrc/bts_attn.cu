@@ -24,6 +24,8 @@
 // (bts_coarse.cuh) are included into this translation unit.
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "bts_internal.cuh"
 #include "bts_tc.cuh"
 
@@ -406,7 +408,8 @@ __device__ __forceinline__ void head_sync(int hj)
 __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     k_ball_attn_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ perm, int64_t npad,
-                     int64_t rows, int lm, int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O)
+                     int64_t rows, int lm, int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O,
+                     uint32_t *ctr)
 {
     using L = PairPipe;
     constexpr int NS = L::NS;
@@ -419,6 +422,10 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     __shared__ uint32_t sKeyMask[2][4];
     __shared__ __align__(8) uint64_t sBarS[2], sBarO[2], sFull[NS], sEmpty[NS];
     __shared__ uint32_t sTmem;
+    __shared__ int32_t sRows[NS][128];  // rows of the stage's item (-1: dummy slot), for the consumers
+    __shared__ int64_t sItem[NS];       // the stage's item, -1 when the CTA has no more work
+    __shared__ int64_t sClaim;          // next item, claimed by the first producer thread
+    __shared__ int sAbort[2];           // a head's warpgroup stops after a wait that ran out
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m = 1 << lm;
@@ -438,6 +445,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    if (tid < 2) sAbort[tid] = 0;
     if (tid == 0) {
         for (int j = 0; j < 2; ++j) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sBarS[j])) : "memory");
@@ -455,7 +463,6 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     tc_fence_after();
     const uint32_t tmem = sTmem;
     const int32_t oob = rows < 0x7FFFFFFF ? int32_t(rows) : -1;  // a row outside the tensor reads zeros
-    const int64_t first = blockIdx.x, stride = gridDim.x;
 
     auto raw_row = [&](int64_t item, int rr) -> int32_t {  // items < 2^31: 32-bit index arithmetic
         if (item >= items) return -1;
@@ -473,27 +480,36 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
 
     if (warp >= 8) {
         // ---------------- producers: lanes 0-15 of warp 8 + w take rows 4g..4g+3, g = 16 w + lane ----------------
+        // Work is claimed dynamically: the first item of a CTA is its block index, every later one comes from
+        // the launch's counter, so CTAs that start late (the GPU busy with other work) simply take fewer items.
+        // The next item is claimed, and its perm rows requested, right after the current item's gathers.
         const int pw = warp - 8, g = 16 * pw + lane;
-        auto load_rows = [&](int64_t item, int32_t (&rr)[4]) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) rr[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
-        };
-        int32_t nrows[4];
-        load_rows(first, nrows);
         bool pok = true;
-        int it = 0;
-        for (int64_t item = first; item < items; item += stride, ++it) {
+        int64_t item = blockIdx.x;
+        int32_t crow[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) crow[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
+        for (int it = 0;; ++it) {
             const int stage = it & (NS - 1);
+            const uint32_t bar = smem_u32(&sFull[stage]);
+            if (it >= NS) pok = mbar_wait(smem_u32(&sEmpty[stage]), ((it / NS) + 1) & 1) && pok;
+            if (item >= items) {  // no more work: tell the consumers through the free stage
+                if (tid == 8 * 32) {
+                    sItem[stage] = -1;
+                    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+                }
+                break;
+            }
             int32_t rr[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int32_t x = check(nrows[i]);
+                const int32_t x = check(crow[i]);
                 rr[i] = x >= 0 ? x : oob;
+                if (lane < 16) sRows[stage][4 * g + i] = x;
             }
-            load_rows(item + stride, nrows);  // consumed by the next iteration
-            if (it >= NS) pok = pok && mbar_wait(smem_u32(&sEmpty[stage]), ((it / NS) + 1) & 1);
-            const uint32_t bar = smem_u32(&sFull[stage]);
-            if (tid == 8 * 32) mbar_expect_tx(bar, L::STAGE);
+            if (tid == 8 * 32) sItem[stage] = item;
+            asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");  // rows and item stored
+            if (tid == 8 * 32) mbar_expect_tx(bar, L::STAGE);                  // publishes rows and item
             asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");  // armed before any gather lands
             if (lane < 16) {
                 const int32_t col = int32_t(uint32_t(item) % uint32_t(HP)) * 2 * D;
@@ -502,8 +518,14 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                 tma_gather4(dq + L::TILE, &tmK, col, rr[0], rr[1], rr[2], rr[3], bar);
                 tma_gather4(dq + 2 * L::TILE, &tmV, col, rr[0], rr[1], rr[2], rr[3], bar);
             }
+            // claim the next item after the gathers are on their way (a producer whose wait ran out hands out
+            // no further work); its perm rows load while the next stage frees up
+            if (tid == 8 * 32) sClaim = pok ? int64_t(gridDim.x) + int64_t(atomicAdd(ctr, 1u)) : items;
+            asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");
+            item = sClaim;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) crow[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
         }
-        (void)pok;
     } else {
         // ---------------- consumers ----------------
         const int hj = warp >> 2;  // head of the pair this warpgroup owns
@@ -512,20 +534,21 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         const uint32_t tS = tmem + 128 * hj, tO = tS + 64, tSum = tS + 96;  // this warpgroup's columns
         const uint32_t barS = smem_u32(&sBarS[hj]), barO = smem_u32(&sBarO[hj]);
         const uint32_t lanebase = uint32_t((warp & 3) * 32) << 16;
-        int32_t qcur = check(raw_row(first, r)), qnext = raw_row(first + stride, r);
         bool ok = true;
-        int it = 0;
-        for (int64_t item = first; item < items; item += stride, ++it) {
+        for (int it = 0;; ++it) {
             const int stage = it & (NS - 1);
-            const int32_t qafter = raw_row(item + 2 * stride, r);
+            ok = ok && mbar_wait(smem_u32(&sFull[stage]), (it / NS) & 1);
+            if (!ok) sAbort[hj] = 1;
+            const int32_t qcur = sRows[stage][r];  // this thread's query row (-1: dummy slot)
             {
                 const uint32_t kb = __ballot_sync(0xffffffffu, qcur >= 0);
                 if (lane == 0) sKeyMask[hj][warp & 3] = kb;
             }
-            ok = ok && mbar_wait(smem_u32(&sFull[stage]), (it / NS) & 1);
             tc_fence_before();
             head_sync(hj);
             tc_fence_after();
+            const int64_t item = sItem[stage];
+            if (item < 0 || sAbort[hj]) break;  // the same decision for the whole warpgroup
             const uint32_t sq = base + stage * L::STAGE, sk = sq + L::TILE, sv = sk + L::TILE;
             if (issuer) {
                 if (ok) {
@@ -635,8 +658,6 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                     }
                 }
             }
-            qcur = check(qnext);
-            qnext = qafter;
             tc_fence_before();
             head_sync(hj);  // this head's S/P and O are free again
             tc_fence_after();
@@ -647,6 +668,15 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     if (warp == 0) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::COLS) : "memory");
+    }
+    if (tid == 0) {
+        // the last CTA to finish resets the launch's counters for the next launch that uses them
+        __threadfence();
+        if (atomicAdd(ctr + 1, 1u) == gridDim.x - 1) {
+            ctr[0] = 0u;
+            ctr[1] = 0u;
+            __threadfence();
+        }
     }
 }
 
@@ -682,24 +712,36 @@ static bool row_map(CUtensorMap *map, const void *base, int64_t rows, int hd, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Work counters of the head-pair kernel: launch k uses pair k mod kPairCounters ([0] items claimed so far,
+// [1] CTAs finished); the last CTA of a launch sets both back to zero.  Launches that run at the same time
+// therefore need distinct pairs: up to kPairCounters launches may be in flight together.
+constexpr int kPairCounters = 256;
+static __device__ uint32_t g_pair_ctr[kPairCounters][2];
+
 static bt_status launch_pair(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
                              int64_t rows, int lm, int H, void *O, cudaStream_t st)
 {
     static bool set[64] = {false};
     static int sms[64] = {0};
+    static uint32_t *ctrs[64] = {nullptr};
+    static std::atomic<uint32_t> next_pair{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
-    if (dev >= 64 || !set[dev]) {
+    if (dev >= 64) return BT_ERR_UNSUPPORTED;
+    if (!set[dev]) {
         if (cudaFuncSetAttribute(k_ball_attn_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(PairPipe::BYTES)))
             return BT_ERR_CUDA;
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BT_ERR_CUDA;
-        if (dev < 64) {
-            sms[dev] = n;
-            set[dev] = true;
-        }
+        // host code sees only a stand-in for the counter array: ask the runtime for its device address
+        void *addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_pair_ctr) != cudaSuccess || !addr) return BT_ERR_CUDA;
+        ctrs[dev] = static_cast<uint32_t *>(addr);
+        sms[dev] = n;
+        set[dev] = true;
     }
+    uint32_t *ctr = ctrs[dev] + 2 * (next_pair.fetch_add(1u) % kPairCounters);
     CUtensorMap mq, mk, mv;
     if (!row_map(&mq, Q, rows, H * 32, 64) || !row_map(&mk, K, rows, H * 32, 64) || !row_map(&mv, V, rows, H * 32, 64))
         return BT_ERR_CUDA;
@@ -709,7 +751,7 @@ static bt_status launch_pair(const void *Q, const void *K, const void *V, const 
     const int64_t grid = items < int64_t(nsm) * PairPipe::PER_SM ? items : int64_t(nsm) * PairPipe::PER_SM;
     const float sl2 = 1.4426950408889634f / sqrtf(32.0f);
     k_ball_attn_pair<<<unsigned(grid), PairPipe::THREADS, PairPipe::BYTES, st>>>(
-        mq, mk, mv, perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O));
+        mq, mk, mv, perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O), ctr);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 
