@@ -381,8 +381,7 @@ struct PairPipe {
     static constexpr uint32_t RB = 128;                 // bytes of one row of a head pair
     static constexpr uint32_t TILE = 128 * RB;          // Q, K or V of one item (16 KB)
     static constexpr uint32_t STAGE = 3 * TILE;
-    static constexpr uint32_t ONES_OFF = NS * STAGE;
-    static constexpr uint32_t BYTES = ONES_OFF + 16 * 128 * 2 + 1024;
+    static constexpr uint32_t BYTES = NS * STAGE + 1024;
     static constexpr uint32_t COLS = 256;
     static constexpr int CONSUMERS = 256;               // two warpgroups, one per head of the pair
     static constexpr int PRODUCERS = 64;                // two warps that gather the next item's rows
@@ -414,12 +413,11 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     using L = PairPipe;
     constexpr int NS = L::NS;
     constexpr int D = 32;
-    constexpr uint32_t SBO8 = 8 * L::RB, ONES_SBO = 16 * 128, SW128 = 2;
+    constexpr uint32_t SBO8 = 8 * L::RB, SW128 = 2;
     constexpr uint32_t IDESC_S = idesc_bf16(128, false);
     constexpr uint32_t IDESC_O = idesc_bf16(D, true);
-    constexpr uint32_t IDESC_SUM = idesc_bf16(16, false);
     extern __shared__ __align__(1024) uint8_t psm[];
-    __shared__ uint32_t sKeyMask[2][4];
+    __shared__ uint32_t sKeyMask[NS][2][4];  // per stage: valid keys of each head's tile, by 32-key group
     __shared__ __align__(8) uint64_t sBarS[2], sBarO[2], sFull[NS], sEmpty[NS];
     __shared__ uint32_t sTmem;
     __shared__ int32_t sRows[NS][128];  // rows of the stage's item (-1: dummy slot), for the consumers
@@ -433,12 +431,6 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     const uint32_t base = (smem_u32(psm) + 1023u) & ~1023u;  // swizzled tiles need 1024-byte alignment
     uint8_t *gbase = psm + (base - smem_u32(psm));
 
-    for (int i = tid; i < 16 * 128 * 2 / 16; i += L::THREADS) {
-        const int c = i >> 4, rr = i & 15;
-        const uint32_t off = (rr >> 3) * ONES_SBO + c * 128 + (rr & 7) * 16;
-        const uint32_t one = (rr == 0) ? 0x3F803F80u : 0u;
-        *reinterpret_cast<uint4 *>(gbase + L::ONES_OFF + off) = make_uint4(one, one, one, one);
-    }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sTmem)),
                      "r"(L::COLS)
@@ -528,37 +520,44 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         }
     } else {
         // ---------------- consumers ----------------
+        // Per item: S = Q K^T, softmax (row sums in registers, on the FMA pipe), P V, O read into registers; then this
+        // head's TMEM is free, so the next item's S is issued before this item's scale-and-store epilogue.
         const int hj = warp >> 2;  // head of the pair this warpgroup owns
         const int r = tid & 127;   // query row (TMEM lane) this thread owns
         const bool issuer = r == 0;
-        const uint32_t tS = tmem + 128 * hj, tO = tS + 64, tSum = tS + 96;  // this warpgroup's columns
+        const uint32_t tS = tmem + 128 * hj, tO = tS + 64;  // this warpgroup's columns
         const uint32_t barS = smem_u32(&sBarS[hj]), barO = smem_u32(&sBarO[hj]);
         const uint32_t lanebase = uint32_t((warp & 3) * 32) << 16;
         bool ok = true;
-        for (int it = 0;; ++it) {
-            const int stage = it & (NS - 1);
-            ok = ok && mbar_wait(smem_u32(&sFull[stage]), (it / NS) & 1);
+        // Waits for stage `st` of round `it`, publishes this warp's key mask, and reads the stage's item and
+        // this thread's query row after the warpgroup barrier (so every thread takes the same decision).
+        auto head = [&](int itn, int st, int32_t &q, int64_t &itm) -> bool {
+            ok = ok && mbar_wait(smem_u32(&sFull[st]), (itn / NS) & 1);
             if (!ok) sAbort[hj] = 1;
-            const int32_t qcur = sRows[stage][r];  // this thread's query row (-1: dummy slot)
-            {
-                const uint32_t kb = __ballot_sync(0xffffffffu, qcur >= 0);
-                if (lane == 0) sKeyMask[hj][warp & 3] = kb;
-            }
+            q = sRows[st][r];  // -1: dummy slot
+            const uint32_t kb = __ballot_sync(0xffffffffu, q >= 0);
+            if (lane == 0) sKeyMask[st][hj][warp & 3] = kb;
             tc_fence_before();
             head_sync(hj);
             tc_fence_after();
-            const int64_t item = sItem[stage];
-            if (item < 0 || sAbort[hj]) break;  // the same decision for the whole warpgroup
-            const uint32_t sq = base + stage * L::STAGE, sk = sq + L::TILE, sv = sk + L::TILE;
-            if (issuer) {
-                if (ok) {
+            itm = sItem[st];
+            const bool go = itm >= 0 && !sAbort[hj];
+            if (go && issuer && ok) {
+                const uint32_t sq = base + st * L::STAGE, sk = sq + L::TILE;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_bf16(tS, smem_desc_sw(sq + 64 * hj + 32 * kk, 16, SBO8, SW128),
-                                 smem_desc_sw(sk + 64 * hj + 32 * kk, 16, SBO8, SW128), IDESC_S, kk > 0);
-                }
-                mma_commit(barS);  // arrives at once when nothing was issued: a failed wait ends quickly
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_bf16(tS, smem_desc_sw(sq + 64 * hj + 32 * kk, 16, SBO8, SW128),
+                             smem_desc_sw(sk + 64 * hj + 32 * kk, 16, SBO8, SW128), IDESC_S, kk > 0);
+                mma_commit(barS);
             }
+            return go;
+        };
+        int32_t qcur = -1;
+        int64_t item = -1;
+        bool go = head(0, 0, qcur, item);
+        for (int it = 0; go; ++it) {
+            const int stage = it & (NS - 1);
+            const uint32_t sv = base + stage * L::STAGE + 2 * L::TILE;
             ok = ok && mbar_wait(barS, it & 1);
             tc_fence_after();
 
@@ -572,7 +571,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                     bm = (c * 32 >= ball0 && c * 32 < ball0 + m) ? 0xffffffffu : 0u;
                 else
                     bm = (c * 32 <= ball0 && ball0 < c * 32 + 32) ? (((1u << m) - 1u) << (ball0 - c * 32)) : 0u;
-                cmask[c] = bm & sKeyMask[hj][c];
+                cmask[c] = bm & sKeyMask[stage][hj][c];
             }
             float mx = -INFINITY;
 #pragma unroll
@@ -591,6 +590,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                 }
             }
             const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
+            float rsum = 0.0f;  // row sum of the weights (before their rounding to bf16 for the P V product)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
@@ -608,6 +608,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                         }
                         const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                         pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                        rsum += p0 + p1;
                     }
                 } else {
 #pragma unroll
@@ -621,46 +622,45 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
             tc_fence_after();
             if (issuer) {
                 if (ok) {
-                    const uint32_t so1 = base + L::ONES_OFF;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t tp = tS + kk * 8;
-                        mma_bf16_ts(tO, tp, smem_desc_sw(sv + 64 * hj + kk * 16 * L::RB, 16, SBO8, SW128), IDESC_O,
-                                    kk > 0);
-                        mma_bf16_ts(tSum, tp, smem_desc(so1 + kk * 256, 128, ONES_SBO), IDESC_SUM, kk > 0);
-                    }
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tO, tS + kk * 8, smem_desc_sw(sv + 64 * hj + kk * 16 * L::RB, 16, SBO8, SW128),
+                                    IDESC_O, kk > 0);
                 }
                 mma_commit(barO);
                 mma_commit(smem_u32(&sEmpty[stage]));  // this head is done with the stage
             }
             ok = ok && mbar_wait(barO, it & 1);
             tc_fence_after();
-            if (ok) {
-                uint32_t sum_bits, o[32];
-                tmem_ld1_nowait(tSum + lanebase, sum_bits);
-                tmem_ld32_nowait(tO + lanebase, o);
-                tmem_wait_ld();
-                const float sum = __uint_as_float(sum_bits);
-                const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+            uint32_t o[32];
+            tmem_ld32_nowait(tO + lanebase, o);
+            tmem_wait_ld();
+            tc_fence_before();
+            head_sync(hj);  // this head's S/P and O columns are free again
+            tc_fence_after();
+
+            // next item's S on the tensor core while this item's rows are scaled and stored
+            int32_t qn = -1;
+            int64_t itemn = -1;
+            go = head(it + 1, (it + 1) & (NS - 1), qn, itemn);
+            if (ok && qcur >= 0) {
+                const float inv = rsum > 0.0f ? 1.0f / rsum : 0.0f;
                 const int h = int(uint32_t(item) % uint32_t(HP)) * 2 + hj;
-                if (qcur >= 0) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qcur) * H + h) * D);
+                uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qcur) * H + h) * D);
 #pragma unroll
-                    for (int t = 0; t < D / 8; ++t) {
-                        uint32_t w[4];
+                for (int t = 0; t < D / 8; ++t) {
+                    uint32_t w[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * t + 2 * e]) * inv,
-                                                                            __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
-                            w[e] = *reinterpret_cast<const uint32_t *>(&pb);
-                        }
-                        dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[8 * t + 2 * e]) * inv,
+                                                                        __uint_as_float(o[8 * t + 2 * e + 1]) * inv);
+                        w[e] = *reinterpret_cast<const uint32_t *>(&pb);
                     }
+                    dst[t] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-            tc_fence_before();
-            head_sync(hj);  // this head's S/P and O are free again
-            tc_fence_after();
+            qcur = qn;
+            item = itemn;
         }
     }
     tc_fence_before();
