@@ -29,7 +29,7 @@
 
 namespace bts {
 
-constexpr int kSortTile = 1024;      // keys per radix tile
+constexpr int kSortTile = 2048;      // keys per radix tile
 constexpr int kSortThreads = 256;
 constexpr int kLevelThreads = 512;
 constexpr int kLevelTileMin = 512;       // smallest wide-level tile, slots per list (or m when m is larger)
@@ -42,6 +42,7 @@ constexpr int kCounterLevel0 = 8;
 
 struct Plan {
     int32_t B, m, T, TP, nlev, sort_tiles;
+    int32_t rec;  // 1: record path (every cloud a power-of-two slot count of at most 2^21)
     int64_t npad;
     int64_t pad[BT_MAX_CLOUDS + 1];
     int64_t n[BT_MAX_CLOUDS];
@@ -142,6 +143,11 @@ static bt_status make_plan(const int64_t *offsets, int32_t B, int32_t m, Plan &P
             if (sn <= P.T || sn % P.TP || sn / P.TP < 1) return BT_ERR_INTERNAL;
         }
     if (P.TP > kLevelTileMax || P.T > kTailMax || P.T < m || (P.T & 1)) return BT_ERR_INTERNAL;
+    P.rec = 1;
+    for (int b = 0; b < B; ++b) {
+        const int64_t np = P.pad[b + 1] - P.pad[b];
+        if ((np & (np - 1)) || np > (int64_t(1) << 21)) P.rec = 0;
+    }
     return BT_OK;
 }
 
@@ -285,7 +291,8 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
                                                             const uint32_t *__restrict__ vin,
                                                             uint32_t *__restrict__ kout, uint32_t *__restrict__ vout,
                                                             const uint32_t *__restrict__ hist, uint32_t *sst,
-                                                            uint32_t *counters, uint32_t *status)
+                                                            uint32_t *counters, uint32_t *status,
+                                                            uint32_t *__restrict__ rank_out)
 {
     constexpr int NT = kSortThreads, NW = NT / 32, PER_WARP = kSortTile / NW, ROUNDS = PER_WARP / 32;
     constexpr int SHIFT = 8 * PASS;
@@ -372,8 +379,9 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
             record_error(status, BT_ERR_INTERNAL);
             continue;
         }
-        if (PASS < 3) kout[seg_base + rel] = kk;
+        if (kout) kout[seg_base + rel] = kk;  // the last pass writes sorted keys only when asked
         vout[seg_base + rel] = sval[j];
+        if (PASS == 3 && rank_out) rank_out[int64_t(a) * P.npad + sval[j]] = uint32_t(rel);  // the id's rank on axis a
     }
 }
 
@@ -840,6 +848,418 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
     for (int e = tid; e < sT; e += NT) {
         const uint32_t pid = ps[local_ok(L[3 * T + e], sT, status)];
         const int64_t li = int64_t(pid) - P.pad[b];
+        perm[seg + e] = li < P.n[b] ? int32_t(P.row0[b] + li) : -1;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 4b. record path for large clouds (every cloud a power-of-two slot count of
+//     at most 2^21): after the presort, every list element becomes an 8-byte
+//     record of the point's ranks on x, y and z (its positions in the three
+//     sorted orders, 21 bits each).  Ranks are distinct, so comparing ranks is
+//     comparing (coordinate, id): the wide levels and the tail classify by
+//     rank, move only records, and gather nothing.  The index list is not
+//     carried: the tail sorts every leaf's ids at the end.
+// ---------------------------------------------------------------------------
+constexpr int kRankBits = 21;
+constexpr uint64_t kRankMask = (uint64_t(1) << kRankBits) - 1;
+
+__device__ __forceinline__ uint32_t rrank(uint64_t r, int a) { return uint32_t((r >> (kRankBits * a)) & kRankMask); }
+
+// R0[a][p] = ranks of the point at position p of axis a's sorted list.
+__global__ void __launch_bounds__(256) k_records(Plan P, const uint32_t *__restrict__ ids,
+                                                 const uint32_t *__restrict__ rnk, unsigned long long *__restrict__ rec,
+                                                 uint32_t *status)
+{
+    const int64_t np = P.npad;
+    const int64_t t = int64_t(blockIdx.x) * 256 + threadIdx.x;
+    if (t >= 3 * np) return;
+    const int a = int(t / np);
+    const int64_t p = t - a * np;
+    int b = 0;
+    while (b + 1 < P.B && P.pad[b + 1] <= p) ++b;
+    const uint32_t id = ids[t];
+    if (id < uint32_t(P.pad[b]) || id >= uint32_t(P.pad[b + 1])) {  // never index with a foreign id
+        record_error(status, BT_ERR_INTERNAL);
+        rec[t] = 0;
+        return;
+    }
+    uint64_t r = 0;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const uint32_t v = k == a ? uint32_t(p - P.pad[b]) : rnk[k * np + id];
+        r |= uint64_t(v & uint32_t(kRankMask)) << (kRankBits * k);
+    }
+    rec[t] = r;
+}
+
+// One wide level on records (the same tiling and offsets as k_level, three lists of 8-byte records).
+template <int EPT>
+__global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level_r(
+    Plan P, int lev, const uint32_t *__restrict__ skeys, const unsigned long long *__restrict__ rin,
+    unsigned long long *__restrict__ rout, unsigned long long *agg, uint32_t *counters, uint32_t *status)
+{
+    constexpr int NT = kLevelThreads;
+    extern __shared__ __align__(16) unsigned long long sr[];  // [3][TP]
+    __shared__ unsigned long long scratch[2 * (NT / 32) + 1];
+    __shared__ uint16_t s_wcnt[3][EPT][NT / 32];  // left slots per (list, round, warp), then their prefixes
+    __shared__ uint32_t s_tile, s_excl[3], s_cand[3], s_ltot[3];
+    __shared__ int s_axis;
+    __shared__ float s_ext[3];
+    const int tid = threadIdx.x;
+    if (tid == 0) s_tile = atomicAdd(&counters[kCounterLevel0 + lev], 1u);
+    __syncthreads();
+    const int id = int(s_tile);
+    const int64_t np = P.npad;
+    const int TP = P.TP;
+    int b = 0;
+    int64_t r = id;
+    for (;;) {
+        const int64_t sb = P.pad[b + 1] - P.pad[b];
+        const int64_t nt = ((sb >> lev) > P.T) ? sb / TP : 0;
+        if (r < nt || b + 1 >= P.B) break;
+        r -= nt;
+        ++b;
+    }
+    const int64_t s = (P.pad[b + 1] - P.pad[b]) >> lev, half = s >> 1;
+    const int64_t tps = s / TP;
+    if (tps < 1 || TP > EPT * NT) {
+        if (tid == 0) record_error(status, BT_ERR_INTERNAL);
+        return;
+    }
+    const int64_t kseg = r / tps;
+    const int j = int(r - kseg * tps);
+    const int64_t seg = P.pad[b] + kseg * s;
+    const int64_t nreal = max64(0, min64(s, P.n[b] - kseg * s));
+    const int64_t tile0 = seg + int64_t(j) * TP;
+    if (tid < 3) {
+        // extent of axis tid from the keys at the node's lowest and highest real rank; candidate median rank
+        const unsigned long long *la = rin + tid * np;
+        const uint32_t pr = rrank(la[seg + half], tid);
+        float e = 0.0f;
+        if (nreal > 0) {
+            const uint32_t r0 = rrank(la[seg], tid), r1 = rrank(la[seg + nreal - 1], tid);
+            const uint32_t *ka = skeys + tid * np + P.pad[b];
+            e = __fsub_rn(key_float(ka[r1]), key_float(ka[r0]));
+        }
+        s_ext[tid] = e;
+        s_cand[tid] = pr;
+    }
+    {
+        unsigned long long t[3][EPT];
+#pragma unroll
+        for (int l = 0; l < 3; ++l)
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int i = tid + q * NT;
+                t[l][q] = i < TP ? rin[l * np + tile0 + i] : 0ull;
+            }
+#pragma unroll
+        for (int l = 0; l < 3; ++l)
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int i = tid + q * NT;
+                if (i < TP) sr[l * TP + i] = t[l][q];
+            }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int ax = 0;
+        if (s_ext[1] > s_ext[ax]) ax = 1;
+        if (s_ext[2] > s_ext[ax]) ax = 2;
+        s_axis = ax;
+    }
+    __syncthreads();
+    const int ax = s_axis;
+    const uint32_t prank = s_cand[ax];
+    // classification in coalesced order (slot i = q * NT + tid, conflict-free shared-memory reads): a ballot
+    // per (list, round) gives each slot's rank among the left slots of its warp's 32, and a scan of the
+    // per-(round, warp) counts in slot order gives the tile's offsets
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    unsigned long long v[3][EPT];
+    uint32_t bal[3][EPT];
+#pragma unroll
+    for (int l = 0; l < 3; ++l)
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int i = q * NT + tid;
+            bool left = false;
+            v[l][q] = 0ull;
+            if (i < TP) {
+                v[l][q] = sr[l * TP + i];
+                left = (l == ax) ? (int64_t(j) * TP + i < half) : (rrank(v[l][q], ax) < prank);
+            }
+            bal[l][q] = __ballot_sync(0xffffffffu, left);
+            if (lane == 0) s_wcnt[l][q][warp] = uint16_t(__popc(bal[l][q]));
+        }
+    __syncthreads();
+    if (warp < 3) {
+        // exclusive scan of list `warp`'s EPT * (NT / 32) counts, slot order (round-major), one lane per 4
+        constexpr int NC = EPT * (NT / 32), PER = (NC + 31) / 32;
+        uint16_t *c = &s_wcnt[warp][0][0];
+        uint32_t loc[PER], run = 0;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int k = lane * PER + u;
+            loc[u] = k < NC ? c[k] : 0u;
+            run += loc[u];
+        }
+        uint32_t inc = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        uint32_t ex = inc - run;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int k = lane * PER + u;
+            if (k < NC) c[k] = uint16_t(ex);
+            ex += loc[u];
+        }
+        if (lane == 31) s_ltot[warp] = inc;
+    }
+    __syncthreads();
+    const unsigned long long tot =
+        uint64_t(s_ltot[0]) | (uint64_t(s_ltot[1]) << 16) | (uint64_t(s_ltot[2]) << 32);
+    unsigned long long *node_agg = agg + size_t(lev) * (np / TP) + (id - j);
+    if (tid == 0) {
+        unsigned long long w = kAggPublished;
+#pragma unroll
+        for (int l = 0; l < 3; ++l) w |= ((tot >> (16 * l)) & 0xFFFFull) << (15 * l);
+        st_relaxed_u64(node_agg + j, w);
+    }
+    {
+        unsigned long long a01 = 0, a2 = 0;
+        for (int t = tid; t < j; t += NT) {
+            unsigned long long w = ld_relaxed_u64(node_agg + t);
+            int spins = 0;
+            while (!(w & kAggPublished)) {
+                if (++spins > kSpinLimit) {
+                    record_error(status, BT_ERR_TIMEOUT);
+                    w = kAggPublished;
+                    break;
+                }
+                __nanosleep(32);
+                w = ld_relaxed_u64(node_agg + t);
+            }
+            a01 += (w & 0x7FFFull) | (((w >> 15) & 0x7FFFull) << 32);
+            a2 += (w >> 30) & 0x7FFFull;
+        }
+        block_sum2<NT>(a01, a2, scratch);
+        if (tid == 0) {
+            s_excl[0] = uint32_t(a01);
+            s_excl[1] = uint32_t(a01 >> 32);
+            s_excl[2] = uint32_t(a2);
+        }
+    }
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+        const int nl = int(s_ltot[l]);
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int i = q * NT + tid;
+            if (i < TP) {
+                const bool left = (bal[l][q] >> lane) & 1u;
+                const int lb = int(s_wcnt[l][q][warp]) + __popc(bal[l][q] & lt);  // left slots before i
+                sr[l * TP + (left ? lb : nl + (i - lb))] = v[l][q];
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+        const int nl = int(s_ltot[l]);
+        const int64_t exl = s_excl[l];
+        for (int i = tid; i < TP; i += NT) {
+            const int64_t dst = i < nl ? exl + i : half + (int64_t(j) * TP - exl) + (i - nl);
+            if ((i < nl && dst >= half) || dst < 0 || dst >= s) {
+                record_error(status, BT_ERR_INTERNAL);
+                continue;
+            }
+            rout[l * np + seg + dst] = sr[l * TP + i];
+        }
+    }
+}
+
+constexpr int kTailRThreads = 512;
+
+static size_t tail_r_smem_bytes(int T)
+{
+    // records [2][3][T] + per node of the levels: pivot rank (4 B), axis (1 B), scan prefix (8 B) for T/2 nodes
+    return size_t(48) * T + size_t(T / 2) * 13 + 16;
+}
+
+// The remaining levels of one node of T slots (T a power of two) on records in shared memory; then each leaf's
+// ids (from the x ranks) are sorted ascending and written to perm.
+template <int EPT>  // slots per thread: 4 for nodes of up to 2048 slots (two CTAs per SM), 8 for 4096
+__global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan P, const uint32_t *__restrict__ skeys,
+                                                         const unsigned long long *__restrict__ r0buf,
+                                                         const unsigned long long *__restrict__ r1buf,
+                                                         const uint32_t *__restrict__ xids, int32_t *__restrict__ perm,
+                                                         uint32_t *status)
+{
+    constexpr int NT = kTailRThreads;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ unsigned long long scratch[NT / 32 + 1];
+    const int T = P.T;
+    unsigned long long *R = reinterpret_cast<unsigned long long *>(dsm);  // [2][3][T]
+    unsigned long long *segpre = R + 6 * T;                              // [T/2]
+    uint32_t *pvr = reinterpret_cast<uint32_t *>(segpre + T / 2);         // [T/2] pivot rank
+    uint8_t *axs = reinterpret_cast<uint8_t *>(pvr + T / 2);              // [T/2]
+    __shared__ uint16_t wcnt[3 * EPT * (kTailRThreads / 32)];             // left slots per (list, round, warp)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int id = blockIdx.x;
+    int b = 0;
+    while (b + 1 < P.B && P.tail0[b + 1] <= id) ++b;
+    const int k = id - P.tail0[b];
+    const int64_t np = P.npad;
+    const int sT = int(min64(P.pad[b + 1] - P.pad[b], T));
+    const int64_t seg = P.pad[b] + int64_t(k) * sT;
+    const int nreal = int(max64(0, min64(sT, P.n[b] - int64_t(k) * sT)));
+    const unsigned long long *rin = (P.glev[b] & 1) ? r1buf : r0buf;
+    const int m = P.m;
+    const int lsT = 31 - __clz(sT);
+    for (int i = tid; i < 3 * sT; i += NT) {
+        const int l = i >> lsT, e = i & (sT - 1);
+        R[l * T + e] = rin[l * np + seg + e];
+    }
+    __syncthreads();
+    int cur = 0;
+    const uint32_t *kb = skeys + P.pad[b];
+    for (int sz = sT, lsz = lsT; sz > m; sz >>= 1, --lsz) {
+        const int half = sz >> 1, nsub = sT >> lsz;
+        unsigned long long *L = R + cur * 3 * T, *Ln = R + (cur ^ 1) * 3 * T;
+        for (int q = tid; q < nsub; q += NT) {
+            const int start = q << lsz;
+            const int nr = max(0, min(sz, nreal - start));
+            float ext[3] = {0.0f, 0.0f, 0.0f};
+            if (nr > 0) {
+#pragma unroll
+                for (int a = 0; a < 3; ++a)
+                    ext[a] = __fsub_rn(key_float(kb[a * np + rrank(L[a * T + start + nr - 1], a)]),
+                                       key_float(kb[a * np + rrank(L[a * T + start], a)]));
+            }
+            int ax = 0;
+            if (ext[1] > ext[ax]) ax = 1;
+            if (ext[2] > ext[ax]) ax = 2;
+            axs[q] = uint8_t(ax);
+            pvr[q] = rrank(L[ax * T + start + half], ax);
+        }
+        __syncthreads();
+        // coalesced classification (slot e = q * NT + tid): ballots, then a scan of the per-(round, warp)
+        // left counts in slot order; a node's offsets are that prefix minus the prefix at the node's start
+        unsigned long long v[3][EPT];
+        uint32_t bal[3][EPT];
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = q * NT + tid;
+            const bool ok = e < sT;
+            const int sub = ok ? (e >> lsz) : 0;
+            const int ax = axs[sub];
+            const uint32_t pr = pvr[sub];
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+                v[l][q] = ok ? L[l * T + e] : 0ull;
+                const bool left = ok && ((l == ax) ? (e & (sz - 1)) < half : rrank(v[l][q], ax) < pr);
+                bal[l][q] = __ballot_sync(0xffffffffu, left);
+                if (lane == 0) wcnt[(l * EPT + q) * (NT / 32) + warp] = uint16_t(__popc(bal[l][q]));
+            }
+        }
+        __syncthreads();
+        if (warp < 3) {
+            constexpr int NC = EPT * (NT / 32), PER = (NC + 31) / 32;
+            uint16_t *c = wcnt + warp * NC;
+            uint32_t loc[PER], run = 0;
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int k = lane * PER + u;
+                loc[u] = k < NC ? c[k] : 0u;
+                run += loc[u];
+            }
+            uint32_t inc = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            uint32_t ex = inc - run;
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int k = lane * PER + u;
+                if (k < NC) c[k] = uint16_t(ex);
+                ex += loc[u];
+            }
+        }
+        __syncthreads();
+        uint32_t lb[3][EPT];  // left slots before each of this thread's slots, over the whole tile
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = q * NT + tid;
+#pragma unroll
+            for (int l = 0; l < 3; ++l)
+                lb[l][q] = uint32_t(wcnt[(l * EPT + q) * (NT / 32) + warp]) + __popc(bal[l][q] & lt);
+            if (e < sT && (e & (sz - 1)) == 0)
+                segpre[e >> lsz] = uint64_t(lb[0][q]) | (uint64_t(lb[1][q]) << 16) | (uint64_t(lb[2][q]) << 32);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = q * NT + tid;
+            if (e < sT) {
+                const int sub = e >> lsz, start = sub << lsz;
+                const unsigned long long sp = segpre[sub];
+#pragma unroll
+                for (int l = 0; l < 3; ++l) {
+                    const int pre = int(lb[l][q] - uint32_t((sp >> (16 * l)) & 0xFFFFu));
+                    const bool left = (bal[l][q] >> lane) & 1u;
+                    const int dst = left ? start + pre : start + half + (e - start - pre);
+                    if ((left && pre >= half) || dst < start || dst >= start + sz)
+                        record_error(status, BT_ERR_INTERNAL);  // never store outside the node
+                    else
+                        Ln[l * T + dst] = v[l][q];
+                }
+            }
+        }
+        __syncthreads();
+        cur ^= 1;
+    }
+    // ids of every slot (from the x rank), then every leaf of m slots sorted ascending by id (bitonic, in place)
+    uint32_t *ids = reinterpret_cast<uint32_t *>(R + (cur ^ 1) * 3 * T);  // the free record buffer
+    {
+        const unsigned long long *L = R + cur * 3 * T;
+        const uint32_t *xb = xids + P.pad[b];
+        for (int e = tid; e < sT; e += NT) ids[e] = xb[rrank(L[e], 0)];
+    }
+    __syncthreads();
+    const int lm = 31 - __clz(m);  // m is a power of two on this path
+    for (int kk = 2; kk <= m; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            for (int i = tid; i < sT / 2; i += NT) {
+                // pair (lo, lo + jj): lo has bit jj clear
+                const int lo = ((i & ~(jj - 1)) << 1) | (i & (jj - 1));
+                const int hi = lo + jj;
+                const bool up = kk == m ? true : ((lo & kk) == 0);
+                const uint32_t x = ids[lo], y = ids[hi];
+                if ((x > y) == up) {
+                    ids[lo] = y;
+                    ids[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    (void)lm;
+    for (int e = tid; e < sT; e += NT) {
+        const uint32_t pid = ids[e];
+        const int64_t li = int64_t(pid) - P.pad[b];
+        if (li < 0 || li >= P.pad[b + 1] - P.pad[b]) {
+            record_error(status, BT_ERR_INTERNAL);
+            perm[seg + e] = -1;
+            continue;
+        }
         perm[seg + e] = li < P.n[b] ? int32_t(P.row0[b] + li) : -1;
     }
 }
@@ -1352,6 +1772,14 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
             cudaFuncSetAttribute(k_sort_pass<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
             cudaFuncSetAttribute(k_level<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(4 * kLevelTileMax * sizeof(uint32_t))) ||
+            cudaFuncSetAttribute(k_level_r<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(3 * 4 * kLevelThreads * sizeof(uint64_t))) ||
+            cudaFuncSetAttribute(k_level_r<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(3 * kLevelTileMax * sizeof(uint64_t))) ||
+            cudaFuncSetAttribute(k_tail_r<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(tail_r_smem_bytes(4 * kTailRThreads))) ||
+            cudaFuncSetAttribute(k_tail_r<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(tail_r_smem_bytes(8 * kTailRThreads))) ||
             cudaFuncSetAttribute(k_tail<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(tail_smem_bytes(1024))) ||
             cudaFuncSetAttribute(k_tail<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1368,14 +1796,58 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
     }
     if (cudaMemsetAsync(ws, 0, L.ctrl_end, st) != cudaSuccess) return BT_ERR_CUDA;
     k_init<<<P.sort_tiles, kSortThreads, 0, st>>>(P, coords, keys, lists + 3 * np, hist, status);
+    if (P.rec) {
+        // presort; the last pass also leaves the sorted keys (list buffer 1) and every id's rank on each axis
+        // (over the keys, no longer needed); then records, wide levels and tail on records
+        const int sort_grid = 3 * P.sort_tiles;
+        uint32_t *skeys = lists + 4 * np;
+        unsigned long long *R0 = reinterpret_cast<unsigned long long *>(sk);
+        unsigned long long *R1 = reinterpret_cast<unsigned long long *>(sv);
+        k_sort_pass<0><<<sort_grid, kSortThreads, sort_smem, st>>>(P, keys, nullptr, sk, sv, hist, sst, counters,
+                                                                   status, nullptr);
+        k_sort_pass<1><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk, sv, sk + 3 * np, sv + 3 * np, hist, sst,
+                                                                   counters, status, nullptr);
+        k_sort_pass<2><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk + 3 * np, sv + 3 * np, sk, sv, hist, sst,
+                                                                   counters, status, nullptr);
+        k_sort_pass<3><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk, sv, skeys, lists, hist, sst, counters,
+                                                                   status, keys);
+        k_records<<<unsigned((3 * np + 255) / 256), 256, 0, st>>>(P, lists, keys, R0, status);
+        for (int lev = 0; lev < P.nlev; ++lev) {
+            int64_t tiles = 0;
+            for (int b = 0; b < P.B; ++b) {
+                const int64_t sb = P.pad[b + 1] - P.pad[b];
+                if ((sb >> lev) > P.T) tiles += sb / P.TP;
+            }
+            const unsigned long long *rin = (lev & 1) ? R1 : R0;
+            unsigned long long *rout = (lev & 1) ? R0 : R1;
+            const size_t lsm = size_t(3) * P.TP * sizeof(uint64_t);
+            const unsigned g = unsigned(tiles);
+            if (P.TP <= kLevelThreads)
+                k_level_r<1><<<g, kLevelThreads, lsm, st>>>(P, lev, skeys, rin, rout, lagg, counters, status);
+            else if (P.TP <= 2 * kLevelThreads)
+                k_level_r<2><<<g, kLevelThreads, lsm, st>>>(P, lev, skeys, rin, rout, lagg, counters, status);
+            else if (P.TP <= 4 * kLevelThreads)
+                k_level_r<4><<<g, kLevelThreads, lsm, st>>>(P, lev, skeys, rin, rout, lagg, counters, status);
+            else
+                k_level_r<8><<<g, kLevelThreads, lsm, st>>>(P, lev, skeys, rin, rout, lagg, counters, status);
+        }
+        if (P.T <= 4 * kTailRThreads)
+            k_tail_r<4><<<P.tail0[P.B], kTailRThreads, tail_r_smem_bytes(P.T), st>>>(P, skeys, R0, R1, lists, perm,
+                                                                                     status);
+        else
+            k_tail_r<8><<<P.tail0[P.B], kTailRThreads, tail_r_smem_bytes(P.T), st>>>(P, skeys, R0, R1, lists, perm,
+                                                                                     status);
+        return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
+    }
     const int sort_grid = 3 * P.sort_tiles;
-    k_sort_pass<0><<<sort_grid, kSortThreads, sort_smem, st>>>(P, keys, nullptr, sk, sv, hist, sst, counters, status);
+    k_sort_pass<0><<<sort_grid, kSortThreads, sort_smem, st>>>(P, keys, nullptr, sk, sv, hist, sst, counters, status,
+                                                               nullptr);
     k_sort_pass<1><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk, sv, sk + 3 * np, sv + 3 * np, hist, sst,
-                                                               counters, status);
+                                                               counters, status, nullptr);
     k_sort_pass<2><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk + 3 * np, sv + 3 * np, sk, sv, hist, sst,
-                                                               counters, status);
+                                                               counters, status, nullptr);
     k_sort_pass<3><<<sort_grid, kSortThreads, sort_smem, st>>>(P, sk, sv, nullptr, lists, hist, sst, counters,
-                                                               status);
+                                                               status, nullptr);
     for (int lev = 0; lev < P.nlev; ++lev) {
         int64_t tiles = 0;
         for (int b = 0; b < P.B; ++b) {
