@@ -47,8 +47,8 @@ LAYERS = 2
 # dram__bytes_write.sum, profiles/k_ball_attn_pair_gauss_mix.md) and the hash of the attention source it was
 # taken on (code lines only).  Reported only while that source is unchanged; null otherwise.
 ROOF_KERNEL = "k_ball_attn_pair"
-ROOF_TRAFFIC = {"bytes": 108863616,
-                "source_sha256": "3bad3a2f81bdb71f6c63c4d6ee28a226168576b60ee4f9de717a66e96d913761"}
+ROOF_TRAFFIC = {"bytes": 107585280,
+                "source_sha256": "892247f66eedbc89913662f91044579159012d6e9fec7753340516613e33acb3"}
 _ATTN_SOURCES = ("ball_tree_sparse_b200/csrc/bts_attn.cu", "ball_tree_sparse_b200/csrc/bts_tc.cuh")
 
 
@@ -79,6 +79,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-suite", action="store_true", help="skip the other workloads")
     p.add_argument("--suite-steps", type=int, default=20)
+    p.add_argument("--suite-only", default="",
+                   help="comma-separated suite workloads to time on their own (tiny, ellipsoid_bsa, box_cluster, "
+                        "gauss_mix_coarse_levels, ragged); skips the headline step")
     return p.parse_args()
 
 
@@ -388,9 +391,27 @@ def _bf16_dev(a, dev):
     return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
 
 
-def suite(bts, dev, steps, flush, peak):
-    """The other synthetic workloads, each timed on its own (layer = tree build + ball attention)."""
+def suite(bts, dev, steps, flush, peak, only=None):
+    """The other synthetic workloads, each timed on its own (layer = tree build + ball attention).
+    `only`: names of the workloads to run (all when None)."""
     res = {}
+
+    def want(name):
+        return only is None or name in only
+    if want("tiny"):
+        _suite_tiny(bts, dev, steps, flush, res)
+    if want("ellipsoid_bsa"):
+        _suite_ellipsoid(bts, dev, steps, flush, res)
+    if want("box_cluster"):
+        _suite_box(bts, dev, steps, flush, peak, res)
+    if want("gauss_mix_coarse_levels"):
+        _suite_coarse(bts, dev, steps, flush, res)
+    if want("ragged"):
+        _suite_ragged(bts, dev, steps, flush, res)
+    return res
+
+
+def _suite_tiny(bts, dev, steps, flush, res):
     # tiny: fp32, one layer
     wl = workloads.tiny()
     c = torch.from_numpy(wl.coords).to(dev)
@@ -407,6 +428,8 @@ def suite(bts, dev, steps, flush, peak):
     res["tiny"] = {"points": wl.n_total, "layers": 1, "dtype": "f32", "ms_per_step": ms,
                    "points_per_s_per_layer": wl.n_total / (ms / 1e3)}
 
+
+def _suite_ellipsoid(bts, dev, steps, flush, res):
     # ellipsoid: one layer of tree build + BSA (ball, compression, top-8 selection, gates)
     wl = workloads.ellipsoid()
     L = wl.layers[0]
@@ -442,19 +465,31 @@ def suite(bts, dev, steps, flush, peak):
                                     "query-coarsened: compression and selection with each group's pooled query"}
     del q, k, v, x, out, bws
 
-    # box + cluster, 1,048,576 points: two layers (original and rotated tree), as the headline step
+
+def _suite_box(bts, dev, steps, flush, peak, res):
+    # box + cluster, 1,048,576 points: two layers (original and rotated tree), as the headline step; and one
+    # tree build alone against its algorithmic bytes (coordinates read, 16 B per point per level, perm written)
     wl = workloads.box_cluster()
     st = Step(bts, wl, dev)
     ms = statistics.mean(timed_graph(lambda: st.body(), steps, 3, flush))
     a_ms = statistics.mean(timed_graph(
         lambda: bts.bt_ball_attention(*st.qkv[1], st.perm[1], wl.m, out=st.out[1]), steps, 3, flush))
+    b_ms = statistics.mean(timed_graph(
+        lambda: bts.bt_build_segmented(st.coords, wl.offsets, wl.m, perm=st.perm[0], ws=st.ws[0]), steps, 3, flush))
     nbytes = 4 * wl.n_total * wl.H * wl.d * 2 + 4 * st.npad
+    levels = int(round(math.log2(st.npad // wl.m)))
+    build_bytes = st.npad * (12 + 4 + 32 * levels)
     res["box_cluster"] = {"points": wl.n_total, "layers": 2, "ms_per_step": ms,
                           "points_per_s_per_layer": 2 * wl.n_total / (ms / 1e3), "attention_ms": a_ms,
                           "attention_gbs": nbytes / (a_ms / 1e3) / 1e9,
-                          "attention_frac_of_measured_hbm": nbytes / (a_ms / 1e3) / 1e9 / peak}
+                          "attention_frac_of_measured_hbm": nbytes / (a_ms / 1e3) / 1e9 / peak,
+                          "build_ms": b_ms, "build_algorithmic_bytes": build_bytes,
+                          "build_gbs": build_bytes / (b_ms / 1e3) / 1e9,
+                          "build_frac_of_measured_hbm": build_bytes / (b_ms / 1e3) / 1e9 / peak}
     del st
 
+
+def _suite_coarse(bts, dev, steps, flush, res):
     # coarser levels: gauss_mix 4 x 16384 on a tree of leaf size 1 (every power-of-two stride is a tree level);
     # attention one and two levels up: Q/K/V pooled to nodes of 2 or 4 slots, balls of 128 nodes, copied back
     wl = workloads.gauss_mix()
@@ -487,6 +522,8 @@ def suite(bts, dev, steps, flush, peak):
     res["gauss_mix_coarse_levels"] = entry
     del q, k, v, out, perm1, ws1
 
+
+def _suite_ragged(bts, dev, steps, flush, res):
     # ragged batch of 8 clouds, padded with dummies: segmented build + masked ball attention
     wl = workloads.ragged()
     L = wl.layers[0]
@@ -503,7 +540,6 @@ def suite(bts, dev, steps, flush, peak):
     ms = statistics.mean(timed_graph(rag_step, steps, 3, flush))
     res["ragged"] = {"points": wl.n_total, "padded_slots": npad, "clouds": wl.batch, "layers": 1, "ms_per_step": ms,
                      "points_per_s_per_layer": wl.n_total / (ms / 1e3)}
-    return res
 
 
 # ---------------------------------------------------------------------------
@@ -527,6 +563,16 @@ def main():
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.suite_only:
+        # the named suite workloads alone (for profiling one of them); no headline line
+        names = {x.strip() for x in args.suite_only.split(",") if x.strip()}
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        res = suite(bts, dev, args.suite_steps, flush, _peaks()[0], only=names)
+        if rank == 0:
+            print(json.dumps({"suite_only": sorted(names), "workloads": res}))
+        if dist is not None:
+            dist.destroy_process_group()
+        return
     wl = workloads.gauss_mix()
     st = Step(bts, wl, dev)
     st.capture()
