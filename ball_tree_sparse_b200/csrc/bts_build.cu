@@ -1287,7 +1287,7 @@ __global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan
 // Every CTA of a cluster takes the same sequence of cluster barriers.
 // ---------------------------------------------------------------------------
 constexpr int kClusterThreads = 512;
-constexpr int kClusterMaxChunk = 1024;  // slots per CTA: 8 lists x 16 B x 1024 = 128 KB of records
+constexpr int kClusterMaxChunk = 1024;  // slots per CTA: 6 lists x 16 B x 1024 = 96 KB of records
 constexpr int kClusterMaxCtas = 16;     // non-portable cluster size (B200 allows 16)
 constexpr int kClusterEpt = kClusterMaxChunk / kClusterThreads;     // slots per thread in a level
 static_assert(int64_t(kClusterMaxCtas) * kClusterMaxChunk < 65536, "cluster-path positions fit 16-bit lanes");
@@ -1298,9 +1298,10 @@ constexpr int kClusterRankWarps = 4;  // warps that rank one axis' slots in a so
 
 static size_t cluster_smem_bytes(int CS)
 {
-    // records [2][4][CS] + scratch (per-warp digit counts [3][4][256] u16 in the sort, node pivots in the
-    // levels: 12 KB) + received digit counts [16][3][256] u16 + digit starts and offsets [2][3][256] u32
-    return size_t(8) * CS * sizeof(uint4) + size_t(12) * 1024 + size_t(kClusterMaxCtas) * 3 * 256 * 2 +
+    // records [2][3][CS] + scratch (per-warp digit counts [3][4][256] u16 in the sort, node pivots in the
+    // levels, leaf ids at the end: 12 KB) + received digit counts [16][3][256] u16 + digit starts and offsets
+    // [2][3][256] u32
+    return size_t(6) * CS * sizeof(uint4) + size_t(12) * 1024 + size_t(kClusterMaxCtas) * 3 * 256 * 2 +
            size_t(6) * 256 * 4;
 }
 
@@ -1315,8 +1316,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(16) uint8_t dsm[];
     constexpr int RW = kClusterRankWarps;
-    uint4 *const recs = reinterpret_cast<uint4 *>(dsm);                   // [2][4][CS]
-    uint16_t *const wh = reinterpret_cast<uint16_t *>(recs + 8 * CS);     // [3][RW][256]; local levels reuse it
+    uint4 *const recs = reinterpret_cast<uint4 *>(dsm);                   // [2][3][CS]
+    uint16_t *const wh = reinterpret_cast<uint16_t *>(recs + 6 * CS);     // [3][RW][256]; later levels reuse it
     uint16_t *const rcv = wh + 12 * 1024 / 2;                             // [NC][3][256] every CTA's digit counts
     uint32_t *const tst = reinterpret_cast<uint32_t *>(rcv + kClusterMaxCtas * 3 * 256);  // [3][256] starts here
     uint32_t *const off = tst + 3 * 256;                                  // [3][256] global position - local
@@ -1336,9 +1337,10 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
     const int n = int(P.n[b]);
     const int m = P.m;
     const int pos0 = rank << lc;  // cloud-local position of this CTA's first slot, and id of its first point
-    auto L = [&](int buf, int l) { return recs + (buf * 4 + l) * CS; };
+    auto L = [&](int buf, int l) { return recs + (buf * 3 + l) * CS; };
 
     // --- records of this CTA's points; every list starts in id order -------
+    // (three lists, X, Y and Z; records carry the id, so no index list is kept: leaves are sorted by id last)
     for (int i = tid; i < C; i += NT) {
         const int id = pos0 + i;
         uint4 r = make_uint4(kDummyKey, kDummyKey, kDummyKey, uint32_t(id));
@@ -1351,7 +1353,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
             r.z = float_key(z);
         }
 #pragma unroll
-        for (int l = 0; l < 4; ++l) L(0, l)[i] = r;
+        for (int l = 0; l < 3; ++l) L(0, l)[i] = r;
     }
 
     // --- presort: lists 0..2 end sorted by (key of their axis, id) ---------
@@ -1501,11 +1503,11 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         const uint32_t pk = s_pk, pid = s_pid;
         const int ept = C >= NT ? C / NT : 1;
         const int i0 = tid * ept;
-        uint4 v[4][EPT];
-        uint32_t lbits[4] = {0, 0, 0, 0};
+        uint4 v[3][EPT];
+        uint32_t lbits[3] = {0, 0, 0};
         unsigned long long packed = 0;
 #pragma unroll
-        for (int l = 0; l < 4; ++l)
+        for (int l = 0; l < 3; ++l)
 #pragma unroll
             for (int q = 0; q < EPT; ++q) {
                 const int i = i0 + q;
@@ -1534,7 +1536,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         __syncthreads();
         const unsigned long long exn = s_excl;
 #pragma unroll
-        for (int l = 0; l < 4; ++l) {
+        for (int l = 0; l < 3; ++l) {
             const int excl = int((exn >> (16 * l)) & 0xFFFFu);
             int run = int((ex >> (16 * l)) & 0xFFFFu);
             uint4 *Ln = L(cb ^ 1, l);
@@ -1550,7 +1552,10 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                         continue;
                     }
                     const int pos = nstart + dst;
-                    st_cluster_v4(cluster_addr(Ln + (pos & cmask), pos >> lc), v[l][q]);
+                    if ((pos >> lc) == rank)  // stays in this CTA (the split axis' own list always does)
+                        Ln[pos & cmask] = v[l][q];
+                    else
+                        st_cluster_v4(cluster_addr(Ln + (pos & cmask), pos >> lc), v[l][q]);
                 }
             }
         }
@@ -1588,8 +1593,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                 spid[q] = med.w;
             }
             __syncthreads();
-            uint4 v[4][EPT];
-            uint32_t lbits[4] = {0, 0, 0, 0};
+            uint4 v[3][EPT];
+            uint32_t lbits[3] = {0, 0, 0};
             unsigned long long packed = 0;
 #pragma unroll
             for (int q = 0; q < EPT; ++q) {
@@ -1599,7 +1604,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                     const int ax = sax[sub];
                     const uint32_t pk = spk[sub], pid = spid[sub];
 #pragma unroll
-                    for (int l = 0; l < 4; ++l) {
+                    for (int l = 0; l < 3; ++l) {
                         v[l][q] = L(cb, l)[i];
                         const bool left = (l == ax) ? off_in < half : before(rkey(v[l][q], ax), v[l][q].w, pk, pid);
                         if (left) {
@@ -1618,7 +1623,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                     if (q < ept && i < C) {
                         if ((i & (sz - 1)) == 0) segpre[i >> ls] = run;
 #pragma unroll
-                        for (int l = 0; l < 4; ++l)
+                        for (int l = 0; l < 3; ++l)
                             if ((lbits[l] >> q) & 1u) run += 1ull << (16 * l);
                     }
                 }
@@ -1633,7 +1638,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                         const int sub = i >> ls, start = sub << ls;
                         const unsigned long long sp = segpre[sub];
 #pragma unroll
-                        for (int l = 0; l < 4; ++l) {
+                        for (int l = 0; l < 3; ++l) {
                             const int pre = int(((run >> (16 * l)) & 0xFFFFu) - ((sp >> (16 * l)) & 0xFFFFu));
                             const bool left = (lbits[l] >> q) & 1u;
                             const int dst = left ? start + pre : start + half + (i - start - pre);
@@ -1651,10 +1656,29 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         }
     }
 
-    // --- perm: the index list holds every leaf's ids in ascending order ----
-    const uint4 *I = L(cb, 3);
+    // --- perm: every leaf's ids (from list X), sorted ascending (bitonic in place) ----
+    uint32_t *ids = reinterpret_cast<uint32_t *>(wh);  // [C]
+    {
+        const uint4 *X = L(cb, 0);
+        for (int i = tid; i < C; i += NT) ids[i] = X[i].w;
+    }
+    __syncthreads();
+    for (int kk = 2; kk <= m; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            for (int i = tid; i < C / 2; i += NT) {
+                const int lo = ((i & ~(jj - 1)) << 1) | (i & (jj - 1)), hi = lo + jj;
+                const bool up = kk == m || (lo & kk) == 0;  // every leaf of m slots ends ascending
+                const uint32_t x = ids[lo], y = ids[hi];
+                if ((x > y) == up) {
+                    ids[lo] = y;
+                    ids[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
     for (int i = tid; i < C; i += NT) {
-        const uint32_t id = I[i].w;
+        const uint32_t id = ids[i];
         perm[P.pad[b] + pos0 + i] = int(id) < n ? int32_t(P.row0[b] + id) : -1;
     }
 }
@@ -1679,7 +1703,7 @@ static bool cluster_shape(const Plan &P, int &NC, int &CS)
     NC = 4;
     while (NC < kClusterMaxCtas && mx > int64_t(NC) * kClusterMaxChunk) NC *= 2;
     for (int b = 0; b < P.B; ++b)
-        if ((P.pad[b + 1] - P.pad[b]) < NC) return false;
+        if ((P.pad[b + 1] - P.pad[b]) < int64_t(NC) * P.m) return false;  // every leaf inside one CTA
     CS = int(mx / NC);
     return true;
 }
