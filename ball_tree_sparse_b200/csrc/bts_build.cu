@@ -307,7 +307,9 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
     for (int i = tid; i < NW * 256; i += NT) (&whist[0][0])[i] = 0;
     __syncthreads();
     const int id = int(s_tile);
-    const int a = id / P.sort_tiles, r = id - a * P.sort_tiles;
+    // tiles of the three axes interleaved in dispatch order: a third as many tiles of one segment in flight, so
+    // the look-back walks back over fewer unfinished predecessors (they still precede in dispatch order)
+    const int a = id % 3, r = id / 3;
     int b = 0;
     while (b + 1 < P.B && P.sort_tile0[b + 1] <= r) ++b;
     const int k = r - P.sort_tile0[b];
@@ -357,7 +359,8 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
     const uint32_t gb = block_exclusive_scan<NT, uint32_t>(hc, scratch, nullptr);
     if (tid < 256) {
         const uint32_t excl =
-            lookback<16>(&sst[(size_t(PASS) * 3 * P.sort_tiles + id) * 256 + tid], 256, k, dcount, status);
+            lookback<16>(&sst[(size_t(PASS) * 3 * P.sort_tiles + size_t(a) * P.sort_tiles + r) * 256 + tid], 256,
+                         k, dcount, status);
         tstart[tid] = ts;
         gpos[tid] = gb + excl - ts;  // modulo 2^32; + local index gives the position in the segment
     }
@@ -381,7 +384,12 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
         }
         if (kout) kout[seg_base + rel] = kk;  // the last pass writes sorted keys only when asked
         vout[seg_base + rel] = sval[j];
-        if (PASS == 3 && rank_out) rank_out[int64_t(a) * P.npad + sval[j]] = uint32_t(rel);  // the id's rank on axis a
+        if (PASS == 3 && rank_out) {  // the id's rank on axis a; ids come from earlier passes: check them
+            if (sval[j] < uint32_t(P.pad[b]) || sval[j] >= uint32_t(P.pad[b + 1]))
+                record_error(status, BT_ERR_INTERNAL);
+            else
+                rank_out[int64_t(a) * P.npad + sval[j]] = uint32_t(rel);
+        }
     }
 }
 
@@ -938,7 +946,12 @@ __global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level_r(
         const uint32_t pr = rrank(la[seg + half], tid);
         float e = 0.0f;
         if (nreal > 0) {
-            const uint32_t r0 = rrank(la[seg], tid), r1 = rrank(la[seg + nreal - 1], tid);
+            uint32_t r0 = rrank(la[seg], tid), r1 = rrank(la[seg + nreal - 1], tid);
+            const uint32_t nb = uint32_t(P.pad[b + 1] - P.pad[b]);
+            if (r0 >= nb || r1 >= nb) {  // a rank outside the cloud: never index with it
+                record_error(status, BT_ERR_INTERNAL);
+                r0 = r1 = 0;
+            }
             const uint32_t *ka = skeys + tid * np + P.pad[b];
             e = __fsub_rn(key_float(ka[r1]), key_float(ka[r0]));
         }
@@ -1122,6 +1135,7 @@ __global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan
     const unsigned long long *rin = (P.glev[b] & 1) ? r1buf : r0buf;
     const int m = P.m;
     const int lsT = 31 - __clz(sT);
+    const int64_t sTc = P.pad[b + 1] - P.pad[b];  // slots of the cloud: every rank is below it
     for (int i = tid; i < 3 * sT; i += NT) {
         const int l = i >> lsT, e = i & (sT - 1);
         R[l * T + e] = rin[l * np + seg + e];
@@ -1138,9 +1152,14 @@ __global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan
             float ext[3] = {0.0f, 0.0f, 0.0f};
             if (nr > 0) {
 #pragma unroll
-                for (int a = 0; a < 3; ++a)
-                    ext[a] = __fsub_rn(key_float(kb[a * np + rrank(L[a * T + start + nr - 1], a)]),
-                                       key_float(kb[a * np + rrank(L[a * T + start], a)]));
+                for (int a = 0; a < 3; ++a) {
+                    uint32_t r1 = rrank(L[a * T + start + nr - 1], a), r0 = rrank(L[a * T + start], a);
+                    if (r0 >= uint32_t(sTc) || r1 >= uint32_t(sTc)) {  // a rank outside the cloud
+                        record_error(status, BT_ERR_INTERNAL);
+                        r0 = r1 = 0;
+                    }
+                    ext[a] = __fsub_rn(key_float(kb[a * np + r1]), key_float(kb[a * np + r0]));
+                }
             }
             int ax = 0;
             if (ext[1] > ext[ax]) ax = 1;
@@ -1231,7 +1250,15 @@ __global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan
     {
         const unsigned long long *L = R + cur * 3 * T;
         const uint32_t *xb = xids + P.pad[b];
-        for (int e = tid; e < sT; e += NT) ids[e] = xb[rrank(L[e], 0)];
+        for (int e = tid; e < sT; e += NT) {
+            const uint32_t rx = rrank(L[e], 0);
+            if (rx >= uint32_t(sTc)) {  // a rank outside the cloud: never index with it
+                record_error(status, BT_ERR_INTERNAL);
+                ids[e] = uint32_t(P.pad[b]);
+            } else {
+                ids[e] = xb[rx];
+            }
+        }
     }
     __syncthreads();
     const int lm = 31 - __clz(m);  // m is a power of two on this path
