@@ -140,16 +140,17 @@ __global__ void __launch_bounds__(kMeanWarps * 32) k_bsa_means(const __nv_bfloat
 // ---------------------------------------------------------------------------
 // Gates: one thread per row, kGateOut outputs at a time in registers.  W is
 // staged once per CTA with its rows padded to a multiple of kGateOut (zeros),
-// so the inner loop is one X value (conflict-free, rows padded by one word)
-// and kGateOut/4 broadcast float4 reads of W per kGateOut FMAs.  X is staged
-// kGateCols columns at a time with coalesced loads.
-constexpr int kGateRows = 128, kGateCols = 64, kGateOut = 24;
+// and kGateOut/4 broadcast float4 reads of W per kGateOut FMAs.  X streams
+// through shared memory kGateCols columns at a time, double-buffered: the next
+// slice is loaded into registers (coalesced float4) while the current one is
+// used, so the loads of one slice overlap the FMAs of the other.
+constexpr int kGateRows = 128, kGateCols = 32, kGateOut = 24;
 
 static int gate_out_padded(int H) { return (3 * H + kGateOut - 1) / kGateOut * kGateOut; }
 
 static size_t gate_smem_bytes(int C, int H)
 {
-    return (size_t(C) * gate_out_padded(H) + size_t(kGateRows) * (kGateCols + 1)) * 4;
+    return (size_t(C) * gate_out_padded(H) + size_t(2) * kGateRows * (kGateCols + 1)) * 4;
 }
 
 __global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict__ X, int64_t rows, int C,
@@ -158,8 +159,9 @@ __global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict
 {
     extern __shared__ __align__(16) float gsm[];
     constexpr int XP = kGateCols + 1;
+    constexpr int U = kGateRows * kGateCols / 4 / kGateRows;  // float4 of a slice per thread
     const int NO = 3 * H;
-    float *sW = gsm, *sX = gsm + size_t(C) * NOP;
+    float *sW = gsm, *sX = gsm + size_t(C) * NOP;  // sX: [2][kGateRows][XP]
     const int tid = threadIdx.x;
     {
         // W rows padded to NOP columns with zeros; loads batched 8 per thread ahead of their stores
@@ -187,38 +189,55 @@ __global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict
     }
     const int64_t r0 = int64_t(blockIdx.x) * kGateRows, r = r0 + tid;
     const bool vec4 = (C % 4) == 0 && (reinterpret_cast<uintptr_t>(X) % 16) == 0;
+    const int nslice = (C + kGateCols - 1) / kGateCols;
+    // one slice of X into registers: row rr = i / (kGateCols/4), columns c0 + 4*(i % (kGateCols/4)) .. +3
+    auto load_slice = [&](int c0, float4 (&t)[U]) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+            const int c = c0 + 4 * c4;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r0 + rr < rows) {
+                const float *src = X + (r0 + rr) * C + c;
+                if (vec4 && c + 4 <= C) {
+                    v = *reinterpret_cast<const float4 *>(src);
+                } else {
+                    if (c < C) v.x = src[0];
+                    if (c + 1 < C) v.y = src[1];
+                    if (c + 2 < C) v.z = src[2];
+                    if (c + 3 < C) v.w = src[3];
+                }
+            }
+            t[u] = v;
+        }
+    };
+    auto store_slice = [&](int buf, const float4 (&t)[U]) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+            float *d = sX + (size_t(buf) * kGateRows + rr) * XP + 4 * c4;
+            d[0] = t[u].x;
+            d[1] = t[u].y;
+            d[2] = t[u].z;
+            d[3] = t[u].w;
+        }
+    };
     for (int j0 = 0; j0 < NO; j0 += kGateOut) {
         float acc[kGateOut];
 #pragma unroll
         for (int j = 0; j < kGateOut; ++j) acc[j] = (bg && j0 + j < NO) ? bg[j0 + j] : 0.0f;
-        for (int c0 = 0; c0 < C; c0 += kGateCols) {
+        float4 t[U];
+        load_slice(0, t);
+        __syncthreads();  // W is staged; neither buffer is read any more
+        store_slice(0, t);
+        __syncthreads();
+        for (int k = 0; k < nslice; ++k) {
+            const int c0 = k * kGateCols;
+            if (k + 1 < nslice) load_slice(c0 + kGateCols, t);  // in flight while slice k is used
+            const float *xs = sX + (size_t(k & 1) * kGateRows + tid) * XP;
             const int cw = C - c0 < kGateCols ? C - c0 : kGateCols;
-            __syncthreads();  // W is staged / the previous X tile is consumed
-            if (cw == kGateCols && vec4) {
-                // full tile, float4 loads, all issued before the first store
-                constexpr int U = kGateRows * kGateCols / 4 / kGateRows;  // float4 per thread
-                float4 t[U];
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
-                    t[u] = (r0 + rr < rows) ? *reinterpret_cast<const float4 *>(X + (r0 + rr) * C + c0 + 4 * c4)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
-                    float *d = sX + rr * XP + 4 * c4;
-                    d[0] = t[u].x; d[1] = t[u].y; d[2] = t[u].z; d[3] = t[u].w;
-                }
-            } else {
-                for (int i = tid; i < kGateRows * cw; i += kGateRows) {
-                    const int rr = i / cw, cc = i - rr * cw;
-                    sX[rr * XP + cc] = (r0 + rr < rows) ? X[(r0 + rr) * C + c0 + cc] : 0.0f;
-                }
-            }
-            __syncthreads();
             for (int cc = 0; cc < cw; ++cc) {
-                const float x = sX[tid * XP + cc];
+                const float x = xs[cc];
                 const float4 *w4 = reinterpret_cast<const float4 *>(sW + size_t(c0 + cc) * NOP + j0);
 #pragma unroll
                 for (int j4 = 0; j4 < kGateOut / 4; ++j4) {
@@ -229,6 +248,8 @@ __global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict
                     acc[4 * j4 + 3] = fmaf(x, w.w, acc[4 * j4 + 3]);
                 }
             }
+            if (k + 1 < nslice) store_slice((k + 1) & 1, t);  // the other buffer: nobody reads it now
+            __syncthreads();
         }
         if (r < rows) {
 #pragma unroll
