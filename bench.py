@@ -190,8 +190,9 @@ class Step:
             self.ev[key].record(s)
 
     def body(self, capturing=False):
-        """Both trees are built concurrently (they depend only on the coordinates); the two attention
-        layers run one after the other on the main stream."""
+        """Both trees are built concurrently (they depend only on the coordinates); the slot maps
+        (inverse of tree A, A->B map) follow tree B on the side stream once tree A is built, beside
+        layer A's attention; the two attention layers run one after the other on the main stream."""
         bts, wl = self.bts, self.wl
         main = torch.cuda.current_stream()
         self._mark("a0", capturing)
@@ -201,11 +202,13 @@ class Step:
             bts.bt_build_segmented(self.rot, wl.offsets, wl.m, perm=self.perm[1], ws=self.ws[1])
         bts.bt_build_segmented(self.coords, wl.offsets, wl.m, perm=self.perm[0], ws=self.ws[0])
         self._mark("a1", capturing)
+        self.side.wait_stream(main)  # tree A is built
+        with torch.cuda.stream(self.side):
+            bts.bt_invert_perm(self.perm[0], self.n, inv=self.inv)
+            bts.bt_compose(self.inv, self.perm[1], out=self.map)
         bts.bt_ball_attention(*self.qkv[0], self.perm[0], wl.m, out=self.out[0])
         self._mark("a2", capturing)
         main.wait_stream(self.side)
-        bts.bt_invert_perm(self.perm[0], self.n, inv=self.inv)
-        bts.bt_compose(self.inv, self.perm[1], out=self.map)
         self._mark("b1", capturing)
         bts.bt_ball_attention(*self.qkv[1], self.perm[1], wl.m, out=self.out[1])
         self._mark("b2", capturing)
