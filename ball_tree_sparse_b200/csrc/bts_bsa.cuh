@@ -21,8 +21,8 @@
 //                  empty balls masked, top-k.
 //   k_bsa_attn_tc  persistent tcgen05 kernel over (group, head) items: the
 //                  compression and selection branches as flash-style online
-//                  softmax over chunks of 128 keys (S and P in TMEM, P V and
-//                  the row sums on the tensor core), then the gated sum with
+//                  softmax over chunks of 128 keys (S and P in TMEM, P V on the
+//                  tensor core, row sums in registers), then the gated sum with
 //                  the ball branch, scattered through perm.
 //   k_bsa_coarse   the query-coarsening variant of the two branches: one CTA
 //                  per (group, head) with the pooled query, then the gated sum.
@@ -348,8 +348,7 @@ struct BsaPipe {
     static constexpr uint32_t Q_OFF = 0;
     static constexpr uint32_t STAGE_OFF = QK_BYTES;      // 2 stages of (K chunk, V chunk)
     static constexpr uint32_t STAGE = 2 * QK_BYTES;
-    static constexpr uint32_t ONES_OFF = STAGE_OFF + 2 * STAGE;
-    static constexpr uint32_t BYTES = ONES_OFF + 16 * 128 * 2;
+    static constexpr uint32_t BYTES = STAGE_OFF + 2 * STAGE;
     static constexpr uint32_t COLS = D == 32 ? 128 : 256;
     static constexpr int PER_SM = D == 32 ? 4 : 2;
 };
@@ -366,10 +365,9 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
     using L = BsaPipe<D>;
     constexpr int KCH = D / 8;
     constexpr int UPT = 128 * KCH / kTcThreads;
-    constexpr uint32_t QK_SBO = KCH * 128, V_SBO = 16 * 128, ONES_SBO = 16 * 128;
+    constexpr uint32_t QK_SBO = KCH * 128, V_SBO = 16 * 128;
     constexpr uint32_t IDESC_S = idesc_bf16(128, false);
     constexpr uint32_t IDESC_O = idesc_bf16(D, true);
-    constexpr uint32_t IDESC_SUM = idesc_bf16(16, false);
     extern __shared__ __align__(1024) uint8_t bsm[];
     __shared__ uint32_t sKeyMask[4];
     __shared__ __align__(8) uint64_t sBarS, sBarO;
@@ -377,12 +375,6 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t base = smem_u32(bsm);
-    for (int i = tid; i < 16 * 128 * 2 / 16; i += kTcThreads) {
-        const int c = i >> 4, rr = i & 15;
-        const uint32_t off = (rr >> 3) * ONES_SBO + c * 128 + (rr & 7) * 16;
-        const uint32_t one = (rr == 0) ? 0x3F803F80u : 0u;
-        *reinterpret_cast<uint4 *>(bsm + L::ONES_OFF + off) = make_uint4(one, one, one, one);
-    }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sTmem)),
                      "r"(L::COLS)
@@ -398,7 +390,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sTmem, tS = tmem, tO = tmem + 64, tSum = tmem + 64 + D;
+    const uint32_t tmem = sTmem, tS = tmem, tO = tmem + 64;
     const uint32_t barS = smem_u32(&sBarS), barO = smem_u32(&sBarO);
     const uint32_t lanebase = uint32_t(warp * 32) << 16;
     const int ncc = (nb + 127) / 128;  // compression chunks
@@ -509,6 +501,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                 const float m_new = fmaxf(m_run, mx == -INFINITY ? -INFINITY : mx * sl2);
                 const float mref = m_new == -INFINITY ? 0.0f : m_new;
                 const float alpha = m_run == -INFINITY ? 0.0f : ex2(m_run - mref);
+                float csum = 0.0f;  // this chunk's row sum of the weights, on the FMA pipe
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     uint32_t pk[16];
@@ -524,6 +517,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                             p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
                             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                             pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                            csum += p0 + p1;
                         }
                     } else {
 #pragma unroll
@@ -536,21 +530,16 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                 __syncthreads();
                 tc_fence_after();
                 if (tid == 0 && ok) {
-                    const uint32_t so1 = base + L::ONES_OFF;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
+                    for (int kk = 0; kk < 8; ++kk)
                         mma_bf16_ts(tO, tS + kk * 8, smem_desc(sv + kk * 256, 128, V_SBO), IDESC_O, kk > 0);
-                        mma_bf16_ts(tSum, tS + kk * 8, smem_desc(so1 + kk * 256, 128, ONES_SBO), IDESC_SUM, kk > 0);
-                    }
                     mma_commit(barO);
                 }
                 ok = ok && mbar_wait(barO, nO & 1);
                 ++nO;
                 tc_fence_after();
                 if (ok) {
-                    uint32_t sb;
-                    tmem_ld1(tSum + lanebase, sb);
-                    l_run = l_run * alpha + __uint_as_float(sb);
+                    l_run = l_run * alpha + csum;
 #pragma unroll
                     for (int c32 = 0; c32 < D; c32 += 32) {
                         uint32_t o[32];
