@@ -1115,7 +1115,6 @@ __global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan
 {
     constexpr int NT = kTailRThreads;
     extern __shared__ __align__(16) uint8_t dsm[];
-    __shared__ unsigned long long scratch[NT / 32 + 1];
     const int T = P.T;
     unsigned long long *R = reinterpret_cast<unsigned long long *>(dsm);  // [2][3][T]
     unsigned long long *segpre = R + 6 * T;                              // [T/2]
@@ -1727,7 +1726,7 @@ static bool cluster_shape(const Plan &P, int &NC, int &CS)
         mx = std::max<int64_t>(mx, np);
     }
     if (mx > int64_t(kClusterMaxCtas) * kClusterMaxChunk) return false;
-    NC = 4;
+    NC = 4;  // at least four CTAs: a small cloud spread over four runs faster than in one CTA alone
     while (NC < kClusterMaxCtas && mx > int64_t(NC) * kClusterMaxChunk) NC *= 2;
     for (int b = 0; b < P.B; ++b)
         if ((P.pad[b + 1] - P.pad[b]) < int64_t(NC) * P.m) return false;  // every leaf inside one CTA
