@@ -95,6 +95,15 @@ def _peaks():
         return 6650.0, "fallback"
 
 
+def _tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s): the measured burst figure, else the recipe's fallback."""
+    try:
+        d = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(d["bf16_tflops"]), "measured bf16_tflops"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 class ClockSampler:
     """nvidia-smi samples (SM clock, throttle reasons) while the timed region runs."""
 
@@ -637,7 +646,9 @@ def main():
     e2e_value = aggregate_value(world, LAYERS, wl.n_total, e2e_steps, e_total)
 
     peak, peak_kind = _peaks()
+    tpeak, tpeak_kind = _tensor_peak()
     attn_bytes = 4 * wl.n_total * wl.H * wl.d * 2 + 4 * st.npad  # Q, K, V read + O written, perm read
+    attn_flop = 4 * wl.m * wl.d * wl.H * wl.n_total  # Q K^T and P V inside every ball
     attn_avg_ms = statistics.mean(attn_ms)
     achieved = attn_bytes / (attn_avg_ms / 1e3) / 1e9
     line = {
@@ -649,7 +660,12 @@ def main():
                    "l2": "256 MB write between timed steps", "graph": "one CUDA graph per step"},
         "roofline": {"bound": "hbm", "kernel": ROOF_KERNEL, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
-                     "bytes_per_launch": attn_bytes, "avg_launch_ms": attn_avg_ms, "traffic": roof_traffic()},
+                     "bytes_per_launch": attn_bytes, "avg_launch_ms": attn_avg_ms, "traffic": roof_traffic(),
+                     # context: the same launch against the dense bf16 tensor peak (4 m d H flop per point); at
+                     # 64 flop per byte the HBM roofline caps it near a quarter of that peak
+                     "tensor_context": {"tflops": attn_flop / (attn_avg_ms / 1e3) / 1e12,
+                                        "frac_of_dense_bf16": attn_flop / (attn_avg_ms / 1e3) / 1e12 / tpeak,
+                                        "peak_tflops": tpeak, "peak_source": tpeak_kind}},
         "breakdown_ms_per_step": {k: v / args.steps for k, v in parts.items()},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
