@@ -44,7 +44,7 @@ UNIT = "points/s"
 LAYERS = 2
 
 # DRAM traffic of one launch of the dominant kernel on this workload (ncu dram__bytes_read.sum +
-# dram__bytes_write.sum, profiles/k_ball_attn_pair_gauss_mix.md) and the hash of the attention source it was
+# dram__bytes_write.sum, mean of two launches of the bench step) and the hash of the attention source it was
 # taken on (code lines only).  Reported only while that source is unchanged; null otherwise.
 ROOF_KERNEL = "k_ball_attn_pair"
 ROOF_TRAFFIC = {"bytes": 107585280,

@@ -53,7 +53,7 @@ typedef enum {
     BT_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than *_workspace_size() */
     BT_ERR_CUDA = 5,        /* a CUDA runtime call failed */
     BT_ERR_TIMEOUT = 6,     /* an inter-block wait gave up (found on the device) */
-    BT_ERR_UNSUPPORTED = 7, /* a valid request this build does not handle */
+    BT_ERR_UNSUPPORTED = 7, /* a valid request the library does not handle */
     BT_ERR_INTERNAL = 8     /* a consistency check inside a kernel failed (found on the device);
                                the output of that call is not valid */
 } bt_status;
