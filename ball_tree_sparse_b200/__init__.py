@@ -35,6 +35,7 @@ _SIGS = {
     "bt_build_workspace_size": ([_P, _i32, _i32], _sz),
     "bt_build": ([_P, _i64, _i32, _P, _P, _sz, _P], ctypes.c_int),
     "bt_build_segmented": ([_P, _P, _i32, _i32, _P, _P, _P, _sz, _P], ctypes.c_int),
+    "bt_build_segmented_ex": ([_P, _P, _i32, _i32, _P, _P, _P, _sz, ctypes.c_uint32, _P], ctypes.c_int),
     "bt_build_device_status": ([_P, _P], ctypes.c_int),
     "bt_build_noalloc": ([_P, _i64, _i32, _P, _P, _P], ctypes.c_int),
     "bt_rotate_z": ([_P, _i64, _P, _P], ctypes.c_int),
@@ -134,6 +135,20 @@ def bt_build(coords: torch.Tensor, m: int, perm: torch.Tensor | None = None, ws:
 def bt_build_segmented(coords: torch.Tensor, offsets, m: int, perm: torch.Tensor | None = None,
                        ws: torch.Tensor | None = None, stream=None):
     """Ball trees of a batch of clouds (padded with dummies).  Returns (perm int32 [sum Npad], pad_offsets)."""
+    return _segmented("bt_build_segmented", coords, offsets, m, perm, ws, stream)
+
+
+BT_BUILD_NARROW = 1
+
+
+def bt_build_segmented_ex(coords: torch.Tensor, offsets, m: int, flags: int = 0, perm: torch.Tensor | None = None,
+                          ws: torch.Tensor | None = None, stream=None):
+    """bt_build_segmented with flags (BT_BUILD_NARROW: half the SMs per cloud, for a build beside other
+    kernels); the result does not depend on the flags."""
+    return _segmented("bt_build_segmented_ex", coords, offsets, m, perm, ws, stream, flags)
+
+
+def _segmented(name, coords, offsets, m, perm, ws, stream, *flags):
     off = _offsets_array(offsets)
     B = len(off) - 1
     pad = np.zeros(B + 1, np.int64)
@@ -142,9 +157,8 @@ def bt_build_segmented(coords: torch.Tensor, offsets, m: int, perm: torch.Tensor
         perm = torch.empty(sum(sizes), dtype=torch.int32, device=coords.device)
     if ws is None:
         ws = workspace(off, m, coords.device)
-    _check("bt_build_segmented",
-           _lib.bt_build_segmented(_dptr(coords), off.ctypes.data_as(_P), B, m, _dptr(perm),
-                                   pad.ctypes.data_as(_P), _dptr(ws), ws.numel(), _stream(stream)))
+    _check(name, getattr(_lib, name)(_dptr(coords), off.ctypes.data_as(_P), B, m, _dptr(perm),
+                                     pad.ctypes.data_as(_P), _dptr(ws), ws.numel(), *flags, _stream(stream)))
     return perm, pad
 
 

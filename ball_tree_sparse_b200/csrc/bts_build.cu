@@ -1293,63 +1293,103 @@ __global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan
 // ---------------------------------------------------------------------------
 // 5. whole build of clouds of at most kClusterMaxCtas * kClusterMaxChunk slots
 //    in one launch: one thread-block cluster per cloud, the cloud's lists in
-//    the distributed shared memory of its CTAs.
+//    the distributed shared memory of its CTAs as 8-byte records.
 //
-// Every list element is a 16-byte record (key x, key y, key z, cloud-local
-// id), so classifying an element against any axis' median needs no gather.
 // CTA r of a cluster holds slots r*C .. r*C+C-1 of each list (C = npad / NC).
-//   sort    - per axis, four stable 8-bit LSD passes over the cluster: every
-//             CTA ranks its slots locally (warp match + per-warp digit
-//             counts), the CTAs' digit counts are exchanged, and every record
-//             is stored into the CTA that holds its global position.
+//   sort    - three lists (X, Y, Z) of (key, id) records, four stable 8-bit
+//             LSD passes over the cluster: every CTA ranks its slots locally
+//             (ballot digit matching, per-warp digit counts), pushes its digit
+//             counts to every CTA and stores every record into the CTA that
+//             holds its global position.  The last pass stores, in place of
+//             the record, its key into the axis' sorted-key table and its
+//             position - the point's rank on that axis - into the rank table
+//             of the CTA that owns the point's id.
+//   records - every CTA packs the three ranks and the id of each of its
+//             points into one 64-bit rank record and stores it at its rank in
+//             each of the three lists.  A rank orders points by (key, id) on
+//             its axis, so every later comparison is one of ranks.
 //   levels  - while a node spans several CTAs: each CTA classifies its slots
-//             against the node's median (read from the node's lists in the
-//             owning CTAs), publishes its four left counts, sums those of
-//             the node's CTAs before it and stores every record at its
-//             position in the other list buffer of the owning CTA.  Below
-//             that, nodes lie inside one CTA and the levels run in its own
-//             shared memory.
-//   output  - perm from the index list (ids ascending inside every leaf).
+//             against the median rank on the node's widest axis (extents from
+//             the sorted-key tables at the first and last rank of each list),
+//             publishes its three left counts, sums those of the node's CTAs
+//             before it and stores every record at its position in the other
+//             list buffer of the owning CTA.  Below that, nodes lie inside one
+//             CTA and the levels run in its own shared memory.
+//   output  - perm from list X's ids (ascending inside every leaf).
 // Every CTA of a cluster takes the same sequence of cluster barriers.
 // ---------------------------------------------------------------------------
 constexpr int kClusterThreads = 512;
-constexpr int kClusterMaxChunk = 1024;  // slots per CTA: 6 lists x 16 B x 1024 = 96 KB of records
+constexpr int kClusterMaxChunk = 2048;   // slots per CTA (narrow clusters, and clouds of 32,768 slots)
+constexpr int kClusterWideChunk = 1024;  // slots per CTA of the default (wide) clusters
 constexpr int kClusterMaxCtas = 16;     // non-portable cluster size (B200 allows 16)
-constexpr int kClusterEpt = kClusterMaxChunk / kClusterThreads;     // slots per thread in a level
-static_assert(int64_t(kClusterMaxCtas) * kClusterMaxChunk < 65536, "cluster-path positions fit 16-bit lanes");
+constexpr int kClusterRankWarps = 4;    // warps that rank one axis' slots in a sort pass
+static_assert(int64_t(kClusterMaxCtas) * kClusterMaxChunk <= 65536, "ranks and ids fit 16-bit fields");
 
-__device__ __forceinline__ uint32_t rkey(const uint4 &r, int a) { return a == 0 ? r.x : (a == 1 ? r.y : r.z); }
+// Field a of a rank record: the rank on axis a (0..2) or the cloud-local id (3).
+__device__ __forceinline__ uint32_t rfield(unsigned long long r, int a) { return uint32_t(r >> (16 * a)) & 0xFFFFu; }
 
-constexpr int kClusterRankWarps = 4;  // warps that rank one axis' slots in a sort pass
-
-static size_t cluster_smem_bytes(int CS)
+__device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long v)
 {
-    // records [2][3][CS] + scratch (per-warp digit counts [3][4][256] u16 in the sort, node pivots in the
-    // levels, leaf ids at the end: 12 KB) + received digit counts [16][3][256] u16 + digit starts and offsets
-    // [2][3][256] u32
-    return size_t(6) * CS * sizeof(uint4) + size_t(12) * 1024 + size_t(kClusterMaxCtas) * 3 * 256 * 2 +
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u16(uint32_t addr, uint16_t v)
+{
+    asm volatile("st.shared::cluster.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// Split cluster barrier: arrive, other work, then wait.  Every thread of every CTA of the cluster takes
+// both, in this order, between any two cluster.sync() calls.
+__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+
+// Scratch shared by the phases in turn: per-warp digit counts [3][RW][256] u16 (sort), the rank table
+// [3][CS] u16 (last pass, records), per-node prefix, pivot rank and axis [CS/2] (u64 + u16 + u8, levels),
+// leaf ids [CS] u32 (output).
+__host__ __device__ __forceinline__ size_t cluster_scratch_bytes(int CS)
+{
+    const size_t counts = size_t(3) * kClusterRankWarps * 256 * 2, tables = size_t(6) * CS;
+    return counts > tables ? counts : tables;
+}
+
+// records [2][3][CS] u64 + sorted keys [3][CS] u32 + scratch + received digit counts [NC][3][256] u16 +
+// digit starts and offsets [2][3][256] u32
+static size_t cluster_smem_bytes(int NC, int CS)
+{
+    return size_t(6) * CS * 8 + size_t(3) * CS * 4 + cluster_scratch_bytes(CS) + size_t(NC) * 3 * 256 * 2 +
            size_t(6) * 256 * 4;
 }
 
 // NC CTAs per cluster; every cloud has a power-of-two slot count npad, and CTA r holds slots r*C..r*C+C-1
-// with C = npad / NC = 2^lc.  CS (>= every cloud's C) is the list stride in shared memory.
-template <int NC>
-__global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, int CS, const float *__restrict__ coords,
-                                                                      int32_t *__restrict__ perm, uint32_t *status)
+// with C = npad / NC = 2^lc.  CS (>= every cloud's C, <= CMAX) is the list stride in shared memory.
+template <int NC, int CMAX>
+__global__ void __launch_bounds__(kClusterThreads, 1)
+    k_cluster_build(Plan P, int CS, const float *__restrict__ coords, int32_t *__restrict__ perm, uint32_t *status)
 {
     namespace cg = cooperative_groups;
-    constexpr int NT = kClusterThreads, EPT = kClusterEpt;
+    constexpr int NT = kClusterThreads, EPT = CMAX / NT > 0 ? CMAX / NT : 1;
+    constexpr int RW = kClusterRankWarps;
+    constexpr int RQ = CMAX / RW / 32;  // rounds per ranking warp (at most)
+    static_assert(RQ >= 1 && 3 * RW <= NT / 32, "ranking warps");
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(16) uint8_t dsm[];
-    constexpr int RW = kClusterRankWarps;
-    uint4 *const recs = reinterpret_cast<uint4 *>(dsm);                   // [2][3][CS]
-    uint16_t *const wh = reinterpret_cast<uint16_t *>(recs + 6 * CS);     // [3][RW][256]; later levels reuse it
-    uint16_t *const rcv = wh + 12 * 1024 / 2;                             // [NC][3][256] every CTA's digit counts
-    uint32_t *const tst = reinterpret_cast<uint32_t *>(rcv + kClusterMaxCtas * 3 * 256);  // [3][256] starts here
-    uint32_t *const off = tst + 3 * 256;                                  // [3][256] global position - local
+    unsigned long long *const recs = reinterpret_cast<unsigned long long *>(dsm);  // [2][3][CS]
+    uint32_t *const kt = reinterpret_cast<uint32_t *>(recs + 6 * CS);              // [3][CS] sorted keys
+    uint8_t *const scr = reinterpret_cast<uint8_t *>(kt + 3 * CS);
+    uint16_t *const wh = reinterpret_cast<uint16_t *>(scr);   // [3][RW][256]
+    uint16_t *const rtab = reinterpret_cast<uint16_t *>(scr); // [3][CS] rank of each of this CTA's ids
+    uint16_t *const rcv = reinterpret_cast<uint16_t *>(scr + cluster_scratch_bytes(CS));  // [NC][3][256]
+    uint32_t *const tst = reinterpret_cast<uint32_t *>(rcv + NC * 3 * 256);  // [3][256] starts here
+    uint32_t *const off = tst + 3 * 256;                                       // [3][256] global position - local
     __shared__ unsigned long long scratch[NT / 32 + 1];
     __shared__ unsigned long long s_cnt, s_excl;
-    __shared__ uint32_t s_ck[3], s_cid[3], s_pk, s_pid;
+    __shared__ uint32_t s_pr[3], s_piv;
     __shared__ float s_ext[3];
     __shared__ int s_ax;
 
@@ -1364,45 +1404,50 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
     const int m = P.m;
     const int pos0 = rank << lc;  // cloud-local position of this CTA's first slot, and id of its first point
     auto L = [&](int buf, int l) { return recs + (buf * 3 + l) * CS; };
+    // the key at rank r of axis a (every rank below npad by the bounds checks of its callers)
+    auto key_at = [&](int a, uint32_t r) { return ld_cluster_u32(cluster_addr(kt + a * CS + (r & cmask), r >> lc)); };
 
-    // --- records of this CTA's points; every list starts in id order -------
-    // (three lists, X, Y and Z; records carry the id, so no index list is kept: leaves are sorted by id last)
+    // No CTA touches another's shared memory before every CTA of the cluster has started (this arrive, and
+    // its wait before the first remote store), or after that CTA may have exited (the arrive after the last
+    // remote load, and its wait at the end).
+    cluster_arrive_relaxed();
+
+    // --- (key, id) records of this CTA's points; every list starts in id order
     for (int i = tid; i < C; i += NT) {
         const int id = pos0 + i;
-        uint4 r = make_uint4(kDummyKey, kDummyKey, kDummyKey, uint32_t(id));
+        uint32_t k[3] = {kDummyKey, kDummyKey, kDummyKey};
         if (id < n) {
             const float *c = coords + (P.row0[b] + id) * 3;
             const float x = c[0], y = c[1], z = c[2];
             if (!isfinite(x) || !isfinite(y) || !isfinite(z)) record_error(status, BT_ERR_NONFINITE);
-            r.x = float_key(x);
-            r.y = float_key(y);
-            r.z = float_key(z);
+            k[0] = float_key(x);
+            k[1] = float_key(y);
+            k[2] = float_key(z);
         }
 #pragma unroll
-        for (int l = 0; l < 3; ++l) L(0, l)[i] = r;
+        for (int l = 0; l < 3; ++l) L(0, l)[i] = k[l] | (uint64_t(id) << 32);
     }
 
-    // --- presort: lists 0..2 end sorted by (key of their axis, id) ---------
-    // Warps 4a..4a+3 rank axis a: warp 4a+w takes the w-th quarter of the CTA's slots, 32 per round.
-    constexpr int RQ = kClusterMaxChunk / RW / 32;  // rounds per ranking warp (at most)
-    const int QW = C >= RW * 32 ? C / RW : 32;      // slots of one ranking warp's contiguous block
-    const int ra = warp / RW, rw = warp % RW;       // axis and quarter of a ranking warp (ra < 3)
+    // --- presort: list a ends sorted by (key of axis a, id) -----------------
+    // Warps RW*a..RW*a+RW-1 rank axis a: warp RW*a+w takes the w-th block of the CTA's slots, 32 per round.
+    const int QW = C >= RW * 32 ? C / RW : 32;  // slots of one ranking warp's contiguous block
+    const int ra = warp / RW, rw = warp % RW;   // axis and block of a ranking warp (ra < 3)
     const uint32_t lt = (1u << lane) - 1u;
     for (int pass = 0; pass < 4; ++pass) {
         const int sh = 8 * pass;
         for (int i = tid; i < 3 * RW * 256 / 8; i += NT) reinterpret_cast<uint4 *>(wh)[i] = make_uint4(0, 0, 0, 0);
         __syncthreads();
-        uint4 rec[RQ];
+        unsigned long long rec[RQ];
         uint32_t dig[RQ], rnk[RQ];
         if (ra < 3) {
-            const uint4 *cur = L(0, ra);
+            const unsigned long long *cur = L(0, ra);
             uint16_t *w = wh + (ra * RW + rw) * 256;
 #pragma unroll
             for (int q = 0; q < RQ; ++q) {
                 const int e = rw * QW + q * 32 + lane;
                 const bool ok = q * 32 < QW && e < C;
-                rec[q] = ok ? cur[e] : make_uint4(0, 0, 0, 0);
-                dig[q] = ok ? ((rkey(rec[q], ra) >> sh) & 255u) : 256u;
+                rec[q] = ok ? cur[e] : 0ull;
+                dig[q] = ok ? ((uint32_t(rec[q]) >> sh) & 255u) : 256u;
             }
 #pragma unroll
             for (int q = 0; q < RQ; ++q) {
@@ -1437,6 +1482,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
             for (int a = 0; a < 3; ++a) tst[a * 256 + tid] = uint32_t((ts >> (16 * a)) & 0xFFFFu);
         }
         __syncthreads();
+        if (pass == 0) cluster_wait_acquire();  // every CTA of the cluster has started
         // push this CTA's digit counts to every other CTA of the cluster (posted stores)
         for (int i = tid; i < (NC - 1) * 96; i += NT) {
             const int c = (rank + 1 + i / 96) % NC, part = i % 96;
@@ -1444,7 +1490,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
             st_cluster_v4(cluster_addr(reinterpret_cast<const uint4 *>(rcv + rank * 3 * 256) + part, c), v);
         }
         if (ra < 3) {
-            uint4 *stg = L(1, ra);
+            unsigned long long *stg = L(1, ra);
             const uint16_t *w = wh + (ra * RW + rw) * 256;
 #pragma unroll
             for (int q = 0; q < RQ; ++q)
@@ -1476,22 +1522,42 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         __syncthreads();
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
-            const uint4 *stg = L(1, a);
+            const unsigned long long *stg = L(1, a);
             for (int j = tid; j < C; j += NT) {
-                const uint4 r = stg[j];
-                const uint32_t g = off[a * 256 + ((rkey(r, a) >> sh) & 255u)] + uint32_t(j);
-                if (g >= uint32_t(npad)) {  // counts disagree: never store outside the cluster's lists
+                const unsigned long long r = stg[j];
+                const uint32_t key = uint32_t(r), id = uint32_t(r >> 32);
+                const uint32_t g = off[a * 256 + ((key >> sh) & 255u)] + uint32_t(j);
+                if (g >= uint32_t(npad) || id >= uint32_t(npad)) {  // never store outside the cluster's lists
                     record_error(status, BT_ERR_INTERNAL);
                     continue;
                 }
-                st_cluster_v4(cluster_addr(L(0, a) + (g & cmask), g >> lc), r);
+                if (pass < 3) {
+                    st_cluster_u64(cluster_addr(L(0, a) + (g & cmask), g >> lc), r);
+                } else {  // g is the point's rank on axis a
+                    st_cluster_u32(cluster_addr(kt + a * CS + (g & cmask), g >> lc), key);
+                    st_cluster_u16(cluster_addr(rtab + a * CS + (id & cmask), id >> lc), uint16_t(g));
+                }
             }
         }
-        cluster.sync();  // every record is in place for the next pass
+        cluster.sync();  // every record (last pass: every key and rank) is in place
     }
 
+    // --- rank records, stored at their rank in each list (buffer 1) ---------
+    for (int i = tid; i < C; i += NT) {
+        const uint32_t r3[3] = {rtab[i], rtab[CS + i], rtab[2 * CS + i]};
+        if (r3[0] >= uint32_t(npad) || r3[1] >= uint32_t(npad) || r3[2] >= uint32_t(npad)) {
+            record_error(status, BT_ERR_INTERNAL);
+            continue;
+        }
+        const unsigned long long rec = r3[0] | (uint64_t(r3[1]) << 16) | (uint64_t(r3[2]) << 32) |
+                                       (uint64_t(pos0 + i) << 48);
+#pragma unroll
+        for (int a = 0; a < 3; ++a) st_cluster_u64(cluster_addr(L(1, a) + (r3[a] & cmask), r3[a] >> lc), rec);
+    }
+    cluster.sync();  // every list holds its rank records
+
     // --- levels whose nodes span several CTAs ------------------------------
-    int cb = 0;
+    int cb = 1;
     int ls = lnp;  // log2 of the node size
     while ((1 << ls) > m && ls > lc) {
         const int s = 1 << ls, half = s >> 1;
@@ -1501,19 +1567,21 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         const int nreal = max(0, min(s, n - nstart));
         if (tid < 3) {
             const int a = tid;
-            const uint4 *La = L(cb, a);
+            const unsigned long long *La = L(cb, a);
             const int pm = nstart + half;
-            const uint4 med = ld_cluster_v4(cluster_addr(La + (pm & cmask), pm >> lc));
+            const unsigned long long med = ld_cluster_u64(cluster_addr(La + (pm & cmask), pm >> lc));
             float e = 0.0f;
             if (nreal > 0) {
                 const int p1 = nstart + nreal - 1;
-                const uint4 f = ld_cluster_v4(cluster_addr(La + (nstart & cmask), nstart >> lc));
-                const uint4 l = ld_cluster_v4(cluster_addr(La + (p1 & cmask), p1 >> lc));
-                e = __fsub_rn(key_float(rkey(l, a)), key_float(rkey(f, a)));
+                const uint32_t r0 = rfield(ld_cluster_u64(cluster_addr(La + (nstart & cmask), nstart >> lc)), a);
+                const uint32_t r1 = rfield(ld_cluster_u64(cluster_addr(La + (p1 & cmask), p1 >> lc)), a);
+                if (r0 >= uint32_t(npad) || r1 >= uint32_t(npad))
+                    record_error(status, BT_ERR_INTERNAL);
+                else
+                    e = __fsub_rn(key_float(key_at(a, r1)), key_float(key_at(a, r0)));
             }
             s_ext[a] = e;
-            s_ck[a] = rkey(med, a);
-            s_cid[a] = med.w;
+            s_pr[a] = rfield(med, a);
         }
         __syncthreads();
         if (tid == 0) {
@@ -1521,15 +1589,14 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
             if (s_ext[1] > s_ext[ax]) ax = 1;
             if (s_ext[2] > s_ext[ax]) ax = 2;
             s_ax = ax;
-            s_pk = s_ck[ax];
-            s_pid = s_cid[ax];
+            s_piv = s_pr[ax];
         }
         __syncthreads();
         const int ax = s_ax;
-        const uint32_t pk = s_pk, pid = s_pid;
+        const uint32_t piv = s_piv;
         const int ept = C >= NT ? C / NT : 1;
         const int i0 = tid * ept;
-        uint4 v[3][EPT];
+        unsigned long long v[3][EPT];
         uint32_t lbits[3] = {0, 0, 0};
         unsigned long long packed = 0;
 #pragma unroll
@@ -1537,11 +1604,10 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
 #pragma unroll
             for (int q = 0; q < EPT; ++q) {
                 const int i = i0 + q;
-                v[l][q] = make_uint4(0, 0, 0, 0);
+                v[l][q] = 0ull;
                 if (q < ept && i < C) {
                     v[l][q] = L(cb, l)[i];
-                    const bool left = (l == ax) ? ((j << lc) + i < half)
-                                                : before(rkey(v[l][q], ax), v[l][q].w, pk, pid);
+                    const bool left = (l == ax) ? ((j << lc) + i < half) : (rfield(v[l][q], ax) < piv);
                     if (left) {
                         lbits[l] |= 1u << q;
                         packed += 1ull << (16 * l);
@@ -1565,7 +1631,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         for (int l = 0; l < 3; ++l) {
             const int excl = int((exn >> (16 * l)) & 0xFFFFu);
             int run = int((ex >> (16 * l)) & 0xFFFFu);
-            uint4 *Ln = L(cb ^ 1, l);
+            unsigned long long *Ln = L(cb ^ 1, l);
 #pragma unroll
             for (int q = 0; q < EPT; ++q) {
                 const int i = i0 + q;
@@ -1581,7 +1647,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                     if ((pos >> lc) == rank)  // stays in this CTA (the split axis' own list always does)
                         Ln[pos & cmask] = v[l][q];
                     else
-                        st_cluster_v4(cluster_addr(Ln + (pos & cmask), pos >> lc), v[l][q]);
+                        st_cluster_u64(cluster_addr(Ln + (pos & cmask), pos >> lc), v[l][q]);
                 }
             }
         }
@@ -1592,10 +1658,9 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
 
     // --- levels inside this CTA --------------------------------------------
     {
-        uint32_t *spk = reinterpret_cast<uint32_t *>(wh);                  // [C/2] pivot key per node
-        uint32_t *spid = spk + kClusterMaxChunk / 2;                        // [C/2] pivot id
-        unsigned long long *segpre = reinterpret_cast<unsigned long long *>(spid + kClusterMaxChunk / 2);  // [C/2]
-        uint8_t *sax = reinterpret_cast<uint8_t *>(segpre + kClusterMaxChunk / 2);                        // [C/2]
+        unsigned long long *segpre = reinterpret_cast<unsigned long long *>(scr);  // [C/2] left counts before a node
+        uint16_t *spr = reinterpret_cast<uint16_t *>(segpre + CS / 2);            // [C/2] pivot rank per node
+        uint8_t *sax = reinterpret_cast<uint8_t *>(spr + CS / 2);                 // [C/2] split axis per node
         const int ept = C >= NT ? C / NT : 1;
         const int i0 = tid * ept;
         for (; (1 << ls) > m; --ls) {
@@ -1606,20 +1671,22 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                 float e[3] = {0.0f, 0.0f, 0.0f};
                 if (nr > 0) {
 #pragma unroll
-                    for (int a = 0; a < 3; ++a)
-                        e[a] = __fsub_rn(key_float(rkey(L(cb, a)[start + nr - 1], a)),
-                                         key_float(rkey(L(cb, a)[start], a)));
+                    for (int a = 0; a < 3; ++a) {
+                        const uint32_t r0 = rfield(L(cb, a)[start], a), r1 = rfield(L(cb, a)[start + nr - 1], a);
+                        if (r0 >= uint32_t(npad) || r1 >= uint32_t(npad))
+                            record_error(status, BT_ERR_INTERNAL);
+                        else
+                            e[a] = __fsub_rn(key_float(key_at(a, r1)), key_float(key_at(a, r0)));
+                    }
                 }
                 int ax = 0;
                 if (e[1] > e[ax]) ax = 1;
                 if (e[2] > e[ax]) ax = 2;
-                const uint4 med = L(cb, ax)[start + half];
                 sax[q] = uint8_t(ax);
-                spk[q] = rkey(med, ax);
-                spid[q] = med.w;
+                spr[q] = uint16_t(rfield(L(cb, ax)[start + half], ax));
             }
             __syncthreads();
-            uint4 v[3][EPT];
+            unsigned long long v[3][EPT];
             uint32_t lbits[3] = {0, 0, 0};
             unsigned long long packed = 0;
 #pragma unroll
@@ -1628,11 +1695,11 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
                 if (q < ept && i < C) {
                     const int sub = i >> ls, off_in = i & (sz - 1);
                     const int ax = sax[sub];
-                    const uint32_t pk = spk[sub], pid = spid[sub];
+                    const uint32_t pr = spr[sub];
 #pragma unroll
                     for (int l = 0; l < 3; ++l) {
                         v[l][q] = L(cb, l)[i];
-                        const bool left = (l == ax) ? off_in < half : before(rkey(v[l][q], ax), v[l][q].w, pk, pid);
+                        const bool left = (l == ax) ? off_in < half : rfield(v[l][q], ax) < pr;
                         if (left) {
                             lbits[l] |= 1u << q;
                             packed += 1ull << (16 * l);
@@ -1682,11 +1749,14 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         }
     }
 
+    // the in-CTA levels read other CTAs' sorted-key tables: no CTA leaves before all of them are done
+    cluster_arrive_release();
+
     // --- perm: every leaf's ids (from list X), sorted ascending (bitonic in place) ----
-    uint32_t *ids = reinterpret_cast<uint32_t *>(wh);  // [C]
+    uint32_t *ids = reinterpret_cast<uint32_t *>(scr);  // [C]
     {
-        const uint4 *X = L(cb, 0);
-        for (int i = tid; i < C; i += NT) ids[i] = X[i].w;
+        const unsigned long long *X = L(cb, 0);
+        for (int i = tid; i < C; i += NT) ids[i] = rfield(X[i], 3);
     }
     __syncthreads();
     for (int kk = 2; kk <= m; kk <<= 1) {
@@ -1707,6 +1777,7 @@ __global__ void __launch_bounds__(kClusterThreads, 1) k_cluster_build(Plan P, in
         const uint32_t id = ids[i];
         perm[P.pad[b] + pos0 + i] = int(id) < n ? int32_t(P.row0[b] + id) : -1;
     }
+    cluster_wait_acquire();
 }
 
 static size_t tail_smem_bytes(int T)
@@ -1715,9 +1786,11 @@ static size_t tail_smem_bytes(int T)
     return size_t(T) * 16 + size_t(T / 2) * (8 + 4 + 2 + 1) + size_t(8) * T * 2 + 16;
 }
 
-// Cluster size and list stride for the one-launch path, or false when a cloud does not fit it: every cloud's
-// slot count must be a power of two (m a power of two) of at most kClusterMaxCtas * kClusterMaxChunk.
-static bool cluster_shape(const Plan &P, int &NC, int &CS)
+// Cluster size, chunk bound and list stride for the one-launch path, or false when a cloud does not fit it:
+// every cloud's slot count must be a power of two (m a power of two) of at most kClusterMaxCtas *
+// kClusterMaxChunk.  Wide clusters hold 1,024 slots per CTA (the fastest build of one batch on an idle
+// device); narrow ones 2,048, so a cloud takes half the SMs.
+static bool cluster_shape(const Plan &P, bool narrow, int &NC, int &CMAX, int &CS)
 {
     int64_t mx = 0;
     for (int b = 0; b < P.B; ++b) {
@@ -1726,22 +1799,24 @@ static bool cluster_shape(const Plan &P, int &NC, int &CS)
         mx = std::max<int64_t>(mx, np);
     }
     if (mx > int64_t(kClusterMaxCtas) * kClusterMaxChunk) return false;
+    const int chunk = narrow ? kClusterMaxChunk : kClusterWideChunk;
+    CMAX = mx > int64_t(kClusterMaxCtas) * chunk ? kClusterMaxChunk : chunk;
     NC = 4;  // at least four CTAs: a small cloud spread over four runs faster than in one CTA alone
-    while (NC < kClusterMaxCtas && mx > int64_t(NC) * kClusterMaxChunk) NC *= 2;
+    while (NC < kClusterMaxCtas && mx > int64_t(NC) * CMAX) NC *= 2;
     for (int b = 0; b < P.B; ++b)
         if ((P.pad[b + 1] - P.pad[b]) < int64_t(NC) * P.m) return false;  // every leaf inside one CTA
-    CS = int(mx / NC);
+    CS = int(std::max<int64_t>(mx / NC, 16));  // a stride of at least 16 keeps every array 16-byte aligned
     return true;
 }
 
-template <int NC>
+template <int NC, int CMAX>
 static cudaError_t cluster_launch(const Plan &P, int CS, const float *coords, int32_t *perm, uint32_t *status,
                                   cudaStream_t st, int *max_clusters)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(P.B * NC));
     cfg.blockDim = dim3(kClusterThreads);
-    cfg.dynamicSmemBytes = cluster_smem_bytes(CS);
+    cfg.dynamicSmemBytes = cluster_smem_bytes(NC, CS);
     cfg.stream = st;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -1751,48 +1826,61 @@ static cudaError_t cluster_launch(const Plan &P, int CS, const float *coords, in
     cfg.attrs = at;
     cfg.numAttrs = 1;
     if (max_clusters) {  // set-up query: attributes, then how many such clusters fit the device
-        cudaError_t e = cudaFuncSetAttribute(k_cluster_build<NC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(cluster_smem_bytes(kClusterMaxChunk)));
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(k_cluster_build<NC>,
+        cudaError_t e = cudaFuncSetAttribute(k_cluster_build<NC, CMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(cluster_smem_bytes(NC, CMAX)));
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(k_cluster_build<NC, CMAX>,
                                                        cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         cfg.gridDim = dim3(unsigned(NC));
-        cfg.dynamicSmemBytes = cluster_smem_bytes(kClusterMaxChunk);
-        if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(max_clusters, k_cluster_build<NC>, &cfg);
+        cfg.dynamicSmemBytes = cluster_smem_bytes(NC, CMAX);
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveClusters(max_clusters, k_cluster_build<NC, CMAX>, &cfg);
         return e;
     }
-    return cudaLaunchKernelEx(&cfg, k_cluster_build<NC>, P, CS, coords, perm, status);
+    return cudaLaunchKernelEx(&cfg, k_cluster_build<NC, CMAX>, P, CS, coords, perm, status);
 }
 
-static cudaError_t cluster_dispatch(int NC, const Plan &P, int CS, const float *coords, int32_t *perm,
+static cudaError_t cluster_dispatch(int NC, int CMAX, const Plan &P, int CS, const float *coords, int32_t *perm,
                                     uint32_t *status, cudaStream_t st, int *max_clusters)
 {
-    switch (NC) {
-    case 4: return cluster_launch<4>(P, CS, coords, perm, status, st, max_clusters);
-    case 8: return cluster_launch<8>(P, CS, coords, perm, status, st, max_clusters);
-    case 16: return cluster_launch<16>(P, CS, coords, perm, status, st, max_clusters);
-    default: return cudaErrorInvalidValue;
+    if (CMAX == 1024) {
+        switch (NC) {
+        case 4: return cluster_launch<4, 1024>(P, CS, coords, perm, status, st, max_clusters);
+        case 8: return cluster_launch<8, 1024>(P, CS, coords, perm, status, st, max_clusters);
+        case 16: return cluster_launch<16, 1024>(P, CS, coords, perm, status, st, max_clusters);
+        default: return cudaErrorInvalidValue;
+        }
     }
+    if (CMAX == 2048) {
+        switch (NC) {
+        case 4: return cluster_launch<4, 2048>(P, CS, coords, perm, status, st, max_clusters);
+        case 8: return cluster_launch<8, 2048>(P, CS, coords, perm, status, st, max_clusters);
+        case 16: return cluster_launch<16, 2048>(P, CS, coords, perm, status, st, max_clusters);
+        default: return cudaErrorInvalidValue;
+        }
+    }
+    return cudaErrorInvalidValue;
 }
 
-// Whether clusters of NC CTAs with the largest chunk's shared memory can run on this device (cached per device).
-static bool cluster_runs(int dev, int NC)
+// How many clusters of NC CTAs with the largest chunk's shared memory the device holds at once (0: none;
+// cached per device).
+static int cluster_capacity(int dev, int NC, int CMAX)
 {
-    static int cache[64][5] = {};  // 0 unknown, 1 yes, 2 no; index log2(NC)
+    static int cache[64][5][2] = {};  // -1 none, else the count; 0 unknown; index log2(NC), CMAX / 2048
     int li = 0;
     while ((1 << li) < NC) ++li;
-    if (dev < 0 || dev >= 64 || li > 4) return false;
-    if (cache[dev][li]) return cache[dev][li] == 1;
+    const int ci = CMAX == kClusterMaxChunk ? 1 : 0;
+    if (dev < 0 || dev >= 64 || li > 4) return 0;
+    if (cache[dev][li][ci]) return std::max(cache[dev][li][ci], 0);
     int nclusters = 0;
-    const bool ok = cluster_dispatch(NC, Plan{}, kClusterMaxChunk, nullptr, nullptr, nullptr, nullptr, &nclusters) ==
+    const bool ok = cluster_dispatch(NC, CMAX, Plan{}, CMAX, nullptr, nullptr, nullptr, nullptr, &nclusters) ==
                         cudaSuccess &&
                     nclusters > 0;
     (void)cudaGetLastError();  // a refused query is not an error of this call
-    cache[dev][li] = ok ? 1 : 2;
-    return ok;
+    cache[dev][li][ci] = ok ? nclusters : -1;
+    return ok ? nclusters : 0;
 }
 
 static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm, void *ws, size_t ws_bytes,
-                              cudaStream_t st)
+                              uint32_t flags, cudaStream_t st)
 {
     const Layout L = make_layout(P);
     if (!ws) return BT_ERR_WORKSPACE;
@@ -1837,11 +1925,20 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
             return BT_ERR_CUDA;
         attrs_set[dev] = true;
     }
-    int NC = 0, CS = 0;
-    if (cluster_shape(P, NC, CS) && cluster_runs(dev, NC)) {
+    int NC = 0, CMAX = 0, CS = 0, cap = 0;
+    const bool narrow = (flags & BT_BUILD_NARROW) != 0;
+    if (cluster_shape(P, narrow, NC, CMAX, CS) && (cap = cluster_capacity(dev, NC, CMAX)) > 0) {
+        int nNC = 0, nCMAX = 0, nCS = 0, ncap = 0;
+        if (!narrow && P.B > cap && cluster_shape(P, true, nNC, nCMAX, nCS) &&
+            (ncap = cluster_capacity(dev, nNC, nCMAX)) > 0 && (P.B + ncap - 1) / ncap < (P.B + cap - 1) / cap) {
+            // more clouds than wide clusters fit at once: narrow ones finish the batch in fewer waves
+            NC = nNC;
+            CMAX = nCMAX;
+            CS = nCS;
+        }
         // every cloud fits one cluster: the whole build is one launch; only the status word needs clearing
         if (cudaMemsetAsync(ws, 0, 64, st) != cudaSuccess) return BT_ERR_CUDA;
-        if (cluster_dispatch(NC, P, CS, coords, perm, status, st, nullptr) != cudaSuccess) return BT_ERR_CUDA;
+        if (cluster_dispatch(NC, CMAX, P, CS, coords, perm, status, st, nullptr) != cudaSuccess) return BT_ERR_CUDA;
         return BT_OK;
     }
     if (cudaMemsetAsync(ws, 0, L.ctrl_end, st) != cudaSuccess) return BT_ERR_CUDA;
@@ -1935,11 +2032,12 @@ extern "C" size_t bt_build_workspace_size(const int64_t *offsets, int32_t B, int
     return make_layout(P).total;
 }
 
-extern "C" bt_status bt_build_segmented(const float *coords, const int64_t *offsets, int32_t B, int32_t m,
-                                        int32_t *perm, int64_t *pad_offsets, void *ws, size_t ws_bytes,
-                                        void *stream)
+extern "C" bt_status bt_build_segmented_ex(const float *coords, const int64_t *offsets, int32_t B, int32_t m,
+                                           int32_t *perm, int64_t *pad_offsets, void *ws, size_t ws_bytes,
+                                           uint32_t flags, void *stream)
 {
     if (!coords || !perm) return BT_ERR_ARG;
+    if (flags & ~uint32_t(BT_BUILD_NARROW)) return BT_ERR_ARG;
     Plan P;
     const bt_status s = make_plan(offsets, B, m, P);
     if (s != BT_OK) return s;
@@ -1947,7 +2045,14 @@ extern "C" bt_status bt_build_segmented(const float *coords, const int64_t *offs
         if (offsets[b] <= offsets[b - 1]) return BT_ERR_ARG;
     if (pad_offsets)
         for (int b = 0; b <= B; ++b) pad_offsets[b] = P.pad[b];
-    return launch_build(coords, P, perm, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    return launch_build(coords, P, perm, ws, ws_bytes, flags, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bt_status bt_build_segmented(const float *coords, const int64_t *offsets, int32_t B, int32_t m,
+                                        int32_t *perm, int64_t *pad_offsets, void *ws, size_t ws_bytes,
+                                        void *stream)
+{
+    return bt_build_segmented_ex(coords, offsets, B, m, perm, pad_offsets, ws, ws_bytes, 0u, stream);
 }
 
 extern "C" bt_status bt_build(const float *coords, int64_t N, int32_t m, int32_t *perm, void *ws, size_t ws_bytes,
@@ -2017,7 +2122,7 @@ extern "C" bt_status bt_build_noalloc(const float *coords, int64_t N, int32_t m,
         g_static_ws_addr[dev] = addr;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    s = launch_build(coords, P, perm, g_static_ws_addr[dev], kStaticWsBytes, st);
+    s = launch_build(coords, P, perm, g_static_ws_addr[dev], kStaticWsBytes, 0u, st);
     if (s == BT_OK && status_out &&
         cudaMemcpyAsync(status_out, g_static_ws_addr[dev], sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
             cudaSuccess)

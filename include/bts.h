@@ -106,6 +106,24 @@ bt_status bt_build(const float *coords, int64_t N, int32_t m, int32_t *perm, voi
 bt_status bt_build_segmented(const float *coords, const int64_t *offsets, int32_t B, int32_t m, int32_t *perm,
                              int64_t *pad_offsets, void *ws, size_t ws_bytes, void *stream);
 
+/* Flags of bt_build_segmented_ex. */
+#define BT_BUILD_NARROW 1u
+
+/*
+ * bt_build_segmented with flags; the result is the same for every flag.
+ *   BT_BUILD_NARROW  where every cloud fits the one-launch build (power-of-two
+ *                    slot counts of at most 32,768), give each cloud half the
+ *                    SMs of the default: slower alone, for a build that runs
+ *                    beside other kernels (a second tree on another stream).
+ *                    Without it the library still picks the narrow build when
+ *                    a batch has more clouds than the device holds at once.
+ * Unknown flag bits: BT_ERR_ARG.  Other arguments and errors as for
+ * bt_build_segmented.  The pages build one tree at a time and say nothing of
+ * how the work is spread over a GPU; the flag changes only that.
+ */
+bt_status bt_build_segmented_ex(const float *coords, const int64_t *offsets, int32_t B, int32_t m, int32_t *perm,
+                                int64_t *pad_offsets, void *ws, size_t ws_bytes, uint32_t flags, void *stream);
+
 /*
  * bt_build without a caller workspace, for callers that cannot allocate
  * device memory when they build a tree: code inside a region being captured

@@ -61,6 +61,11 @@ def test_argument_errors_before_any_launch(lib):
     assert lib.bt_ball_attention(one, one, one, None, 128, 128, 32, 2, 48, 1, one, None) == 2  # d = 48
     assert lib.bt_ball_attention(one, one, one, None, 100, 100, 32, 2, 32, 1, one, None) == 2  # npad % m
     assert lib.bt_ball_attention(one, one, one, None, 128, 64, 32, 2, 32, 1, one, None) == 1  # rows < npad
+    lib.bt_build_segmented_ex.argtypes = [P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, ctypes.c_size_t,
+                                          ctypes.c_uint32, P]
+    offs = (ctypes.c_int64 * 2)(0, 1024)
+    assert lib.bt_build_segmented_ex(one, offs, 1, 32, one, None, one, 1 << 30, 2, None) == 1  # unknown flag bit
+    assert lib.bt_build_segmented_ex(None, offs, 1, 32, one, None, one, 1 << 30, 1, None) == 1
     lib.bt_gather.argtypes = [P, P, ctypes.c_int64, ctypes.c_int32, P, P]
     assert lib.bt_gather(one, one, 10, 0, one, None) == 1                   # row_bytes < 1
     i64, i32 = ctypes.c_int64, ctypes.c_int32

@@ -41,9 +41,12 @@ SINGLE = [
     (128, 128, "uniform"),
     (1, 1, "uniform"),
     (1024 * 8, 1024, "uniform"),
-    # one-launch cluster path at its largest cloud (16,384 slots)
+    # one-launch cluster path: 16,384 slots (1,024 per CTA), 32,768 slots (its largest cloud, 2,048 per CTA)
     (16384, 128, "tied"),
-    # record path (power-of-two clouds above 16,384 slots) with leaf size 1
+    (2 ** 14, 16, "tied"),
+    (2 ** 15, 256, "tied"),
+    (32768, 64, "uniform"),
+    # record path (power-of-two clouds above 32,768 slots) with leaf size 1
     (2 ** 16, 1, "tied"),
     # index-list path (m not a power of two) with several wide levels
     (3 * 2 ** 15, 3, "tied"),
@@ -74,6 +77,8 @@ def test_build_single_bit_exact(orc, n, m, kind):
                                      ([2000] * 8, 1), ([5, 1, 9], 4),
                                      # one-launch cluster path with few leaves per CTA
                                      ([1200], 4),
+                                     # cluster path, clouds of 32,768, 16,384 and 512 slots in one launch
+                                     ([20000, 9000, 300], 32), ([12000], 64),
                                      # record path: ragged counts, leaf sizes 1, 2, 16 and 64
                                      ([40000], 1), ([70000], 2), ([33000, 20000], 16), ([200000], 64)])
 def test_build_segmented_bit_exact(orc, sizes, m):
@@ -84,6 +89,23 @@ def test_build_segmented_bit_exact(orc, sizes, m):
     assert np.array_equal(got, want)
     if sum(sizes) <= 1 << 15:
         check_tree(got, pts, m, offsets)
+
+
+@pytest.mark.parametrize("sizes,m,flags", [
+    # narrow one-launch clusters (2,048 slots per CTA): 16,384-slot clouds, a ragged mix, a lone 8,192
+    ([16384] * 4, 128, 1), ([20000, 9000, 300], 32, 1), ([5000], 128, 1), ([600], 16, 1),
+    # more clouds than wide clusters fit at once: the library picks narrow ones by itself
+    ([16384] * 12, 128, 0),
+])
+def test_build_flags_bit_exact(orc, sizes, m, flags):
+    pts = np.concatenate([workloads.tied_cloud(s, 90 + i, levels=9) for i, s in enumerate(sizes)])
+    offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    want, pad = orc.build(pts, m, offsets)
+    c = torch.from_numpy(pts).to("cuda")
+    ws = bts.workspace(offsets, m)
+    got, _ = bts.bt_build_segmented_ex(c, offsets, m, flags, ws=ws)
+    assert bts.bt_build_device_status(ws) == 0
+    assert np.array_equal(got.cpu().numpy(), want)
 
 
 def test_workload_tiny(orc):
