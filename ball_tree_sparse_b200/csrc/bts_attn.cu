@@ -590,7 +590,8 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                 }
             }
             const float mxs = mx == -INFINITY ? 0.0f : mx * sl2;
-            float rsum = 0.0f;  // row sum of the weights (before their rounding to bf16 for the P V product)
+            // row sum of the weights (before their rounding to bf16 for the P V product), even and odd keys
+            float rs0 = 0.0f, rs1 = 0.0f;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pk[16];
@@ -600,15 +601,17 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                     const uint32_t cm = cmask[c];
 #pragma unroll
                     for (int j = 0; j < 32; j += 2) {
-                        float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-                        float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
+                        float p0, p1;
+                        ffma2_bcast(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), sl2, -mxs, p0, p1);
+                        p0 = ex2(p0);
+                        p1 = ex2(p1);
                         if (cm != 0xffffffffu) {
                             p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
                             p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
                         }
                         const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                         pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-                        rsum += p0 + p1;
+                        fadd2_acc(rs0, rs1, p0, p1);
                     }
                 } else {
 #pragma unroll
@@ -644,6 +647,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
             int64_t itemn = -1;
             go = head(it + 1, (it + 1) & (NS - 1), qn, itemn);
             if (ok && qcur >= 0) {
+                const float rsum = rs0 + rs1;
                 const float inv = rsum > 0.0f ? 1.0f / rsum : 0.0f;
                 const int h = int(uint32_t(item) % uint32_t(HP)) * 2 + hj;
                 uint4 *dst = reinterpret_cast<uint4 *>(O + (size_t(qcur) * H + h) * D);

@@ -111,6 +111,32 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// (y0, y1) = (x0 * s + c, x1 * s + c), each lane an IEEE fused multiply-add, in one packed FP32
+// instruction (sm_100).
+__device__ __forceinline__ void ffma2_bcast(float x0, float x1, float s, float c, float &y0, float &y1)
+{
+    asm("{\n\t.reg .b64 xa, sa, ca, da;\n\t"
+        "mov.b64 xa, {%2, %3};\n\t"
+        "mov.b64 sa, {%4, %4};\n\t"
+        "mov.b64 ca, {%5, %5};\n\t"
+        "fma.rn.f32x2 da, xa, sa, ca;\n\t"
+        "mov.b64 {%0, %1}, da;\n\t}"
+        : "=f"(y0), "=f"(y1)
+        : "f"(x0), "f"(x1), "f"(s), "f"(c));
+}
+
+// (a0, a1) += (x0, x1) in one packed FP32 instruction (sm_100).
+__device__ __forceinline__ void fadd2_acc(float &a0, float &a1, float x0, float x1)
+{
+    asm("{\n\t.reg .b64 aa, xa;\n\t"
+        "mov.b64 aa, {%0, %1};\n\t"
+        "mov.b64 xa, {%2, %3};\n\t"
+        "add.rn.f32x2 aa, aa, xa;\n\t"
+        "mov.b64 {%0, %1}, aa;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(x0), "f"(x1));
+}
+
 __device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t &r)
 {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
