@@ -903,7 +903,7 @@ __global__ void __launch_bounds__(256) k_records(Plan P, const uint32_t *__restr
 
 // One wide level on records (the same tiling and offsets as k_level, three lists of 8-byte records).
 template <int EPT>
-__global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level_r(
+__global__ void __launch_bounds__(kLevelThreads, 2) k_level_r(
     Plan P, int lev, const uint32_t *__restrict__ skeys, const unsigned long long *__restrict__ rin,
     unsigned long long *__restrict__ rout, unsigned long long *agg, uint32_t *counters, uint32_t *status)
 {
@@ -958,22 +958,20 @@ __global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level_r(
         s_ext[tid] = e;
         s_cand[tid] = pr;
     }
-    {
-        unsigned long long t[3][EPT];
+    // the tile's records stay in shared memory (not registers), so two CTAs fit an SM
 #pragma unroll
-        for (int l = 0; l < 3; ++l)
+    for (int l = 0; l < 3; ++l) {
+        unsigned long long t[EPT];
 #pragma unroll
-            for (int q = 0; q < EPT; ++q) {
-                const int i = tid + q * NT;
-                t[l][q] = i < TP ? rin[l * np + tile0 + i] : 0ull;
-            }
+        for (int q = 0; q < EPT; ++q) {
+            const int i = tid + q * NT;
+            t[q] = i < TP ? rin[l * np + tile0 + i] : 0ull;
+        }
 #pragma unroll
-        for (int l = 0; l < 3; ++l)
-#pragma unroll
-            for (int q = 0; q < EPT; ++q) {
-                const int i = tid + q * NT;
-                if (i < TP) sr[l * TP + i] = t[l][q];
-            }
+        for (int q = 0; q < EPT; ++q) {
+            const int i = tid + q * NT;
+            if (i < TP) sr[l * TP + i] = t[q];
+        }
     }
     __syncthreads();
     if (tid == 0) {
@@ -990,7 +988,6 @@ __global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level_r(
     // per-(round, warp) counts in slot order gives the tile's offsets
     const int lane = tid & 31, warp = tid >> 5;
     const uint32_t lt = (1u << lane) - 1u;
-    unsigned long long v[3][EPT];
     uint32_t bal[3][EPT];
 #pragma unroll
     for (int l = 0; l < 3; ++l)
@@ -998,11 +995,7 @@ __global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level_r(
         for (int q = 0; q < EPT; ++q) {
             const int i = q * NT + tid;
             bool left = false;
-            v[l][q] = 0ull;
-            if (i < TP) {
-                v[l][q] = sr[l * TP + i];
-                left = (l == ax) ? (int64_t(j) * TP + i < half) : (rrank(v[l][q], ax) < prank);
-            }
+            if (i < TP) left = (l == ax) ? (int64_t(j) * TP + i < half) : (rrank(sr[l * TP + i], ax) < prank);
             bal[l][q] = __ballot_sync(0xffffffffu, left);
             if (lane == 0) s_wcnt[l][q][warp] = uint16_t(__popc(bal[l][q]));
         }
@@ -1067,31 +1060,25 @@ __global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level_r(
             s_excl[2] = uint32_t(a2);
         }
     }
+    __syncthreads();
+    // every record straight to its place in the node: a warp's left slots land in one run of consecutive
+    // positions and its right slots in another
 #pragma unroll
     for (int l = 0; l < 3; ++l) {
-        const int nl = int(s_ltot[l]);
+        const int64_t exl = s_excl[l];
 #pragma unroll
         for (int q = 0; q < EPT; ++q) {
             const int i = q * NT + tid;
             if (i < TP) {
                 const bool left = (bal[l][q] >> lane) & 1u;
                 const int lb = int(s_wcnt[l][q][warp]) + __popc(bal[l][q] & lt);  // left slots before i
-                sr[l * TP + (left ? lb : nl + (i - lb))] = v[l][q];
+                const int64_t dst = left ? exl + lb : half + (int64_t(j) * TP - exl) + (i - lb);
+                if ((left && dst >= half) || dst < 0 || dst >= s) {
+                    record_error(status, BT_ERR_INTERNAL);
+                    continue;
+                }
+                rout[l * np + seg + dst] = sr[l * TP + i];
             }
-        }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int l = 0; l < 3; ++l) {
-        const int nl = int(s_ltot[l]);
-        const int64_t exl = s_excl[l];
-        for (int i = tid; i < TP; i += NT) {
-            const int64_t dst = i < nl ? exl + i : half + (int64_t(j) * TP - exl) + (i - nl);
-            if ((i < nl && dst >= half) || dst < 0 || dst >= s) {
-                record_error(status, BT_ERR_INTERNAL);
-                continue;
-            }
-            rout[l * np + seg + dst] = sr[l * TP + i];
         }
     }
 }
