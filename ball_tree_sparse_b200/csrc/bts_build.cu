@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kSortThreads) k_init(Plan P, const float *__re
 // 2. one stable LSD radix pass over 8 bits, all (axis, cloud) segments at once
 // ---------------------------------------------------------------------------
 template <int PASS>
-__global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32_t *__restrict__ kin,
+__global__ void __launch_bounds__(kSortThreads, 4) k_sort_pass(Plan P, const uint32_t *__restrict__ kin,
                                                             const uint32_t *__restrict__ vin,
                                                             uint32_t *__restrict__ kout, uint32_t *__restrict__ vout,
                                                             const uint32_t *__restrict__ hist, uint32_t *sst,
@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
     constexpr int NT = kSortThreads, NW = NT / 32, PER_WARP = kSortTile / NW, ROUNDS = PER_WARP / 32;
     constexpr int SHIFT = 8 * PASS;
     extern __shared__ __align__(16) uint32_t dyn[];
-    uint32_t *skey = dyn, *sval = dyn + kSortTile;
+    // sorted keys and values of the tile; the values in input order (kept out of registers: four CTAs fit an SM)
+    uint32_t *skey = dyn, *sval = dyn + kSortTile, *vin_s = dyn + 2 * kSortTile;
     __shared__ uint32_t whist[NW][256];
     __shared__ uint32_t tstart[256], gpos[256];
     __shared__ uint32_t scratch[NT / 32 + 1];
@@ -318,27 +319,25 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
     const int64_t tile_base = seg_base + int64_t(k) * kSortTile;
     const int cnt = int(min64(kSortTile, seg_size - int64_t(k) * kSortTile));
 
-    uint32_t key[ROUNDS], val[ROUNDS], dig[ROUNDS], rnk[ROUNDS];
+    uint32_t key[ROUNDS], rnk[ROUNDS];
     const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
     for (int q = 0; q < ROUNDS; ++q) {
         const int e = warp * PER_WARP + q * 32 + lane;
         const bool ok = e < cnt;
         key[q] = ok ? kin[tile_base + e] : 0u;
-        if (PASS == 0)
-            val[q] = uint32_t(P.pad[b] + int64_t(k) * kSortTile + e);
-        else
-            val[q] = ok ? vin[tile_base + e] : 0u;
-        dig[q] = ok ? ((key[q] >> SHIFT) & 255u) : (256u + lane);
+        if (ok) vin_s[e] = PASS == 0 ? uint32_t(P.pad[b] + int64_t(k) * kSortTile + e) : vin[tile_base + e];
     }
-    // stable rank of every element among equal digits of its warp, warp counts
+    // stable rank of every element among equal digits of its warp, warp counts (the digit is recomputed from
+    // the key wherever it is needed; slot e < cnt holds an element)
 #pragma unroll
     for (int q = 0; q < ROUNDS; ++q) {
-        const bool ok = dig[q] < 256u;
-        const uint32_t peers = digit_peers(dig[q], ok);
-        const uint32_t base = ok ? whist[warp][dig[q]] : 0u;
+        const bool ok = warp * PER_WARP + q * 32 + lane < cnt;
+        const uint32_t dg = (key[q] >> SHIFT) & 255u;
+        const uint32_t peers = digit_peers(dg, ok);
+        const uint32_t base = ok ? whist[warp][dg] : 0u;
         __syncwarp();
-        if (ok && (peers & lt) == 0u) whist[warp][dig[q]] = base + __popc(peers);
+        if (ok && (peers & lt) == 0u) whist[warp][dg] = base + __popc(peers);
         __syncwarp();
         rnk[q] = base + __popc(peers & lt);
     }
@@ -367,10 +366,12 @@ __global__ void __launch_bounds__(kSortThreads) k_sort_pass(Plan P, const uint32
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < ROUNDS; ++q) {
-        if (dig[q] < 256u) {
-            const uint32_t j = tstart[dig[q]] + whist[warp][dig[q]] + rnk[q];
+        const int e = warp * PER_WARP + q * 32 + lane;
+        if (e < cnt) {
+            const uint32_t dg = (key[q] >> SHIFT) & 255u;
+            const uint32_t j = tstart[dg] + whist[warp][dg] + rnk[q];
             skey[j] = key[q];
-            sval[j] = val[q];
+            sval[j] = vin_s[e];
         }
     }
     __syncthreads();
@@ -1888,7 +1889,7 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
     static bool attrs_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
-    const size_t sort_smem = size_t(2) * kSortTile * 4;
+    const size_t sort_smem = size_t(3) * kSortTile * 4;  // sorted keys, sorted values, values in input order
     const size_t tail_smem = tail_smem_bytes(P.T);
     if (dev < 64 && !attrs_set[dev]) {
         if (cudaFuncSetAttribute(k_sort_pass<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||

@@ -44,6 +44,19 @@ def test_nonfinite_reported_on_device(bad):
     assert bts.bt_build_device_status(ws) == 0
 
 
+@pytest.mark.parametrize("n,m,flags", [(4096, 32, 1), (65536, 128, 0), (3000, 16, 1)])
+def test_nonfinite_reported_on_every_build_shape(n, m, flags):
+    # narrow one-launch clusters, the record path (65,536 slots) and a padded cloud: the status word says
+    # BT_ERR_NONFINITE and a clean build on the same workspace afterwards reports OK
+    pts = workloads.uniform_cloud(n, 5)
+    pts[n // 3, 0] = np.nan
+    ws = bts.workspace([0, n], m)
+    bts.bt_build_segmented_ex(torch.from_numpy(pts).cuda(), [0, n], m, flags, ws=ws)
+    assert bts.bt_build_device_status(ws) == 3
+    bts.bt_build_segmented_ex(torch.from_numpy(workloads.uniform_cloud(n, 6)).cuda(), [0, n], m, flags, ws=ws)
+    assert bts.bt_build_device_status(ws) == 0
+
+
 def test_segmented_argument_errors():
     c = torch.zeros((10, 3), device="cuda")
     for offsets in ([0, 5, 5, 10], [1, 10], [0, 11, 10]):
