@@ -15,7 +15,7 @@
 // Kernels (all on the caller's stream):
 //   k_bsa_means    one CTA per ball: pooled query, coarse key (f32 and bf16)
 //                  and coarse value (bf16), number of real points.
-//   k_bsa_gates    one thread per row, W and an X tile in shared memory.
+//   k_bsa_gates    two rows per thread, W and an X tile in shared memory.
 //   k_bsa_topk     one CTA per (head, 8 groups), one warp per group: scores
 //                  from the pooled query and the f32 coarse keys, own ball and
 //                  empty balls masked, top-k.
@@ -138,13 +138,14 @@ __global__ void __launch_bounds__(kMeanWarps * 32) k_bsa_means(const __nv_bfloat
 }
 
 // ---------------------------------------------------------------------------
-// Gates: one thread per row, kGateOut outputs at a time in registers.  W is
-// staged once per CTA with its rows padded to a multiple of kGateOut (zeros),
-// and kGateOut/4 broadcast float4 reads of W per kGateOut FMAs.  X streams
-// through shared memory kGateCols columns at a time, double-buffered: the next
-// slice is loaded into registers (coalesced float4) while the current one is
-// used, so the loads of one slice overlap the FMAs of the other.
-constexpr int kGateRows = 128, kGateCols = 32, kGateOut = 24;
+// Gates: two rows per thread (rows t and t + kGateThreads of the CTA's
+// kGateRows), kGateOut outputs at a time in registers.  W is staged once per
+// CTA with its rows padded to a multiple of kGateOut (zeros), so one column of
+// X costs two scalar reads of X and kGateOut/4 broadcast float4 reads of W
+// for 2 * kGateOut FMAs.  X streams through shared memory kGateCols columns at
+// a time, double-buffered: the next slice is loaded into registers (coalesced
+// float4) while the current one is used.
+constexpr int kGateThreads = 128, kGateRows = 2 * kGateThreads, kGateCols = 16, kGateOut = 24;
 
 static int gate_out_padded(int H) { return (3 * H + kGateOut - 1) / kGateOut * kGateOut; }
 
@@ -153,48 +154,50 @@ static size_t gate_smem_bytes(int C, int H)
     return (size_t(C) * gate_out_padded(H) + size_t(2) * kGateRows * (kGateCols + 1)) * 4;
 }
 
-__global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict__ X, int64_t rows, int C,
-                                                         const float *__restrict__ W, const float *__restrict__ bg,
-                                                         int H, int NOP, float *__restrict__ gates)
+__global__ void __launch_bounds__(kGateThreads) k_bsa_gates(const float *__restrict__ X, int64_t rows, int C,
+                                                            const float *__restrict__ W,
+                                                            const float *__restrict__ bg, int H, int NOP,
+                                                            float *__restrict__ gates)
 {
     extern __shared__ __align__(16) float gsm[];
-    constexpr int XP = kGateCols + 1;
-    constexpr int U = kGateRows * kGateCols / 4 / kGateRows;  // float4 of a slice per thread
+    constexpr int XP = kGateCols + 1;  // odd row stride: the 32 rows a warp reads sit in 32 banks
+    constexpr int U = kGateRows * kGateCols / 4 / kGateThreads;  // float4 of a slice per thread
     const int NO = 3 * H;
     float *sW = gsm, *sX = gsm + size_t(C) * NOP;  // sX: [2][kGateRows][XP]
     const int tid = threadIdx.x;
     {
         // W rows padded to NOP columns with zeros; loads batched 8 per thread ahead of their stores
         const int total = C * NO, pad = NOP - NO;
-        for (int i0 = 0; i0 < total; i0 += 8 * kGateRows) {
+        for (int i0 = 0; i0 < total; i0 += 8 * kGateThreads) {
             float t[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u * kGateRows + tid;
+                const int i = i0 + u * kGateThreads + tid;
                 t[u] = i < total ? W[i] : 0.0f;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int i = i0 + u * kGateRows + tid;
+                const int i = i0 + u * kGateThreads + tid;
                 if (i < total) {
                     const int c = i / NO, j = i - c * NO;
                     sW[c * NOP + j] = t[u];
                 }
             }
         }
-        for (int i = tid; i < C * pad; i += kGateRows) {
+        for (int i = tid; i < C * pad; i += kGateThreads) {
             const int c = i / pad, j = NO + (i - c * pad);
             sW[c * NOP + j] = 0.0f;
         }
     }
-    const int64_t r0 = int64_t(blockIdx.x) * kGateRows, r = r0 + tid;
+    const int64_t r0 = int64_t(blockIdx.x) * kGateRows;
+    const int64_t ra = r0 + tid, rb = ra + kGateThreads;  // this thread's two rows
     const bool vec4 = (C % 4) == 0 && (reinterpret_cast<uintptr_t>(X) % 16) == 0;
     const int nslice = (C + kGateCols - 1) / kGateCols;
     // one slice of X into registers: row rr = i / (kGateCols/4), columns c0 + 4*(i % (kGateCols/4)) .. +3
     auto load_slice = [&](int c0, float4 (&t)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+            const int i = tid + u * kGateThreads, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
             const int c = c0 + 4 * c4;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (r0 + rr < rows) {
@@ -214,7 +217,7 @@ __global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict
     auto store_slice = [&](int buf, const float4 (&t)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = tid + u * kGateRows, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+            const int i = tid + u * kGateThreads, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
             float *d = sX + (size_t(buf) * kGateRows + rr) * XP + 4 * c4;
             d[0] = t[u].x;
             d[1] = t[u].y;
@@ -222,10 +225,28 @@ __global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict
             d[3] = t[u].w;
         }
     };
-    for (int j0 = 0; j0 < NO; j0 += kGateOut) {
-        float acc[kGateOut];
+    // one column of the slice: x of both rows against kGateOut weights
+    auto column = [&](const float *xa, const float *xb, const float *wrow, float (&aa)[kGateOut],
+                      float (&ab)[kGateOut]) {
+        const float x0 = *xa, x1 = *xb;
+        const float4 *w4 = reinterpret_cast<const float4 *>(wrow);
 #pragma unroll
-        for (int j = 0; j < kGateOut; ++j) acc[j] = (bg && j0 + j < NO) ? bg[j0 + j] : 0.0f;
+        for (int j4 = 0; j4 < kGateOut / 4; ++j4) {
+            const float4 w = w4[j4];
+            aa[4 * j4] = fmaf(x0, w.x, aa[4 * j4]);
+            aa[4 * j4 + 1] = fmaf(x0, w.y, aa[4 * j4 + 1]);
+            aa[4 * j4 + 2] = fmaf(x0, w.z, aa[4 * j4 + 2]);
+            aa[4 * j4 + 3] = fmaf(x0, w.w, aa[4 * j4 + 3]);
+            ab[4 * j4] = fmaf(x1, w.x, ab[4 * j4]);
+            ab[4 * j4 + 1] = fmaf(x1, w.y, ab[4 * j4 + 1]);
+            ab[4 * j4 + 2] = fmaf(x1, w.z, ab[4 * j4 + 2]);
+            ab[4 * j4 + 3] = fmaf(x1, w.w, ab[4 * j4 + 3]);
+        }
+    };
+    for (int j0 = 0; j0 < NO; j0 += kGateOut) {
+        float acc_a[kGateOut], acc_b[kGateOut];
+#pragma unroll
+        for (int j = 0; j < kGateOut; ++j) acc_a[j] = acc_b[j] = (bg && j0 + j < NO) ? bg[j0 + j] : 0.0f;
         float4 t[U];
         load_slice(0, t);
         __syncthreads();  // W is staged; neither buffer is read any more
@@ -234,27 +255,27 @@ __global__ void __launch_bounds__(kGateRows) k_bsa_gates(const float *__restrict
         for (int k = 0; k < nslice; ++k) {
             const int c0 = k * kGateCols;
             if (k + 1 < nslice) load_slice(c0 + kGateCols, t);  // in flight while slice k is used
-            const float *xs = sX + (size_t(k & 1) * kGateRows + tid) * XP;
-            const int cw = C - c0 < kGateCols ? C - c0 : kGateCols;
-            for (int cc = 0; cc < cw; ++cc) {
-                const float x = xs[cc];
-                const float4 *w4 = reinterpret_cast<const float4 *>(sW + size_t(c0 + cc) * NOP + j0);
-#pragma unroll
-                for (int j4 = 0; j4 < kGateOut / 4; ++j4) {
-                    const float4 w = w4[j4];
-                    acc[4 * j4] = fmaf(x, w.x, acc[4 * j4]);
-                    acc[4 * j4 + 1] = fmaf(x, w.y, acc[4 * j4 + 1]);
-                    acc[4 * j4 + 2] = fmaf(x, w.z, acc[4 * j4 + 2]);
-                    acc[4 * j4 + 3] = fmaf(x, w.w, acc[4 * j4 + 3]);
-                }
+            const float *xa = sX + (size_t(k & 1) * kGateRows + tid) * XP;
+            const float *xb = xa + kGateThreads * XP;
+            const float *wr = sW + size_t(c0) * NOP + j0;
+            if (C - c0 >= kGateCols) {
+#pragma unroll 4
+                for (int cc = 0; cc < kGateCols; ++cc) column(xa + cc, xb + cc, wr + size_t(cc) * NOP, acc_a, acc_b);
+            } else {
+                for (int cc = 0; cc < C - c0; ++cc) column(xa + cc, xb + cc, wr + size_t(cc) * NOP, acc_a, acc_b);
             }
             if (k + 1 < nslice) store_slice((k + 1) & 1, t);  // the other buffer: nobody reads it now
             __syncthreads();
         }
-        if (r < rows) {
+        if (ra < rows) {
 #pragma unroll
             for (int j = 0; j < kGateOut; ++j)
-                if (j0 + j < NO) gates[r * NO + j0 + j] = 1.0f / (1.0f + expf(-acc[j]));
+                if (j0 + j < NO) gates[ra * NO + j0 + j] = 1.0f / (1.0f + expf(-acc_a[j]));
+        }
+        if (rb < rows) {
+#pragma unroll
+            for (int j = 0; j < kGateOut; ++j)
+                if (j0 + j < NO) gates[rb * NO + j0 + j] = 1.0f / (1.0f + expf(-acc_b[j]));
         }
     }
 }
@@ -914,7 +935,7 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
     }
     const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
     k_bsa_means<<<nb, kMeanWarps * 32, 0, st>>>(q, k, v, perm, rows, H * D, qbar, kbar, kc, vc, cnt);
-    k_bsa_gates<<<unsigned((rows + kGateRows - 1) / kGateRows), kGateRows, gate_smem_bytes(C, H), st>>>(
+    k_bsa_gates<<<unsigned((rows + kGateRows - 1) / kGateRows), kGateThreads, gate_smem_bytes(C, H), st>>>(
         X, rows, C, Wg, bg, H, gate_out_padded(H), gates);
     if (p.topk > 0)
         k_bsa_topk<D><<<unsigned(int64_t(H) * ((nb + kTopkWarps - 1) / kTopkWarps)), kTopkWarps * 32,
