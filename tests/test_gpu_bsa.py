@@ -87,6 +87,19 @@ def test_bsa_matches_oracle(orc, sizes, H, topk, mask_own, d, coarsen):
     assert err <= TOL, f"max abs err {err}"
 
 
+@pytest.mark.parametrize("C,H", [(13, 10), (40, 2)])
+def test_bsa_gate_shapes(orc, C, H):
+    # gate input widths that are not a multiple of 4 (scalar loads) or of the 16-column slice, and more than
+    # 24 gates per row (H = 10: two passes over the outputs)
+    q, k, v, perm, x, w, b = _case([1500, 700], H, C, 31 + C, 3)
+    got, sel = _run_gpu(q, k, v, perm, x, w, b, 3)
+    _check_selection(sel, orc.bsa(q, k, v, 128, perm, x, w, b, topk=3, mask_own=True, branches=True), 3)
+    ref = orc.bsa(q, k, v, 128, perm, x, w, b, topk=3, mask_own=True, sel_in=sel, branches=True)
+    real = perm[perm >= 0]
+    err = np.abs(got[real] - ref["O"][real]).max()
+    assert err <= TOL, f"max abs err {err}"
+
+
 def test_bsa_selection_pinned_by_exact_ties(orc):
     # every K row equal: every score ties, so the selection is the lowest balls other than the group's own
     q, k, v, perm, x, w, b = _case([128 * 8], 2, 16, 5, 3)
