@@ -2,24 +2,28 @@
 // permutation (the tree of "Erwin: A Tree-based Hierarchical Transformer for
 // Large-scale Physical Systems", author's thread posts 6/N, 9/N and 15/N).
 //
-// Design (sm_100a, one cloud or a batch of clouds):
-//   1. k_init       - per point: fold -0, reject NaN/Inf, write the order-
-//                     preserving keys of x, y, z, the index list, and the
-//                     digit histograms of all four radix passes.
-//   2. k_sort_pass  - four stable 8-bit LSD radix passes that sort, inside
-//                     every cloud, the point ids by each axis' key (ties by
-//                     id).  One launch per pass, tiles chained by a bounded
-//                     decoupled look-back.  Result: lists X, Y, Z.
-//   3. k_level      - one launch per "wide" tree level (nodes larger than the
-//                     shared-memory tail).  A node's widest axis comes from
-//                     the two ends of its sorted lists, its median is the
-//                     element at position s/2 of that axis' list, and all four
-//                     lists (X, Y, Z and the index list I) are split by a
-//                     stable partition, so each stays sorted inside every
-//                     child.  No select pass is needed at any level.
-//   4. k_tail       - one CTA per node of at most T slots finishes all
-//                     remaining levels in shared memory and writes perm from
-//                     the index list (leaves come out in ascending index).
+// Design (sm_100a, one cloud or a batch of clouds).  Every shape sorts each
+// cloud once per axis (order-preserving float keys, ties by id) and then splits
+// the three sorted lists stably at every level: a node's widest axis comes from
+// the two ends of its lists, its median is the element at position s/2 of that
+// axis' list, and every list stays sorted inside both children, so no level
+// needs a selection.  Three shapes of this algorithm, chosen per call:
+//   a. k_cluster_build - clouds of at most 32,768 slots (power-of-two slot
+//                     counts): the whole build in one launch, one thread-block
+//                     cluster per cloud, the lists in distributed shared
+//                     memory as 8-byte records ((key, id) while sorting, the
+//                     point's three ranks and id afterwards).
+//   b. record path  - larger power-of-two clouds (at most 2^21 slots): k_init
+//                     (keys, digit histograms), four radix passes
+//                     (k_sort_pass, tiles chained by a bounded decoupled
+//                     look-back), k_records (every list element becomes the
+//                     point's three ranks), one k_level_r launch per level
+//                     whose nodes exceed the shared-memory tail, and k_tail_r
+//                     (the remaining levels in shared memory, leaves sorted by
+//                     id).
+//   c. index lists  - any other shape: the same presort, then k_level and
+//                     k_tail on the lists X, Y, Z and the index list I, with
+//                     the keys gathered through the lists.
 #include <algorithm>
 #include <cstring>
 
@@ -34,7 +38,7 @@ constexpr int kSortThreads = 256;
 constexpr int kLevelThreads = 512;
 constexpr int kLevelTileMin = 512;       // smallest wide-level tile, slots per list (or m when m is larger)
 constexpr int kLevelTileMax = 4096;      // largest: eight slots of each list per thread
-constexpr int kLevelTilesWanted = 148;   // large builds: about one wide-level tile per SM
+constexpr int kLevelTilesWanted = 148;   // large builds: about one wide-level tile per SM (two fit one)
 constexpr int kTailMax = 4096;         // largest node finished in shared memory
 constexpr int kTailMin = 512;          // smallest tail node (for m <= 512)
 constexpr int kTailCtasWanted = 2 * 148;  // aim for two tail CTAs per SM
@@ -202,16 +206,6 @@ __device__ __forceinline__ unsigned long long ld_cluster_u64(uint32_t addr)
 {
     unsigned long long v;
     asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr)
-{
-    uint4 v;
-    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(addr)
-                 : "memory");
     return v;
 }
 
