@@ -94,6 +94,8 @@ def test_build_segmented_bit_exact(orc, sizes, m):
 @pytest.mark.parametrize("sizes,m,flags", [
     # narrow one-launch clusters (2,048 slots per CTA): 16,384-slot clouds, a ragged mix, a lone 8,192
     ([16384] * 4, 128, 1), ([20000, 9000, 300], 32, 1), ([5000], 128, 1), ([600], 16, 1),
+    # leaf size 1: every level down to single slots (the most in-CTA levels and node pivots)
+    ([32768], 1, 0), ([8192], 1, 1), ([5000, 2100], 1, 0),
     # more clouds than wide clusters fit at once: the library picks narrow ones by itself
     ([16384] * 12, 128, 0),
 ])
