@@ -424,6 +424,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     __shared__ int64_t sItem[NS];       // the stage's item, -1 when the CTA has no more work
     __shared__ int64_t sClaim;          // next item, claimed by the first producer thread
     __shared__ int sAbort[2];           // a head's warpgroup stops after a wait that ran out
+    __shared__ int sLive[2];            // per producer warp: some row of the claimed item is a real point
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m = 1 << lm;
@@ -481,6 +482,25 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         int32_t crow[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) crow[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
+        // An item whose 128 slots are all dummies (the padding at the end of a cloud) has no output: it is
+        // replaced by the next claimed item before it takes a stage.  A perm entry outside Q/K/V counts as a
+        // real row here, so the item still goes through the checks below.
+        auto skip_dead = [&]() {
+            while (item < items) {
+                const bool live = lane < 16 && (crow[0] >= 0 || crow[1] >= 0 || crow[2] >= 0 || crow[3] >= 0);
+                const uint32_t bw = __ballot_sync(0xffffffffu, live);
+                if (lane == 0) sLive[pw] = bw != 0u;
+                asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");
+                const bool dead = !sLive[0] && !sLive[1];
+                if (dead && tid == 8 * 32) sClaim = pok ? int64_t(gridDim.x) + int64_t(atomicAdd(ctr, 1u)) : items;
+                asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");  // sLive read; sClaim written
+                if (!dead) return;
+                item = sClaim;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) crow[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
+            }
+        };
+        skip_dead();
         for (int it = 0;; ++it) {
             const int stage = it & (NS - 1);
             const uint32_t bar = smem_u32(&sFull[stage]);
@@ -517,6 +537,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
             item = sClaim;
 #pragma unroll
             for (int i = 0; i < 4; ++i) crow[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
+            skip_dead();
         }
     } else {
         // ---------------- consumers ----------------
