@@ -746,14 +746,14 @@ static __device__ uint32_t g_pair_ctr[kPairCounters][2];
 static bt_status launch_pair(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
                              int64_t rows, int lm, int H, void *O, cudaStream_t st)
 {
-    static bool set[64] = {false};
+    static std::atomic<bool> set[64] = {};
     static int sms[64] = {0};
     static uint32_t *ctrs[64] = {nullptr};
     static std::atomic<uint32_t> next_pair{0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
-    if (dev >= 64) return BT_ERR_UNSUPPORTED;
-    if (!set[dev]) {
+    if (dev < 0 || dev >= 64) return BT_ERR_UNSUPPORTED;
+    const bt_status s0 = setup_once(set[dev], [&]() -> bt_status {
         if (cudaFuncSetAttribute(k_ball_attn_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(PairPipe::BYTES)))
             return BT_ERR_CUDA;
@@ -764,8 +764,9 @@ static bt_status launch_pair(const void *Q, const void *K, const void *V, const 
         if (cudaGetSymbolAddress(&addr, g_pair_ctr) != cudaSuccess || !addr) return BT_ERR_CUDA;
         ctrs[dev] = static_cast<uint32_t *>(addr);
         sms[dev] = n;
-        set[dev] = true;
-    }
+        return BT_OK;
+    });
+    if (s0 != BT_OK) return s0;
     uint32_t *ctr = ctrs[dev] + 2 * (next_pair.fetch_add(1u) % kPairCounters);
     CUtensorMap mq, mk, mv;
     if (!row_map(&mq, Q, rows, H * 32, 64) || !row_map(&mk, K, rows, H * 32, 64) || !row_map(&mv, V, rows, H * 32, 64))
@@ -801,20 +802,20 @@ static bt_status launch_tc(const void *Q, const void *K, const void *V, const in
                            int64_t rows, int lm, int H, void *O, cudaStream_t st)
 {
     constexpr size_t smem = TcPipe<D>::BYTES;
-    static bool set[64] = {false};
+    static std::atomic<bool> set[64] = {};
     static int sms[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
-    if (dev >= 64 || !set[dev]) {
+    auto init = [&]() -> bt_status {
         if (cudaFuncSetAttribute(k_ball_attn_tc2<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)))
             return BT_ERR_CUDA;
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BT_ERR_CUDA;
-        if (dev < 64) {
-            sms[dev] = n;
-            set[dev] = true;
-        }
-    }
+        if (dev >= 0 && dev < 64) sms[dev] = n;
+        return BT_OK;
+    };
+    const bt_status s0 = (dev >= 0 && dev < 64) ? setup_once(set[dev], init) : init();
+    if (s0 != BT_OK) return s0;
     const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
     const int64_t items = (npad + 127) / 128 * H;
     const int per_sm = TcPipe<D>::PER_SM;

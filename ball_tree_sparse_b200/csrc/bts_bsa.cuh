@@ -915,11 +915,11 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(Q), *k = static_cast<const __nv_bfloat16 *>(K),
                         *v = static_cast<const __nv_bfloat16 *>(V);
 
-    static bool set[64] = {false};
+    static std::atomic<bool> set[64] = {};
     static int sms[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
-    if (dev >= 64 || !set[dev]) {
+    auto init = [&]() -> bt_status {
         if (cudaFuncSetAttribute(k_bsa_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(BsaPipe<D>::BYTES)) ||
             cudaFuncSetAttribute(k_bsa_gates, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) ||
@@ -928,11 +928,11 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
             return BT_ERR_CUDA;
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BT_ERR_CUDA;
-        if (dev < 64) {
-            sms[dev] = n;
-            set[dev] = true;
-        }
-    }
+        if (dev >= 0 && dev < 64) sms[dev] = n;
+        return BT_OK;
+    };
+    const bt_status s0 = (dev >= 0 && dev < 64) ? setup_once(set[dev], init) : init();
+    if (s0 != BT_OK) return s0;
     const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
     k_bsa_means<<<nb, kMeanWarps * 32, 0, st>>>(q, k, v, perm, rows, H * D, qbar, kbar, kc, vc, cnt);
     k_bsa_gates<<<unsigned((rows + kGateRows - 1) / kGateRows), kGateThreads, gate_smem_bytes(C, H), st>>>(

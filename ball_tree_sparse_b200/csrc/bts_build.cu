@@ -1846,18 +1846,21 @@ static cudaError_t cluster_dispatch(int NC, int CMAX, const Plan &P, int CS, con
 // cached per device).
 static int cluster_capacity(int dev, int NC, int CMAX)
 {
-    static int cache[64][5][2] = {};  // -1 none, else the count; 0 unknown; index log2(NC), CMAX / 2048
+    // -1 none, else the count; 0 unknown; index log2(NC), CMAX / 2048.  Concurrent first queries from several
+    // host threads compute the same value; each entry is one atomic word.
+    static std::atomic<int> cache[64][5][2] = {};
     int li = 0;
     while ((1 << li) < NC) ++li;
     const int ci = CMAX == kClusterMaxChunk ? 1 : 0;
     if (dev < 0 || dev >= 64 || li > 4) return 0;
-    if (cache[dev][li][ci]) return std::max(cache[dev][li][ci], 0);
+    const int known = cache[dev][li][ci].load(std::memory_order_relaxed);
+    if (known) return std::max(known, 0);
     int nclusters = 0;
     const bool ok = cluster_dispatch(NC, CMAX, Plan{}, CMAX, nullptr, nullptr, nullptr, nullptr, &nclusters) ==
                         cudaSuccess &&
                     nclusters > 0;
     (void)cudaGetLastError();  // a refused query is not an error of this call
-    cache[dev][li][ci] = ok ? nclusters : -1;
+    cache[dev][li][ci].store(ok ? nclusters : -1, std::memory_order_relaxed);
     return ok ? nclusters : 0;
 }
 
@@ -1880,12 +1883,12 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
     uint32_t *lists = reinterpret_cast<uint32_t *>(w + L.lists);
     const size_t np = size_t(P.npad);
 
-    static bool attrs_set[64] = {false};
+    static std::atomic<bool> attrs_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
     const size_t sort_smem = size_t(3) * kSortTile * 4;  // sorted keys, sorted values, values in input order
     const size_t tail_smem = tail_smem_bytes(P.T);
-    if (dev < 64 && !attrs_set[dev]) {
+    auto init = [&]() -> bt_status {
         if (cudaFuncSetAttribute(k_sort_pass<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
             cudaFuncSetAttribute(k_sort_pass<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
             cudaFuncSetAttribute(k_sort_pass<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sort_smem)) ||
@@ -1905,8 +1908,10 @@ static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm,
             cudaFuncSetAttribute(k_tail<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(tail_smem_bytes(kTailMax))))
             return BT_ERR_CUDA;
-        attrs_set[dev] = true;
-    }
+        return BT_OK;
+    };
+    const bt_status s0 = (dev >= 0 && dev < 64) ? setup_once(attrs_set[dev], init) : init();
+    if (s0 != BT_OK) return s0;
     int NC = 0, CMAX = 0, CS = 0, cap = 0;
     const bool narrow = (flags & BT_BUILD_NARROW) != 0;
     if (cluster_shape(P, narrow, NC, CMAX, CS) && (cap = cluster_capacity(dev, NC, CMAX)) > 0) {
@@ -2079,7 +2084,7 @@ namespace bts {
 constexpr size_t kStaticWsBytes = size_t(8) << 20;
 constexpr int64_t kStaticMaxPoints = 65536;
 static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
-static void *g_static_ws_addr[64] = {};  // device address of g_static_ws, per device ordinal
+static std::atomic<void *> g_static_ws_addr[64] = {};  // device address of g_static_ws, per device ordinal
 }  // namespace bts
 
 extern "C" bt_status bt_build_noalloc(const float *coords, int64_t N, int32_t m, int32_t *perm, int32_t *status_out,
@@ -2097,16 +2102,17 @@ extern "C" bt_status bt_build_noalloc(const float *coords, int64_t N, int32_t m,
     if (make_layout(P).total > kStaticWsBytes) return BT_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BT_ERR_CUDA;
-    if (!g_static_ws_addr[dev]) {
-        // host code only sees a stand-in for the array: ask the runtime for its device address
-        void *addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_static_ws) != cudaSuccess || !addr) return BT_ERR_CUDA;
-        g_static_ws_addr[dev] = addr;
+    void *ws = g_static_ws_addr[dev].load(std::memory_order_acquire);
+    if (!ws) {
+        // host code only sees a stand-in for the array: ask the runtime for its device address (the same
+        // address for every thread that asks)
+        if (cudaGetSymbolAddress(&ws, g_static_ws) != cudaSuccess || !ws) return BT_ERR_CUDA;
+        g_static_ws_addr[dev].store(ws, std::memory_order_release);
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    s = launch_build(coords, P, perm, g_static_ws_addr[dev], kStaticWsBytes, 0u, st);
+    s = launch_build(coords, P, perm, ws, kStaticWsBytes, 0u, st);
     if (s == BT_OK && status_out &&
-        cudaMemcpyAsync(status_out, g_static_ws_addr[dev], sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+        cudaMemcpyAsync(status_out, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
             cudaSuccess)
         return BT_ERR_CUDA;
     return s;

@@ -1,12 +1,29 @@
 // Internal helpers shared by the libbts kernels (device code for sm_100a).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "bts.h"
 
 namespace bts {
+
+// First-time set-up of per-device host state (function attributes, SM counts, symbol addresses): `init`
+// runs under one lock until it succeeds, and `ready` turns true (release) after it, so concurrent first calls
+// from several host threads neither race nor repeat it.  Returns init's status, BT_OK once set up.
+template <typename F>
+inline bt_status setup_once(std::atomic<bool> &ready, F &&init)
+{
+    if (ready.load(std::memory_order_acquire)) return BT_OK;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (ready.load(std::memory_order_relaxed)) return BT_OK;
+    const bt_status s = init();
+    if (s == BT_OK) ready.store(true, std::memory_order_release);
+    return s;
+}
 
 // ---------------------------------------------------------------------------
 // Device status word: the first error recorded wins; 0 = no error.

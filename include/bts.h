@@ -34,6 +34,10 @@
  *    back by bt_build_device_status().  No call traps, aborts or prints.
  *  - Arrays are row-major and contiguous.  Coordinates are float [rows, 3].
  *    Q/K/V/O are [rows, H, d] (H heads of d values per row).
+ *  - Calls may come from several host threads: the per-device set-up on a
+ *    device's first call is done once, under a lock inside the library.
+ *    Workspaces (and bt_build_noalloc's static scratch) are not shared safely
+ *    between builds in flight at the same time; that is the caller's to avoid.
  */
 #ifndef BTS_H
 #define BTS_H
