@@ -1,0 +1,40 @@
+"""Host logic of bench.py that decides whether a run counts: the clock record taken during the timed region
+(median and maximum SM clock, throttle reasons), from synthetic nvidia-smi rows (no GPU, no nvidia-smi)."""
+import bench
+
+
+def _sampler(rows, marks):
+    s = bench.ClockSampler.__new__(bench.ClockSampler)  # no nvidia-smi process
+    s.rows, s.proc, s.marks = rows, None, marks
+    return s
+
+
+def _row(t, sm, reasons=("Not Active",) * 4):
+    return (t, [str(sm), "1965", "700.0", *reasons])
+
+
+def test_clock_summary_uses_the_timed_window():
+    rows = [_row(0.5, 1000), _row(1.5, 1965), _row(2.0, 1950), _row(2.5, 1965), _row(9.0, 500)]
+    out = _sampler(rows, [1.0, 3.0]).summary()
+    assert out["sm_mhz"] == 1965.0 and out["sm_max_mhz"] == 1965.0 and out["samples"] == 3
+    assert out["reasons"] == []
+
+
+def test_clock_summary_reports_active_reasons_by_name():
+    act = ("Not Active", "Active", "Not Active", "Active")  # hw_thermal_slowdown, sw_power_cap
+    rows = [_row(1.0, 1300, act), _row(1.1, 1320)]
+    out = _sampler(rows, [0.0, 2.0]).summary()
+    assert out["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert out["sm_mhz"] == 1310.0
+
+
+def test_clock_summary_without_samples():
+    out = _sampler([], [0.0, 1.0]).summary()
+    assert out["samples"] == 0 and out["sm_mhz"] is None
+    assert out["reasons"] == ["no nvidia-smi samples"]
+
+
+def test_clock_summary_falls_back_to_every_row_outside_the_window():
+    # rows that all lie outside the marks (a sampler that started late) are still summarised
+    out = _sampler([_row(5.0, 1800), _row(6.0, 1900)], [0.0, 1.0]).summary()
+    assert out["samples"] == 2 and out["sm_mhz"] == 1850.0
