@@ -38,3 +38,25 @@ def test_clock_summary_falls_back_to_every_row_outside_the_window():
     # rows that all lie outside the marks (a sampler that started late) are still summarised
     out = _sampler([_row(5.0, 1800), _row(6.0, 1900)], [0.0, 1.0]).summary()
     assert out["samples"] == 2 and out["sm_mhz"] == 1850.0
+
+
+def test_roofline_traffic_only_for_the_source_it_was_measured_on(monkeypatch):
+    h = bench.attention_source_hash()
+    monkeypatch.setattr(bench, "ROOF_TRAFFIC", {"bytes": 123, "source_sha256": h})
+    assert bench.roof_traffic() == 123
+    monkeypatch.setattr(bench, "ROOF_TRAFFIC", {"bytes": 123, "source_sha256": "0" * 64})
+    assert bench.roof_traffic() is None
+    monkeypatch.setattr(bench, "ROOF_TRAFFIC", {"bytes": None, "source_sha256": h})
+    assert bench.roof_traffic() is None
+
+
+def test_attention_source_hash_ignores_comment_lines(tmp_path, monkeypatch):
+    # the hash covers code lines only: a comment-only edit keeps a traffic figure valid
+    src = tmp_path / "k.cu"
+    src.write_text("int a;\n// note\nint b;\n")
+    monkeypatch.setattr(bench, "_ATTN_SOURCES", (str(src),))  # absolute: os.path.join keeps it as it is
+    h0 = bench.attention_source_hash()
+    src.write_text("int a;\n  // another note\nint b;\n")
+    assert bench.attention_source_hash() == h0
+    src.write_text("int a;\nint c;\n")
+    assert bench.attention_source_hash() != h0
