@@ -84,3 +84,16 @@ def test_argument_errors_before_any_launch(lib):
                                         None) == 2                          # 64 coarse tokens, ball of 128
     assert lib.bt_coarse_ball_attention(one, one, one, one, 1024, 1024, 32, 2, 32, 1, 4, one, None, 0,
                                         None) == 4                          # no workspace
+
+
+def test_binding_constants_match_the_header():
+    # the status names, dtype codes, batch limit and build flags the binding passes through the ABI
+    text = open(os.path.join(ROOT, "include", "bts.h")).read()
+    enum = dict((k, int(v)) for k, v in re.findall(r"\b(BT_[A-Z_0-9]+)\s*=\s*(\d+)", text))
+    defines = dict((k, int(v)) for k, v in re.findall(r"#define\s+(BT_[A-Z_0-9]+)\s+(\d+)u?\b", text))
+    b = pytest.importorskip("ball_tree_sparse_b200")
+    assert {v: k for k, v in b.STATUS.items()} == {k: v for k, v in enum.items() if k.startswith("BT_OK") or
+                                                   k.startswith("BT_ERR_")}
+    assert (b.BT_F32, b.BT_BF16) == (enum["BT_F32"], enum["BT_BF16"])
+    assert b.MAX_CLOUDS == defines["BT_MAX_CLOUDS"]
+    assert b.BT_BUILD_NARROW == defines["BT_BUILD_NARROW"]
