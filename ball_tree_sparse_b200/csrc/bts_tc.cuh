@@ -216,7 +216,7 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
 
 // TMA gather: four rows (r0..r3) of a 2-D tensor map, `box width` elements from column col each, into
 // consecutive rows of shared memory (swizzled as the map says); completion is counted on `bar`.
-// Rows outside the tensor read as zeros.  Never with cluster multicast.
+// Rows outside the tensor read as zeros.  Each CTA loads its own tiles; no load is shared across a cluster.
 __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int32_t col, int32_t r0, int32_t r1,
                                             int32_t r2, int32_t r3, uint32_t bar)
 {
