@@ -45,6 +45,7 @@ _SIGS = {
     "bt_scatter": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
     "bt_ball_attention": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
     "bt_attention_device_status": ([_P], ctypes.c_int),
+    "bt_last_device_status": ([_P], ctypes.c_int),
     "bsa_workspace_size": ([_i64, _i64, _i32, _i32, _i32, _i32], _sz),
     "bsa_forward": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _i32, _P, _P, None, _P, _P,
                      _P, _sz, _P], ctypes.c_int),
@@ -304,6 +305,11 @@ def bt_coarse_ball_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, 
            _lib.bt_coarse_ball_attention(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, rows, m, H, d, _dt(Q),
                                          stride, _dptr(out), _dptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def bt_last_device_status(stream=None) -> int:
+    """First device-side error of the library's work on `stream` since the last call (synchronises it)."""
+    return int(_lib.bt_last_device_status(_stream(stream)))
 
 
 def bt_attention_device_status(stream=None) -> int:

@@ -47,7 +47,7 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return
 template <typename T, int D>
 __global__ void k_ball_attn_simt(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
                                  const int32_t *__restrict__ perm, int64_t rows, int m, int H, float scale,
-                                 T *__restrict__ O)
+                                 T *__restrict__ O, uint32_t *status)
 {
     extern __shared__ __align__(16) float fsm[];
     float *sK = fsm, *sV = fsm + m * D;
@@ -57,7 +57,7 @@ __global__ void k_ball_attn_simt(const T *__restrict__ Q, const T *__restrict__ 
     for (int j = threadIdx.x; j < m; j += blockDim.x) {
         int32_t r = perm ? perm[b * m + j] : int32_t(b * m + j);
         if (r >= rows) {  // not a row of Q/K/V: never read or write it
-            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            record_error(status, BT_ERR_INTERNAL);
             r = -1;
         }
         sRow[j] = r;
@@ -144,7 +144,7 @@ template <int D>
 __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
     k_ball_attn_tc2(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
                     const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ perm, int64_t npad,
-                    int64_t rows, int lm, int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O)
+                    int64_t rows, int lm, int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O, uint32_t *status)
 {
     using L = TcPipe<D>;
     constexpr int KCH = D / 8;                 // 16-byte chunks per row of one head
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
         if (!perm) return int32_t(slot);
         const int32_t row = __ldg(perm + slot);
         if (row >= rows) {  // not a row of Q/K/V: never read or write it
-            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            record_error(status, BT_ERR_INTERNAL);
             return -1;
         }
         return row;
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
                          kk > 0);
             mma_commit(barS);
         }
-        ok = ok && mbar_wait(barS, it & 1);
+        ok = ok && mbar_wait(barS, it & 1, status);
         tc_fence_after();
 
         // softmax of row tid; keys outside its ball or dummy get weight 0
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
             }
             mma_commit(barO);
         }
-        ok = ok && mbar_wait(barO, it & 1);
+        ok = ok && mbar_wait(barO, it & 1, status);
         tc_fence_after();
         if (ok) {
             uint32_t sum_bits;
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     k_ball_attn_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ perm, int64_t npad,
                      int64_t rows, int lm, int H, float sl2, int64_t items, __nv_bfloat16 *__restrict__ O,
-                     uint32_t *ctr)
+                     uint32_t *ctr, uint32_t *status)
 {
     using L = PairPipe;
     constexpr int NS = L::NS;
@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     };
     auto check = [&](int32_t row) -> int32_t {
         if (row >= rows) {  // not a row of Q/K/V: never read or write it
-            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            record_error(status, BT_ERR_INTERNAL);
             return -1;
         }
         return row;
@@ -478,6 +478,10 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         // The next item is claimed, and its perm rows requested, right after the current item's gathers.
         const int pw = warp - 8, g = 16 * pw + lane;
         bool pok = true;
+        // the item after `cur`: the launch's next unclaimed item, or without counters a fixed stride of the grid
+        auto claim = [&](int64_t cur) -> int64_t {
+            return ctr ? int64_t(gridDim.x) + int64_t(atomicAdd(ctr, 1u)) : cur + int64_t(gridDim.x);
+        };
         int64_t item = blockIdx.x;
         int32_t crow[4];
 #pragma unroll
@@ -492,7 +496,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                 if (lane == 0) sLive[pw] = bw != 0u;
                 asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");
                 const bool dead = !sLive[0] && !sLive[1];
-                if (dead && tid == 8 * 32) sClaim = pok ? int64_t(gridDim.x) + int64_t(atomicAdd(ctr, 1u)) : items;
+                if (dead && tid == 8 * 32) sClaim = pok ? claim(item) : items;
                 asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");  // sLive read; sClaim written
                 if (!dead) return;
                 item = sClaim;
@@ -504,7 +508,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         for (int it = 0;; ++it) {
             const int stage = it & (NS - 1);
             const uint32_t bar = smem_u32(&sFull[stage]);
-            if (it >= NS) pok = mbar_wait(smem_u32(&sEmpty[stage]), ((it / NS) + 1) & 1) && pok;
+            if (it >= NS) pok = mbar_wait(smem_u32(&sEmpty[stage]), ((it / NS) + 1) & 1, status) && pok;
             if (item >= items) {  // no more work: tell the consumers through the free stage
                 if (tid == 8 * 32) {
                     sItem[stage] = -1;
@@ -532,7 +536,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
             }
             // claim the next item after the gathers are on their way (a producer whose wait ran out hands out
             // no further work); its perm rows load while the next stage frees up
-            if (tid == 8 * 32) sClaim = pok ? int64_t(gridDim.x) + int64_t(atomicAdd(ctr, 1u)) : items;
+            if (tid == 8 * 32) sClaim = pok ? claim(item) : items;
             asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");
             item = sClaim;
 #pragma unroll
@@ -553,7 +557,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         // Waits for stage `st` of round `it`, publishes this warp's key mask, and reads the stage's item and
         // this thread's query row after the warpgroup barrier (so every thread takes the same decision).
         auto head = [&](int itn, int st, int32_t &q, int64_t &itm) -> bool {
-            ok = ok && mbar_wait(smem_u32(&sFull[st]), (itn / NS) & 1);
+            ok = ok && mbar_wait(smem_u32(&sFull[st]), (itn / NS) & 1, status);
             if (!ok) sAbort[hj] = 1;
             q = sRows[st][r];  // -1: dummy slot
             const uint32_t kb = __ballot_sync(0xffffffffu, q >= 0);
@@ -579,7 +583,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         for (int it = 0; go; ++it) {
             const int stage = it & (NS - 1);
             const uint32_t sv = base + stage * L::STAGE + 2 * L::TILE;
-            ok = ok && mbar_wait(barS, it & 1);
+            ok = ok && mbar_wait(barS, it & 1, status);
             tc_fence_after();
 
             // softmax of row r of head hj; keys outside its ball or dummy get weight 0
@@ -654,7 +658,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                 mma_commit(barO);
                 mma_commit(smem_u32(&sEmpty[stage]));  // this head is done with the stage
             }
-            ok = ok && mbar_wait(barO, it & 1);
+            ok = ok && mbar_wait(barO, it & 1, status);
             tc_fence_after();
             uint32_t o[32];
             tmem_ld32_nowait(tO + lanebase, o);
@@ -694,7 +698,7 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::COLS) : "memory");
     }
-    if (tid == 0) {
+    if (tid == 0 && ctr) {
         // the last CTA to finish resets the launch's counters for the next launch that uses them
         __threadfence();
         if (atomicAdd(ctr + 1, 1u) == gridDim.x - 1) {
@@ -737,11 +741,16 @@ static bool row_map(CUtensorMap *map, const void *base, int64_t rows, int hd, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Work counters of the head-pair kernel: launch k uses pair k mod kPairCounters ([0] items claimed so far,
-// [1] CTAs finished); the last CTA of a launch sets both back to zero.  Launches that run at the same time
-// therefore need distinct pairs: up to kPairCounters launches may be in flight together.
-constexpr int kPairCounters = 256;
-static __device__ uint32_t g_pair_ctr[kPairCounters][2];
+// Work counters of the head-pair kernel ([0] items claimed so far, [1] CTAs finished; the last CTA of a launch
+// sets both back to zero).  Launches that run at the same time need distinct pairs:
+//  - eager launches take pair k mod kEagerPairs (the k-th eager launch on the device), so up to kEagerPairs of
+//    them may be in flight together;
+//  - a launch captured into a CUDA graph keeps its pair for as long as the graph exists, so every captured
+//    launch gets a pair of its own from the next kCapturedPairs, never reused; once those are used up,
+//    captured launches run without counters, on a fixed schedule (item i of CTA c is c + i * grid).
+constexpr int kEagerPairs = 256;
+constexpr int kCapturedPairs = 4096;
+static __device__ uint32_t g_pair_ctr[kEagerPairs + kCapturedPairs][2];
 
 static bt_status launch_pair(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
                              int64_t rows, int lm, int H, void *O, cudaStream_t st)
@@ -749,7 +758,8 @@ static bt_status launch_pair(const void *Q, const void *K, const void *V, const 
     static std::atomic<bool> set[64] = {};
     static int sms[64] = {0};
     static uint32_t *ctrs[64] = {nullptr};
-    static std::atomic<uint32_t> next_pair{0};
+    static std::atomic<uint32_t> next_pair[64] = {};
+    static std::atomic<uint32_t> next_captured[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
     if (dev < 0 || dev >= 64) return BT_ERR_UNSUPPORTED;
@@ -767,7 +777,17 @@ static bt_status launch_pair(const void *Q, const void *K, const void *V, const 
         return BT_OK;
     });
     if (s0 != BT_OK) return s0;
-    uint32_t *ctr = ctrs[dev] + 2 * (next_pair.fetch_add(1u) % kPairCounters);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return BT_ERR_CUDA;
+    uint32_t *ctr = nullptr;
+    if (cs == cudaStreamCaptureStatusNone) {
+        ctr = ctrs[dev] + 2 * (next_pair[dev].fetch_add(1u) % kEagerPairs);
+    } else {
+        const uint32_t k = next_captured[dev].fetch_add(1u);
+        if (k < uint32_t(kCapturedPairs)) ctr = ctrs[dev] + 2 * (kEagerPairs + k);
+    }
+    uint32_t *status = stream_status(st);
+    if (!status) return BT_ERR_CUDA;
     CUtensorMap mq, mk, mv;
     if (!row_map(&mq, Q, rows, H * 32, 64) || !row_map(&mk, K, rows, H * 32, 64) || !row_map(&mv, V, rows, H * 32, 64))
         return BT_ERR_CUDA;
@@ -777,7 +797,7 @@ static bt_status launch_pair(const void *Q, const void *K, const void *V, const 
     const int64_t grid = items < int64_t(nsm) * PairPipe::PER_SM ? items : int64_t(nsm) * PairPipe::PER_SM;
     const float sl2 = 1.4426950408889634f / sqrtf(32.0f);
     k_ball_attn_pair<<<unsigned(grid), PairPipe::THREADS, PairPipe::BYTES, st>>>(
-        mq, mk, mv, perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O), ctr);
+        mq, mk, mv, perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O), ctr, status);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 
@@ -791,9 +811,11 @@ static bt_status launch_simt(const void *Q, const void *K, const void *V, const 
         return BT_ERR_CUDA;
     const int threads = ((m + 31) / 32) * 32;
     dim3 grid(unsigned(npad / m), unsigned(H));
+    uint32_t *status = stream_status(st);
+    if (!status) return BT_ERR_CUDA;
     k_ball_attn_simt<T, D><<<grid, threads, smem, st>>>(static_cast<const T *>(Q), static_cast<const T *>(K),
                                                         static_cast<const T *>(V), perm, rows, m, H,
-                                                        1.0f / sqrtf(float(D)), static_cast<T *>(O));
+                                                        1.0f / sqrtf(float(D)), static_cast<T *>(O), status);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 
@@ -821,9 +843,11 @@ static bt_status launch_tc(const void *Q, const void *K, const void *V, const in
     const int per_sm = TcPipe<D>::PER_SM;
     const int64_t grid = items < int64_t(nsm) * per_sm ? items : int64_t(nsm) * per_sm;
     const float sl2 = 1.4426950408889634f / sqrtf(float(D));
+    uint32_t *status = stream_status(st);
+    if (!status) return BT_ERR_CUDA;
     k_ball_attn_tc2<D><<<unsigned(grid), kTcThreads, smem, st>>>(
         static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(K),
-        static_cast<const __nv_bfloat16 *>(V), perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O));
+        static_cast<const __nv_bfloat16 *>(V), perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O), status);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 
@@ -858,17 +882,6 @@ extern "C" bt_status bt_ball_attention(const void *Q, const void *K, const void 
                        : launch_simt<__nv_bfloat16, 64>(Q, K, V, perm, npad, rows, m, H, O, st);
     return d == 32 ? launch_simt<float, 32>(Q, K, V, perm, npad, rows, m, H, O, st)
                    : launch_simt<float, 64>(Q, K, V, perm, npad, rows, m, H, O, st);
-}
-
-extern "C" bt_status bt_attention_device_status(void *stream)
-{
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint32_t h = 0, zero = 0;
-    if (cudaMemcpyFromSymbolAsync(&h, g_attn_status, sizeof(h), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return BT_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return BT_ERR_CUDA;
-    if (h && cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(zero)) != cudaSuccess) return BT_ERR_CUDA;
-    return static_cast<bt_status>(h);
 }
 
 #include "bts_coarse.cuh"

@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kMeanWarps * 32) k_bsa_means(const __nv_bfloat
                                                               float *__restrict__ kbar,
                                                               __nv_bfloat16 *__restrict__ kc,
                                                               __nv_bfloat16 *__restrict__ vc,
-                                                              int32_t *__restrict__ cnt)
+                                                              int32_t *__restrict__ cnt, uint32_t *status)
 {
     constexpr int M = 128;
     __shared__ int32_t srow[M];
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kMeanWarps * 32) k_bsa_means(const __nv_bfloat
     if (tid < M) {
         int32_t r = perm ? perm[b * M + tid] : int32_t(b * M + tid);
         if (r >= rows) {
-            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            record_error(status, BT_ERR_INTERNAL);
             r = -1;
         }
         srow[tid] = r;
@@ -381,7 +381,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                   int nb, const __nv_bfloat16 *__restrict__ kc, const __nv_bfloat16 *__restrict__ vc,
                   const int32_t *__restrict__ cnt, const int32_t *__restrict__ sel, int topk,
                   const float *__restrict__ gates, const __nv_bfloat16 *__restrict__ Oball, float sl2,
-                  __nv_bfloat16 *__restrict__ O)
+                  __nv_bfloat16 *__restrict__ O, uint32_t *status)
 {
     using L = BsaPipe<D>;
     constexpr int KCH = D / 8;
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
 
     auto valid_row = [&](int32_t r) -> int32_t {
         if (r >= rows) {
-            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            record_error(status, BT_ERR_INTERNAL);
             return -1;
         }
         return r;
@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                                  IDESC_S, kk > 0);
                     mma_commit(barS);
                 }
-                ok = ok && mbar_wait(barS, nS & 1);
+                ok = ok && mbar_wait(barS, nS & 1, status);
                 ++nS;
                 tc_fence_after();
                 uint32_t cmask[4];
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                         mma_bf16_ts(tO, tS + kk * 8, smem_desc(sv + kk * 256, 128, V_SBO), IDESC_O, kk > 0);
                     mma_commit(barO);
                 }
-                ok = ok && mbar_wait(barO, nO & 1);
+                ok = ok && mbar_wait(barO, nO & 1, status);
                 ++nO;
                 tc_fence_after();
                 if (ok) {
@@ -689,7 +689,7 @@ __global__ void __launch_bounds__(kCoarseWarps * 32) k_bsa_coarse(const __nv_bfl
                                                                   const int32_t *__restrict__ sel, int topk,
                                                                   const float *__restrict__ gates,
                                                                   const __nv_bfloat16 *__restrict__ Oball, float sl2,
-                                                                  __nv_bfloat16 *__restrict__ O)
+                                                                  __nv_bfloat16 *__restrict__ O, uint32_t *status)
 {
     constexpr int G = D / 8, KPS = 32 / G;  // lanes per key, keys per half-step
     constexpr int NW = kCoarseWarps;
@@ -766,7 +766,7 @@ __global__ void __launch_bounds__(kCoarseWarps * 32) k_bsa_coarse(const __nv_bfl
             const int s = sel[(size_t(g) * H + h) * topk + t];
             if (s < 0) continue;  // uniform across the warp
             if (s >= nb) {
-                record_error(&g_attn_status, BT_ERR_INTERNAL);
+                record_error(status, BT_ERR_INTERNAL);
                 continue;
             }
             for (int i0 = 0; i0 < RPL; i0 += 2 * BI) {
@@ -776,7 +776,7 @@ __global__ void __launch_bounds__(kCoarseWarps * 32) k_bsa_coarse(const __nv_bfl
                     const int64_t j = int64_t(s) * 128 + kslot + KPS * (i0 + u);
                     int32_t row = perm ? perm[j] : int32_t(j);
                     if (row >= rows) {
-                        record_error(&g_attn_status, BT_ERR_INTERNAL);
+                        record_error(status, BT_ERR_INTERNAL);
                         row = -1;
                     }
                     rw[u] = row;
@@ -832,7 +832,7 @@ __global__ void __launch_bounds__(kCoarseWarps * 32) k_bsa_coarse(const __nv_bfl
         const int r = it * NW * KPS + warp * KPS + kslot;
         int32_t qrow = perm ? perm[int64_t(g) * 128 + r] : int32_t(int64_t(g) * 128 + r);
         if (qrow >= rows) {
-            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            record_error(status, BT_ERR_INTERNAL);
             qrow = -1;
         }
         qr[it] = qrow;
@@ -934,7 +934,9 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
     const bt_status s0 = (dev >= 0 && dev < 64) ? setup_once(set[dev], init) : init();
     if (s0 != BT_OK) return s0;
     const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
-    k_bsa_means<<<nb, kMeanWarps * 32, 0, st>>>(q, k, v, perm, rows, H * D, qbar, kbar, kc, vc, cnt);
+    uint32_t *status = stream_status(st);
+    if (!status) return BT_ERR_CUDA;
+    k_bsa_means<<<nb, kMeanWarps * 32, 0, st>>>(q, k, v, perm, rows, H * D, qbar, kbar, kc, vc, cnt, status);
     k_bsa_gates<<<unsigned((rows + kGateRows - 1) / kGateRows), kGateThreads, gate_smem_bytes(C, H), st>>>(
         X, rows, C, Wg, bg, H, gate_out_padded(H), gates);
     if (p.topk > 0)
@@ -948,13 +950,13 @@ static bt_status bsa_launch(const void *Q, const void *K, const void *V, const i
     if (p.coarsen_queries) {
         k_bsa_coarse<D><<<unsigned(items), kCoarseWarps * 32, 0, st>>>(
             k, v, perm, rows, H, nb, qbar, kc, vc, cnt, sel, p.topk, gates, oball,
-            1.4426950408889634f / sqrtf(float(D)), static_cast<__nv_bfloat16 *>(O));
+            1.4426950408889634f / sqrtf(float(D)), static_cast<__nv_bfloat16 *>(O), status);
         return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
     }
     const int64_t grid = items < int64_t(nsm) * BsaPipe<D>::PER_SM ? items : int64_t(nsm) * BsaPipe<D>::PER_SM;
     k_bsa_attn_tc<D><<<unsigned(grid), kTcThreads, BsaPipe<D>::BYTES, st>>>(
         q, k, v, perm, rows, H, nb, kc, vc, cnt, sel, p.topk, gates, oball, 1.4426950408889634f / sqrtf(float(D)),
-        static_cast<__nv_bfloat16 *>(O));
+        static_cast<__nv_bfloat16 *>(O), status);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
 

@@ -47,6 +47,7 @@ constexpr int kCounterLevel0 = 8;
 struct Plan {
     int32_t B, m, T, TP, nlev, sort_tiles;
     int32_t rec;  // 1: record path (every cloud a power-of-two slot count of at most 2^21)
+    uint32_t *sstatus;  // status word of the call's stream: the build's last kernel folds the workspace word in
     int64_t npad;
     int64_t pad[BT_MAX_CLOUDS + 1];
     int64_t n[BT_MAX_CLOUDS];
@@ -853,6 +854,8 @@ __global__ void __launch_bounds__(NT) k_tail(Plan P, const uint32_t *__restrict_
         const int64_t li = int64_t(pid) - P.pad[b];
         perm[seg + e] = li < P.n[b] ? int32_t(P.row0[b] + li) : -1;
     }
+    __syncthreads();
+    if (threadIdx.x == 0) fold_status(status, P.sstatus);
 }
 
 // ---------------------------------------------------------------------------
@@ -1270,6 +1273,8 @@ __global__ void __launch_bounds__(kTailRThreads, EPT <= 4 ? 2 : 1) k_tail_r(Plan
         }
         perm[seg + e] = li < P.n[b] ? int32_t(P.row0[b] + li) : -1;
     }
+    __syncthreads();
+    if (threadIdx.x == 0) fold_status(status, P.sstatus);
 }
 
 // ---------------------------------------------------------------------------
@@ -1760,6 +1765,8 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
         perm[P.pad[b] + pos0 + i] = int(id) < n ? int32_t(P.row0[b] + id) : -1;
     }
     cluster_wait_acquire();
+    __syncthreads();
+    if (threadIdx.x == 0) fold_status(status, P.sstatus);
 }
 
 static size_t tail_smem_bytes(int T)
@@ -1864,9 +1871,12 @@ static int cluster_capacity(int dev, int NC, int CMAX)
     return ok ? nclusters : 0;
 }
 
-static bt_status launch_build(const float *coords, const Plan &P, int32_t *perm, void *ws, size_t ws_bytes,
+static bt_status launch_build(const float *coords, const Plan &P0, int32_t *perm, void *ws, size_t ws_bytes,
                               uint32_t flags, cudaStream_t st)
 {
+    Plan P = P0;
+    P.sstatus = stream_status(st);
+    if (!P.sstatus) return BT_ERR_CUDA;
     const Layout L = make_layout(P);
     if (!ws) return BT_ERR_WORKSPACE;
     if (ws_bytes < L.total) return BT_ERR_WORKSPACE;

@@ -61,7 +61,7 @@ __device__ __forceinline__ void store_f32(T *p, const float (&f)[EPU])
 template <typename T, int EPU>
 __global__ void __launch_bounds__(256) k_pool_mean(PoolTensors<T> a, const int32_t *__restrict__ perm,
                                                    int64_t ncoarse, int64_t rows, int units, int stride,
-                                                   int32_t *__restrict__ cperm)
+                                                   int32_t *__restrict__ cperm, uint32_t *status)
 {
     const int y = blockIdx.y;  // selected without a dynamic index into the parameter array
     const T *__restrict__ src = y == 0 ? a.src[0] : y == 1 ? a.src[1] : a.src[2];
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(256) k_pool_mean(PoolTensors<T> a, const int32
             const int64_t slot = j * stride + i;
             int64_t r = perm ? int64_t(perm[slot]) : slot;
             if (r >= rows) {
-                record_error(&g_attn_status, BT_ERR_INTERNAL);
+                record_error(status, BT_ERR_INTERNAL);
                 r = -1;
             }
             if (r < 0) continue;
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(256) k_pool_mean(PoolTensors<T> a, const int32
 template <typename U>
 __global__ void __launch_bounds__(256) k_unpool(const U *__restrict__ src, const int32_t *__restrict__ perm,
                                                 int64_t npad, int64_t rows, int units, int stride,
-                                                U *__restrict__ dst)
+                                                U *__restrict__ dst, uint32_t *status)
 {
     const int64_t total = npad * units;
     for (int64_t t = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; t < total; t += int64_t(gridDim.x) * blockDim.x) {
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(256) k_unpool(const U *__restrict__ src, const
         const int u = int(t - slot * units);
         const int64_t r = perm ? int64_t(perm[slot]) : slot;
         if (r >= rows) {
-            record_error(&g_attn_status, BT_ERR_INTERNAL);
+            record_error(status, BT_ERR_INTERNAL);
             continue;
         }
         if (r < 0) continue;
@@ -138,13 +138,15 @@ static bt_status launch_pool(PoolTensors<T> a, int nt, const int32_t *perm, int6
     const int64_t nc = npad / stride;
     if (nc == 0) return BT_OK;
     constexpr int VEC = 16 / sizeof(T);
+    uint32_t *status = stream_status(st);
+    if (!status) return BT_ERR_CUDA;
     uintptr_t al = 0;
     for (int i = 0; i < nt; ++i) al |= reinterpret_cast<uintptr_t>(a.src[i]) | reinterpret_cast<uintptr_t>(a.dst[i]);
     if (C % VEC == 0 && al % 16 == 0) {
         const int units = C / VEC;
-        k_pool_mean<T, VEC><<<dim3(stream_grid(nc * units), nt), 256, 0, st>>>(a, perm, nc, rows, units, stride, cperm);
+        k_pool_mean<T, VEC><<<dim3(stream_grid(nc * units), nt), 256, 0, st>>>(a, perm, nc, rows, units, stride, cperm, status);
     } else {
-        k_pool_mean<T, 1><<<dim3(stream_grid(nc * C), nt), 256, 0, st>>>(a, perm, nc, rows, C, stride, cperm);
+        k_pool_mean<T, 1><<<dim3(stream_grid(nc * C), nt), 256, 0, st>>>(a, perm, nc, rows, C, stride, cperm, status);
     }
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
@@ -180,18 +182,20 @@ extern "C" bt_status bt_unpool(const void *Xc, const int32_t *perm, int64_t npad
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t row_bytes = int64_t(C) * (dt == BT_F32 ? 4 : 2);
     const uintptr_t al = reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Xc);
+    uint32_t *status = stream_status(st);
+    if (!status) return BT_ERR_CUDA;
     if (row_bytes % 16 == 0 && al % 16 == 0) {
         const int units = int(row_bytes / 16);
         k_unpool<uint4><<<stream_grid(npad * units), 256, 0, st>>>(static_cast<const uint4 *>(Xc), perm, npad, rows,
-                                                                    units, stride, static_cast<uint4 *>(X));
+                                                                    units, stride, static_cast<uint4 *>(X), status);
     } else if (row_bytes % 4 == 0 && al % 4 == 0) {
         const int units = int(row_bytes / 4);
         k_unpool<uint32_t><<<stream_grid(npad * units), 256, 0, st>>>(static_cast<const uint32_t *>(Xc), perm, npad,
-                                                                       rows, units, stride, static_cast<uint32_t *>(X));
+                                                                       rows, units, stride, static_cast<uint32_t *>(X), status);
     } else {
         const int units = int(row_bytes / 2);
         k_unpool<uint16_t><<<stream_grid(npad * units), 256, 0, st>>>(static_cast<const uint16_t *>(Xc), perm, npad,
-                                                                       rows, units, stride, static_cast<uint16_t *>(X));
+                                                                       rows, units, stride, static_cast<uint16_t *>(X), status);
     }
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }

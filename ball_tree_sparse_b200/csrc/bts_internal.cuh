@@ -40,6 +40,20 @@ __device__ __forceinline__ void record_error(uint32_t *status, uint32_t code)
     if (ld_relaxed(status) == 0u) atomicCAS(status, 0u, code);  // read first: no atomic storm once set
 }
 
+// Device address of the status word of stream `st` on the current device (assigned on the stream's first use;
+// nullptr if the CUDA runtime refused the look-up).  Kernels record into it with record_error().
+uint32_t *stream_status(cudaStream_t st);
+
+// Copies a build workspace's status word into the stream's word (first error wins); called by one thread of
+// every CTA of a build's last kernel, after that CTA's own work, so every error of the build reaches it.
+__device__ __forceinline__ void fold_status(uint32_t *ws_status, uint32_t *stream_word)
+{
+    if (!stream_word) return;
+    __threadfence();
+    const uint32_t v = ld_relaxed(ws_status);
+    if (v) record_error(stream_word, v);
+}
+
 __device__ __forceinline__ void st_relaxed(uint32_t *p, uint32_t v)
 {
     asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");

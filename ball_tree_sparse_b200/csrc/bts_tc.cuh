@@ -9,10 +9,6 @@
 
 namespace bts {
 
-// Device-side status of the attention kernels.  This header is included by
-// exactly one translation unit (bts_attn.cu), which owns the variable.
-__device__ uint32_t g_attn_status;
-
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -61,12 +57,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase; false (and an error recorded) if it never completes.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+// Bounded wait on an mbarrier phase; false (and BT_ERR_TIMEOUT recorded in `status`) if it never completes.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status)
 {
     for (int i = 0; i < (1 << 18); ++i)
         if (mbar_try_wait(bar, parity)) return true;
-    record_error(&g_attn_status, BT_ERR_TIMEOUT);
+    record_error(status, BT_ERR_TIMEOUT);
     return false;
 }
 

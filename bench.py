@@ -85,12 +85,19 @@ def parse():
     p.add_argument("--no-suite", action="store_true", help="skip the other workloads")
     p.add_argument("--suite-steps", type=int, default=20)
     p.add_argument("--suite-only", default="",
-                   help="comma-separated suite workloads to time on their own (tiny, ellipsoid_bsa, box_cluster, "
-                        "gauss_mix_coarse_levels, ragged); skips the headline step")
+                   help="comma-separated suite workloads to time on their own (tiny, ellipsoid, ellipsoid_bsa, rows, "
+                        "box_cluster, gauss_mix_coarse_levels, ragged); skips the headline step")
     return p.parse_args()
 
 
 # ---------------------------------------------------------------------------
+def headline_config(world: int) -> dict:
+    """The `config` of the headline line; the reference arm prints the same one."""
+    return {"workload": "gauss_mix 4x16384 (m=128, H=8, d=32), layers: original + rotated tree",
+            "global_batch": 4 * world, "seq_len": 16384, "parallelism": f"replicas{world}",
+            "l2": "256 MB write between timed steps", "graph": "one CUDA graph per step"}
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -110,7 +117,11 @@ def _tensor_peak():
 
 
 class ClockSampler:
-    """nvidia-smi samples (SM clock, throttle reasons) while the timed region runs."""
+    """nvidia-smi samples (SM clock, throttle reasons), started when the process starts and stopped after the
+    timed region, so that the timed region is inside the sampled span.  A timed region shorter than the sampling
+    period may hold no sample of its own: the summary then takes the samples within one period of it."""
+
+    PERIOD_MS = 20
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -126,8 +137,8 @@ class ClockSampler:
             sel = []
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "100", *sel], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
+                                          "-lms", str(self.PERIOD_MS), *sel], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except Exception:
@@ -137,6 +148,13 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def wait_first(self, timeout_s: float = 10.0) -> bool:
+        """Block until nvidia-smi has printed its first row (or gave up)."""
+        t_end = time.time() + timeout_s
+        while self.proc is not None and not self.rows and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
+        return bool(self.rows)
 
     def mark(self):
         self.marks.append(time.time())
@@ -151,15 +169,21 @@ class ClockSampler:
 
     def summary(self):
         t0, t1 = (self.marks + [0, 0])[:2] if len(self.marks) >= 2 else (0, 1e30)
-        rows = [r for t, r in self.rows if t0 <= t <= t1] or [r for _, r in self.rows]
+        rows = [r for t, r in self.rows if t0 <= t <= t1]
+        window = "timed region"
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+            pad = self.PERIOD_MS / 1e3
+            rows = [r for t, r in self.rows if t0 - pad <= t <= t1 + pad]
+            window = f"timed region +- {self.PERIOD_MS} ms (shorter than the sampling period)"
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0,
+                    "samples_total": len(self.rows)}
         sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
         mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 3 + i and r[3 + i] == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "window": window, "samples_total": len(self.rows)}
 
 
 def _cudart():
@@ -433,8 +457,7 @@ def run_reference(args, wl):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "gauss_mix 4x16384 (m=128, H=8, d=32), layers: original + rotated tree",
-                       "global_batch": 4, "seq_len": 16384, "parallelism": "replicas"},
+            "config": headline_config(args.gpus),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -479,8 +502,12 @@ def suite(bts, dev, steps, flush, peak, only=None):
         return only is None or name in only
     if want("tiny"):
         _suite_tiny(bts, dev, steps, flush, res)
+    if want("ellipsoid"):
+        _suite_ellipsoid_layer(bts, dev, steps, flush, peak, res)
     if want("ellipsoid_bsa"):
         _suite_ellipsoid(bts, dev, steps, flush, res)
+    if want("rows"):
+        _suite_rows(bts, dev, steps, flush, peak, res)
     if want("box_cluster"):
         _suite_box(bts, dev, steps, flush, peak, res)
     if want("gauss_mix_coarse_levels"):
@@ -506,6 +533,59 @@ def _suite_tiny(bts, dev, steps, flush, res):
     ms = statistics.mean(timed_graph(tiny_step, steps, 3, flush))
     res["tiny"] = {"points": wl.n_total, "layers": 1, "dtype": "f32", "ms_per_step": ms,
                    "points_per_s_per_layer": wl.n_total / (ms / 1e3)}
+
+
+def _suite_ellipsoid_layer(bts, dev, steps, flush, peak, res):
+    # the single 65,536-point ellipsoid cloud: one layer = tree build (9 levels, multi-launch path) + plain ball
+    # attention, the layer the metric is quoted on, on one tree of 65,536 points
+    wl = workloads.ellipsoid()
+    L = wl.layers[0]
+    c = torch.from_numpy(wl.coords).to(dev)
+    q, k, v = (_bf16_dev(t, dev) for t in (L.q, L.k, L.v))
+    perm = torch.empty(wl.n_total, dtype=torch.int32, device=dev)
+    ws = bts.workspace([0, wl.n_total], wl.m, dev)
+    out = torch.empty_like(q)
+
+    def layer():
+        bts.bt_build(c, wl.m, perm=perm, ws=ws)
+        bts.bt_ball_attention(q, k, v, perm, wl.m, out=out)
+    ms = statistics.mean(timed_graph(layer, steps, 3, flush))
+    b_ms = statistics.mean(timed_graph(lambda: bts.bt_build(c, wl.m, perm=perm, ws=ws), steps, 3, flush))
+    a_ms = statistics.mean(timed_graph(lambda: bts.bt_ball_attention(q, k, v, perm, wl.m, out=out), steps, 3, flush))
+    nbytes = 4 * wl.n_total * wl.H * wl.d * 2 + 4 * wl.n_total
+    res["ellipsoid"] = {"points": wl.n_total, "layers": 1, "ms_per_step": ms,
+                        "points_per_s_per_layer": wl.n_total / (ms / 1e3), "build_ms": b_ms, "attention_ms": a_ms,
+                        "attention_gbs": nbytes / (a_ms / 1e3) / 1e9,
+                        "attention_frac_of_measured_hbm": nbytes / (a_ms / 1e3) / 1e9 / peak}
+    del q, k, v, out
+
+
+def _suite_rows(bts, dev, steps, flush, peak, res):
+    # standalone row gather into tree order and scatter back (bt_gather / bt_scatter) of one Q-sized tensor, on
+    # the gauss_mix batch (512-byte rows, with padding slots) and on box_cluster (256-byte rows); algorithmic
+    # bytes per slot: the row read, the row written and the 4-byte index
+    entry = {}
+    for name, wl in (("gauss_mix", workloads.gauss_mix()), ("box_cluster", workloads.box_cluster(with_qkv=False))):
+        c = torch.from_numpy(wl.coords).to(dev)
+        npad = int(wl.pad_offsets()[-1])
+        perm = torch.empty(npad, dtype=torch.int32, device=dev)
+        bts.bt_build_segmented(c, wl.offsets, wl.m, perm=perm)
+        x = torch.randn((wl.n_total, wl.H, wl.d), device=dev).to(torch.bfloat16)
+        y = torch.empty((npad, wl.H, wl.d), dtype=torch.bfloat16, device=dev)
+        x2 = torch.empty_like(x)
+        row = wl.H * wl.d * 2
+        g_ms = statistics.mean(timed_graph(lambda: bts.bt_gather(x, perm, out=y), steps, 3, flush))
+        s_ms = statistics.mean(timed_graph(lambda: bts.bt_scatter(y, perm, x2), steps, 3, flush))
+        real = wl.n_total
+        g_bytes = real * 2 * row + (npad - real) * row + 4 * npad  # dummy slots write a zero row
+        s_bytes = real * 2 * row + 4 * npad
+        entry[name] = {"slots": npad, "row_bytes": row, "gather_ms": g_ms,
+                       "gather_gbs": g_bytes / (g_ms / 1e3) / 1e9,
+                       "gather_frac_of_measured_hbm": g_bytes / (g_ms / 1e3) / 1e9 / peak,
+                       "scatter_ms": s_ms, "scatter_gbs": s_bytes / (s_ms / 1e3) / 1e9,
+                       "scatter_frac_of_measured_hbm": s_bytes / (s_ms / 1e3) / 1e9 / peak}
+        del x, y, x2, perm, c
+    res["rows"] = entry
 
 
 def _suite_ellipsoid(bts, dev, steps, flush, res):
@@ -642,11 +722,14 @@ def main():
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    clocks = ClockSampler(local)  # running from here to the end of the timed region
+    clocks.wait_first()
     if args.suite_only:
         # the named suite workloads alone (for profiling one of them); no headline line
         names = {x.strip() for x in args.suite_only.split(",") if x.strip()}
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
         res = suite(bts, dev, args.suite_steps, flush, _peaks()[0], only=names)
+        clocks.stop()
         if rank == 0:
             print(json.dumps({"suite_only": sorted(names), "workloads": res}))
         if dist is not None:
@@ -657,7 +740,6 @@ def main():
     st.capture()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    clocks = ClockSampler(local)
     for _ in range(args.warmup):
         flush.zero_()
         st.graph.replay()
@@ -730,9 +812,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "gauss_mix 4x16384 (m=128, H=8, d=32), layers: original + rotated tree",
-                   "global_batch": 4 * world, "seq_len": 16384, "parallelism": f"replicas{world}",
-                   "l2": "256 MB write between timed steps", "graph": "one CUDA graph per step"},
+        "config": headline_config(world),
         "roofline": {"bound": "hbm", "kernel": ROOF_KERNEL, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
                      "bytes_per_launch": attn_bytes, "avg_launch_ms": attn_avg_ms,

@@ -29,9 +29,14 @@
  *    The library allocates nothing; scratch comes from a caller workspace.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  Argument errors are returned before anything is
- *    enqueued.  Errors found on the device (non-finite coordinates, an
- *    inter-block wait that ran out) are recorded in the workspace and read
- *    back by bt_build_device_status().  No call traps, aborts or prints.
+ *    enqueued.  Errors found on the device (non-finite coordinates, a perm
+ *    entry outside the tensors, an inter-block wait that ran out) are
+ *    recorded, first error wins, in a status word of the stream the call was
+ *    enqueued on, and read back (and cleared) by bt_last_device_status(stream).
+ *    Builds also keep theirs in the workspace (bt_build_device_status).  Work
+ *    captured into a CUDA graph records into the word of the stream it was
+ *    captured on, wherever the graph is later launched.  No call traps, aborts
+ *    or prints.
  *  - Arrays are row-major and contiguous.  Coordinates are float [rows, 3].
  *    Q/K/V/O are [rows, H, d] (H heads of d values per row).
  *  - Calls may come from several host threads: the per-device set-up on a
@@ -148,6 +153,18 @@ bt_status bt_build_noalloc(const float *coords, int64_t N, int32_t m, int32_t *p
                            void *stream);
 
 /*
+ * First device-side error recorded by the library's work enqueued on `stream`
+ * since the previous call for that stream (every call of this header that
+ * launches kernels): synchronises `stream`, then takes and clears the
+ * stream's status word in one atomic step.  Returns BT_OK, BT_ERR_NONFINITE,
+ * BT_ERR_TIMEOUT or BT_ERR_INTERNAL (or BT_ERR_CUDA).  Streams keep separate
+ * words, so a caller neither sees nor clears another stream's errors (the
+ * library holds 1,023 such words per device; streams beyond them share one).
+ * Not for use while `stream` is being captured.
+ */
+bt_status bt_last_device_status(void *stream);
+
+/*
  * Device-side status of the last build that used `ws`: synchronises `stream`,
  * returns BT_OK, BT_ERR_NONFINITE, BT_ERR_TIMEOUT or BT_ERR_INTERNAL (or
  * BT_ERR_CUDA).
@@ -203,7 +220,7 @@ bt_status bt_scatter(const void *Y, const int32_t *idx, int64_t npad, int32_t ro
  *            npad, no dummies).  Gathering by perm and scattering O back is
  *            fused into the attention kernel.  An entry >= rows is never
  *            dereferenced: the slot is treated as a dummy and BT_ERR_INTERNAL
- *            is recorded for bt_attention_device_status().
+ *            is recorded for bt_last_device_status().
  *   npad     number of slots, a multiple of m
  *   rows     number of rows of Q, K, V and O
  *   m        1 <= m <= 256;  H >= 1;  d in {32, 64}
@@ -211,6 +228,15 @@ bt_status bt_scatter(const void *Y, const int32_t *idx, int64_t npad, int32_t ro
  *            names are left untouched
  * Accumulation and softmax are in float.  BT_BF16 with m dividing 128 runs on
  * the tcgen05 tensor cores; other shapes run on the CUDA cores.
+ * Concurrency: the bf16 kernel for d = 32 and even H hands out its work from a
+ * pair of device counters, which launches that run at the same time must not
+ * share.  Eager calls take pair k mod 256 (k-th eager call on the device), so
+ * at most 256 of them may be in flight together.  A call made while `stream`
+ * is being captured gets a pair of its own for the life of the process (4,096
+ * such pairs per device; later captured calls use a fixed schedule with no
+ * counters); two executable graphs instantiated from ONE captured graph share
+ * that pair and must not run at the same time (one executable graph replayed
+ * repeatedly is fine: CUDA orders its launches).
  */
 bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
                             int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream);
@@ -285,7 +311,7 @@ bt_status bsa_forward(const void *Q, const void *K, const void *V, const int32_t
  *   Xc     dt [npad/stride, C] device out, coarse slot order
  *   cperm  int32 [npad/stride] device out, or NULL
  * A perm entry >= rows is skipped and recorded as BT_ERR_INTERNAL in the
- * attention status word (bt_attention_device_status).
+ * stream's status word (bt_last_device_status).
  */
 bt_status bt_pool_mean(const void *X, const int32_t *perm, int64_t npad, int64_t rows, int32_t C, int32_t stride,
                        bt_dtype dt, void *Xc, int32_t *cperm, void *stream);
@@ -314,12 +340,7 @@ bt_status bt_coarse_ball_attention(const void *Q, const void *K, const void *V, 
                                    int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, int32_t stride, void *O,
                                    void *ws, size_t ws_bytes, void *stream);
 
-/*
- * Device-side status of the attention kernels on the current device:
- * synchronises `stream`, returns BT_OK, BT_ERR_TIMEOUT (a tensor-core
- * completion wait that gave up) or BT_ERR_INTERNAL (a perm entry >= rows),
- * and clears the recorded code.
- */
+/* Same as bt_last_device_status (the name of an earlier version of this library). */
 bt_status bt_attention_device_status(void *stream);
 
 #ifdef __cplusplus

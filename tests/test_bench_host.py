@@ -34,10 +34,24 @@ def test_clock_summary_without_samples():
     assert out["reasons"] == ["no nvidia-smi samples"]
 
 
-def test_clock_summary_falls_back_to_every_row_outside_the_window():
-    # rows that all lie outside the marks (a sampler that started late) are still summarised
+def test_clock_summary_takes_rows_within_one_period_of_a_short_window():
+    # a timed region shorter than the sampling period: rows within one period of it count, and say so
+    p = bench.ClockSampler.PERIOD_MS / 1e3
+    rows = [_row(1.0 - p / 2, 1960), _row(1.001 + p / 2, 1965), _row(5.0, 500)]
+    out = _sampler(rows, [1.0, 1.001]).summary()
+    assert out["samples"] == 2 and out["sm_mhz"] == 1962.5
+    assert out["window"].startswith("timed region +-")
+
+
+def test_clock_summary_ignores_rows_far_from_the_window():
+    # rows seconds away from the timed region say nothing about its clocks
     out = _sampler([_row(5.0, 1800), _row(6.0, 1900)], [0.0, 1.0]).summary()
-    assert out["samples"] == 2 and out["sm_mhz"] == 1850.0
+    assert out["samples"] == 0 and out["reasons"] == ["no nvidia-smi samples"]
+
+
+def test_reference_arm_prints_the_headline_config():
+    assert bench.headline_config(1)["parallelism"] == "replicas1"
+    assert bench.headline_config(2)["global_batch"] == 8
 
 
 def test_roofline_traffic_only_for_the_source_it_was_measured_on(monkeypatch):

@@ -1,8 +1,15 @@
 """GPU parity of ball attention against the float64 oracle.
 
 Tolerances (max-abs): 1e-4 for float32 inputs, 2e-2 for bfloat16 inputs and
-outputs (the bf16 path rounds P to bf16 and O to bf16; both errors are far
-below the bound at the RMS these inputs give).
+outputs.  The outputs' RMS is well below 1 (V ~ N(0,1) averaged over up to
+128 keys gives about 0.15), so every bf16 comparison also bounds
+max_abs / RMS(O_oracle) by REL_BF16 = 0.08.  Derivation: the bf16 path rounds
+each weight P to bf16 (relative error at most 2^-9) and each output to bf16
+(at most 2^-9 of |O|); with |V| at most about 4.5 inside a ball and |O| below
+1 that is at most 2^-9 * 4.5 + 2^-9 = 0.011 absolute, 0.077 of an RMS of
+0.143.  Measured: about 0.02 on a few thousand outputs, 0.05 at the tail of
+the 16.7 million outputs of the full 65,536-point layer.  The ratio of every
+comparison is printed.
 """
 import numpy as np
 import pytest
@@ -15,6 +22,7 @@ pytestmark = pytest.mark.gpu
 bts = pytest.importorskip("ball_tree_sparse_b200")
 
 TOL = {workloads.F32: 1e-4, workloads.BF16: 2e-2}
+REL_BF16 = 0.08
 
 
 def _dev(a):
@@ -37,7 +45,7 @@ def _compare(orc, q, k, v, m, perm, dtype, balls=None):
     Q, K, V = _qkv_dev(q, k, v, dtype)
     o = bts.bt_ball_attention(Q, K, V, None if perm is None else _dev(perm), m,
                               npad=None if perm is None else len(perm))
-    assert bts.bt_attention_device_status() == 0
+    assert bts.bt_last_device_status() == 0
     got = _out_np(o)
     want = orc.ball_attention(q, k, v, m, perm, balls=balls)
     if balls is not None:
@@ -45,9 +53,16 @@ def _compare(orc, q, k, v, m, perm, dtype, balls=None):
         rows = slots if perm is None else perm[slots]
         rows = rows[rows >= 0]
         got, want = got[rows], want[rows]
+    return _check(got, want, dtype)
+
+
+def _check(got, want, dtype):
     err = np.abs(got - want).max()
     rms = np.sqrt((want ** 2).mean())
+    print(f"parity: max_abs {err:.3e} rms {rms:.3e} max_abs/rms {err / rms:.3e}")
     assert err <= TOL[dtype], f"max abs err {err} (rms {rms})"
+    if dtype == workloads.BF16:
+        assert err / rms <= REL_BF16, f"max abs err {err} is {err / rms:.3f} of the output rms {rms}"
     return err, rms
 
 
@@ -154,3 +169,49 @@ def test_m1_is_v():
     Q, K, V = _qkv_dev(q, k, v, workloads.F32)
     o = bts.bt_ball_attention(Q, K, V, None, 1).cpu().numpy()
     assert np.array_equal(o, v)
+
+
+def test_ragged_full_size_sampled(orc):
+    """The full 8-cloud ragged batch: masked attention on sampled balls, the partly and fully dummy balls at the
+    end of every cloud among them, and rows named by no slot left untouched."""
+    wl = workloads.ragged()
+    L = wl.layers[0]
+    n = wl.n_total
+    perm_t, pad = bts.bt_build_segmented(_dev(wl.coords), wl.offsets, wl.m)
+    perm = perm_t.cpu().numpy()
+    sizes = np.diff(pad)
+    assert sizes.max() > 32768, "a cloud beyond the one-launch build's 32,768 slots"
+    # 64 extra rows that no slot names: the kernel must leave them as they are
+    extra = 64
+    q, k, v = workloads.random_qkv(n + extra, L.q.shape[1], L.q.shape[2], workloads.BF16, 4242)
+    q[:n], k[:n], v[:n] = L.q, L.k, L.v
+    Q, K, V = _qkv_dev(q, k, v, workloads.BF16)
+    out = torch.full_like(Q, 7.0)
+    bts.bt_ball_attention(Q, K, V, perm_t, wl.m, out=out)
+    assert bts.bt_last_device_status() == 0
+    got = _out_np(out)
+    assert np.all(got[n:] == 7.0)
+    nb = len(perm) // wl.m
+    real = (perm.reshape(nb, wl.m) >= 0).sum(1)
+    partial = np.nonzero((real > 0) & (real < wl.m))[0]
+    assert (real == 0).any() and partial.size >= 8  # every cloud's padding: some balls wholly dummy
+    rng = np.random.Generator(np.random.PCG64(5))
+    big = int(np.argmax(sizes))
+    big_balls = np.arange(pad[big] // wl.m, pad[big + 1] // wl.m)
+    balls = np.unique(np.concatenate([partial, rng.choice(big_balls, 24, replace=False),
+                                      rng.choice(np.nonzero(real == wl.m)[0], 40, replace=False)]))
+    want = orc.ball_attention(q, k, v, wl.m, perm, balls=balls)
+    slots = np.concatenate([np.arange(b * wl.m, (b + 1) * wl.m) for b in balls])
+    rows = perm[slots]
+    rows = rows[rows >= 0]
+    _check(got[rows], want[rows], workloads.BF16)
+    # a row is written exactly once: every real row's output is finite
+    assert np.isfinite(got[:n]).all()
+
+
+def test_ellipsoid_full_size(orc):
+    """The single 65,536-point ellipsoid cloud: plain ball attention over its tree, every output compared."""
+    wl = workloads.ellipsoid()
+    L = wl.layers[0]
+    perm = bts.bt_build(_dev(wl.coords), wl.m).cpu().numpy()
+    _compare(orc, L.q, L.k, L.v, wl.m, perm, workloads.BF16)

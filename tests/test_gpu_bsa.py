@@ -36,7 +36,7 @@ def _run_gpu(q, k, v, perm, x, w, b, topk, mask_own=True, coarsen=False):
     o = bts.bsa_forward(_bf(q), _bf(k), _bf(v), _dev(perm), 128, _dev(x), _dev(w),
                         None if b is None else _dev(b), topk=topk, mask_own_ball=mask_own, sel=sel,
                         coarsen_queries=coarsen)
-    assert bts.bt_attention_device_status() == 0
+    assert bts.bt_last_device_status() == 0
     return o.float().cpu().numpy().astype(np.float64), sel.cpu().numpy()[:, :, :topk]
 
 

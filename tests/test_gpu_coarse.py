@@ -53,7 +53,7 @@ def test_pool_mean_matches_oracle(orc, dtype, C, stride):
         xd, xo = _dev(x), x
     xc, cperm = bts.bt_pool_mean(xd, perm, stride)
     want, wperm = orc.pool_mean(xo, perm.cpu().numpy(), stride)
-    assert bts.bt_attention_device_status() == 0
+    assert bts.bt_last_device_status() == 0
     assert np.array_equal(cperm.cpu().numpy(), wperm)
     got = _host(xc)
     tol = 2.0 ** -8 if dtype == "bf16" else 1e-5
@@ -97,7 +97,7 @@ def test_coarse_ball_attention_matches_oracle(orc, sizes, leaf, m, stride, H, d,
     pts, perm = _tree(sizes, leaf, 30 + stride)
     (q, k, v), (qd, kd, vd) = _qkv(len(pts), H, d, dtype, stride + H)
     got = _host(bts.bt_coarse_ball_attention(qd, kd, vd, perm, m, stride))
-    assert bts.bt_attention_device_status() == 0
+    assert bts.bt_last_device_status() == 0
     want = orc.coarse_ball_attention(q, k, v, m, perm.cpu().numpy(), stride)
     err = np.abs(got - want).max()
     assert err <= (2e-2 if dtype == "bf16" else 1e-4), f"max abs err {err}"

@@ -76,8 +76,8 @@ def test_attention_perm_entry_out_of_range_is_recorded_not_read(orc):
     Q, K, V = (torch.from_numpy(t.view(np.int16)).cuda().view(torch.bfloat16) for t in (q, k, v))
     out = torch.full_like(Q, 7.0)
     bts.bt_ball_attention(Q, K, V, torch.from_numpy(perm).cuda(), m, out=out)
-    assert bts.bt_attention_device_status() == 8  # BT_ERR_INTERNAL, then cleared
-    assert bts.bt_attention_device_status() == 0
+    assert bts.bt_last_device_status() == 8  # BT_ERR_INTERNAL, then cleared
+    assert bts.bt_last_device_status() == 0
     got = out.float().cpu().numpy()
     assert np.all(got[5] == 7.0)  # the slot was treated as a dummy: row 5 is named by no valid slot
     ref_perm = perm.copy()

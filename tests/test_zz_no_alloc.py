@@ -29,7 +29,16 @@ def _noalloc_c(coords, m, perm, status):
 
 
 def test_noalloc_matches_workspace_build_twice():
-    cases = [(workloads.uniform_cloud(65536, 11), 128), (workloads.tied_cloud(32 * 2 ** 9, 12, levels=5), 32)]
+    # Calls in a row on the shared scratch, each checked bit-exact against bt_build:
+    #  - two multi-kernel (record-path) builds of 65,536 slots with different inputs and leaf sizes, so the
+    #    second runs on the counters, histograms and look-back words the first left behind;
+    #  - the index-list path (leaf size 96, not a power of two) after them;
+    #  - a one-launch cluster build (16,384 slots), then a multi-kernel build again.
+    cases = [(workloads.uniform_cloud(65536, 11), 128),
+             (workloads.tied_cloud(65536, 12, levels=5), 64),
+             (workloads.uniform_cloud(96 * 2 ** 9, 13, scale=(3.0, 1.0, 0.5)), 96),
+             (workloads.uniform_cloud(16384, 14), 128),
+             (workloads.tied_cloud(65536, 15, levels=9), 128)]
     for pts, m in cases:
         c = torch.from_numpy(pts).cuda()
         status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
@@ -38,7 +47,7 @@ def test_noalloc_matches_workspace_build_twice():
         want = bts.bt_build(c, m)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
-        assert torch.equal(perm, want)
+        assert torch.equal(perm, want), f"{len(pts)} points, m = {m}"
 
 
 def test_noalloc_rejects_too_many_points():
