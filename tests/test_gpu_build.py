@@ -140,7 +140,7 @@ def test_workload_box_cluster_full_size(orc):
 
 
 def test_workload_ragged_full_size(orc):
-    wl = workloads.ragged()
+    wl = workloads.ragged(with_qkv=False)
     got = _gpu_build(wl.coords, wl.m, wl.offsets)
     want, pad = orc.build(wl.coords, wl.m, wl.offsets)
     assert np.array_equal(got, want)

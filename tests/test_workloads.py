@@ -71,7 +71,7 @@ def test_box_cluster_mixture():
 
 
 def test_ragged_sizes_and_padding():
-    wl = workloads.ragged()
+    wl = workloads.ragged(with_qkv=False)
     sizes = np.diff(wl.offsets)
     assert len(sizes) == 8 and sizes.min() >= 10_000 and sizes.max() < 200_000
     pad = np.diff(wl.pad_offsets())

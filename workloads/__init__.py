@@ -178,7 +178,7 @@ def box_cluster(n: int = 1 << 20, m: int = 128, H: int = 4, d: int = 32, with_qk
 
 
 def ragged(batch: int = 8, n_min: int = 10_000, n_max: int = 200_000, m: int = 128, H: int = 8,
-           d: int = 32) -> Workload:
+           d: int = 32, with_qkv: bool = True) -> Workload:
     """Batch of clouds with log-uniform sizes, Gaussian-mixture coordinates as in gauss_mix.
     Each cloud is padded to m * 2^k slots by dummy points (masked in attention)."""
     wid = 5
@@ -189,8 +189,9 @@ def ragged(batch: int = 8, n_min: int = 10_000, n_max: int = 200_000, m: int = 1
     offsets = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
     n = int(offsets[-1])
     wl = Workload("ragged", coords, offsets, m, H, d, BF16)
-    q, k, v = _qkv(wid, 0, n, H, d, BF16)
-    wl.layers.append(Layer(q, k, v, rotated=False))
+    if with_qkv:
+        q, k, v = _qkv(wid, 0, n, H, d, BF16)
+        wl.layers.append(Layer(q, k, v, rotated=False))
     return wl
 
 
