@@ -44,6 +44,11 @@ _SIGS = {
     "bt_gather": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
     "bt_scatter": ([_P, _P, _i64, _i32, _P, _P], ctypes.c_int),
     "bt_ball_attention": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
+    "bt_qkv_project": ([_P, _i64, _i32, _P, _i32, _i32, ctypes.c_int, _P, _P, _i64, _P, _P, _P, _P], ctypes.c_int),
+    "bt_ball_attention_tree": ([_P, _P, _P, _P, _i64, _i64, _i32, _i32, _i32, ctypes.c_int, _P, _P], ctypes.c_int),
+    "bt_projected_workspace_size": ([_i64, _i64, _i32, _i32, ctypes.c_int], _sz),
+    "bt_projected_ball_attention": ([_P, _P, _i64, _i64, _i32, _P, _i32, _i32, _i32, ctypes.c_int, _P, _P, _sz, _P],
+                                    ctypes.c_int),
     "bt_attention_device_status": ([_P], ctypes.c_int),
     "bt_last_device_status": ([_P], ctypes.c_int),
     "bsa_workspace_size": ([_i64, _i64, _i32, _i32, _i32, _i32], _sz),
@@ -304,6 +309,60 @@ def bt_coarse_ball_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, 
     _check("bt_coarse_ball_attention",
            _lib.bt_coarse_ball_attention(_dptr(Q), _dptr(K), _dptr(V), _dptr(perm), npad, rows, m, H, d, _dt(Q),
                                          stride, _dptr(out), _dptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def bt_qkv_project(X: torch.Tensor, Wt: torch.Tensor, H: int, d: int, perm: torch.Tensor | None = None,
+                   inv: torch.Tensor | None = None, out=None, stream=None):
+    """Q, K, V = X Wt^T.  X [rows, C] original order; Wt [3*H*d, C].  With perm (slot -> row) the outputs are
+    [npad, H, d] in slot order (row r at slot inv[r]; zeros for dummy slots) and inv is computed when not given;
+    without, [rows, H, d] in the original order."""
+    rows, C = X.shape
+    npad = perm.numel() if perm is not None else rows
+    if perm is not None and inv is None:
+        inv = bt_invert_perm(perm, rows, stream=stream)
+    if out is None:
+        out = tuple(torch.empty((npad, H, d), dtype=X.dtype, device=X.device) for _ in range(3))
+    Q, K, V = out
+    _check("bt_qkv_project", _lib.bt_qkv_project(_dptr(X), rows, C, _dptr(Wt), H, d, _dt(X), _dptr(perm), _dptr(inv),
+                                                 npad, _dptr(Q), _dptr(K), _dptr(V), _stream(stream)))
+    return Q, K, V
+
+
+def bt_ball_attention_tree(Qt: torch.Tensor, Kt: torch.Tensor, Vt: torch.Tensor, perm: torch.Tensor, m: int,
+                           rows: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Ball attention of slot-ordered Q/K/V [npad, H, d]; O [rows, H, d] in the original order."""
+    npad, H, d = Qt.shape
+    if out is None:
+        out = torch.empty((rows, H, d), dtype=Qt.dtype, device=Qt.device)
+    _check("bt_ball_attention_tree",
+           _lib.bt_ball_attention_tree(_dptr(Qt), _dptr(Kt), _dptr(Vt), _dptr(perm), npad, rows, m, H, d, _dt(Qt),
+                                       _dptr(out), _stream(stream)))
+    return out
+
+
+def bt_projected_workspace_size(npad: int, rows: int, H: int, d: int, dtype: torch.dtype) -> int:
+    return int(_lib.bt_projected_workspace_size(npad, rows, H, d, BT_F32 if dtype == torch.float32 else BT_BF16))
+
+
+def bt_projected_ball_attention(X: torch.Tensor, perm: torch.Tensor | None, Wt: torch.Tensor, m: int, H: int, d: int,
+                                out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                                npad: int | None = None, stream=None) -> torch.Tensor:
+    """One attention layer from the features: Q/K/V = X Wt^T (in slot order where the tile kernel takes the shape),
+    then ball attention.  X [rows, C]; Wt [3*H*d, C]; returns O [rows, H, d] in the original order."""
+    rows, C = X.shape
+    if npad is None:
+        npad = perm.numel() if perm is not None else rows
+    if out is None:
+        out = torch.empty((rows, H, d), dtype=X.dtype, device=X.device)
+    if ws is None:
+        n = bt_projected_workspace_size(npad, rows, H, d, X.dtype)
+        if n == 0:
+            raise BtsError("bt_projected_workspace_size", 1)
+        ws = torch.empty(n, dtype=torch.uint8, device=X.device)
+    _check("bt_projected_ball_attention",
+           _lib.bt_projected_ball_attention(_dptr(X), _dptr(perm), npad, rows, C, _dptr(Wt), m, H, d, _dt(X),
+                                            _dptr(out), _dptr(ws), ws.numel(), _stream(stream)))
     return out
 
 

@@ -404,6 +404,7 @@ __device__ __forceinline__ void head_sync(int hj)
 // free stage, so the gathers' issue cost is off the compute path.  Stage s is full when its transaction
 // count completes (sFull[s]) and free again when both heads' MMAs that read it have completed (sEmpty[s],
 // two arrivals, each armed by tcgen05.commit after that head's P V product).
+template <bool TREE>
 __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
     k_ball_attn_pair(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const int32_t *__restrict__ perm, int64_t npad,
@@ -529,10 +530,21 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
             asm volatile("bar.sync 3, %0;" ::"n"(L::PRODUCERS) : "memory");  // armed before any gather lands
             if (lane < 16) {
                 const int32_t col = int32_t(uint32_t(item) % uint32_t(HP)) * 2 * D;
-                const uint32_t dq = base + stage * L::STAGE + g * 4 * L::RB;
-                tma_gather4(dq, &tmQ, col, rr[0], rr[1], rr[2], rr[3], bar);
-                tma_gather4(dq + L::TILE, &tmK, col, rr[0], rr[1], rr[2], rr[3], bar);
-                tma_gather4(dq + 2 * L::TILE, &tmV, col, rr[0], rr[1], rr[2], rr[3], bar);
+                if constexpr (TREE) {
+                    // Q/K/V already in slot order: the item's rows are one 128 x 64 tile of each tensor
+                    if (g == 0) {
+                        const int32_t y = int32_t(uint32_t(item) / uint32_t(HP)) * 128;
+                        const uint32_t dq = base + stage * L::STAGE;
+                        tma_load_2d(dq, &tmQ, col, y, bar);
+                        tma_load_2d(dq + L::TILE, &tmK, col, y, bar);
+                        tma_load_2d(dq + 2 * L::TILE, &tmV, col, y, bar);
+                    }
+                } else {
+                    const uint32_t dq = base + stage * L::STAGE + g * 4 * L::RB;
+                    tma_gather4(dq, &tmQ, col, rr[0], rr[1], rr[2], rr[3], bar);
+                    tma_gather4(dq + L::TILE, &tmK, col, rr[0], rr[1], rr[2], rr[3], bar);
+                    tma_gather4(dq + 2 * L::TILE, &tmV, col, rr[0], rr[1], rr[2], rr[3], bar);
+                }
             }
             // claim the next item after the gathers are on their way (a producer whose wait ran out hands out
             // no further work); its perm rows load while the next stage frees up
@@ -741,6 +753,20 @@ static bool row_map(CUtensorMap *map, const void *base, int64_t rows, int hd, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A [rows, cols] bf16 matrix viewed in box_rows x box_cols tiles, 128-byte swizzled (whole-tile loads).
+static bool tile_map(CUtensorMap *map, const void *base, int64_t rows, int cols, int box_cols, int box_rows)
+{
+    const EncodeTiledFn fn = encode_tiled();
+    if (!fn || rows < 1 || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(cols) * 2};
+    const cuuint32_t bx[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+    const cuuint32_t es[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, bx, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Work counters of the head-pair kernel ([0] items claimed so far, [1] CTAs finished; the last CTA of a launch
 // sets both back to zero).  Launches that run at the same time need distinct pairs:
 //  - eager launches take pair k mod kEagerPairs (the k-th eager launch on the device), so up to kEagerPairs of
@@ -752,8 +778,10 @@ constexpr int kEagerPairs = 256;
 constexpr int kCapturedPairs = 4096;
 static __device__ uint32_t g_pair_ctr[kEagerPairs + kCapturedPairs][2];
 
+// tree: Q, K and V are [npad, H, 32] in slot order (whole-tile loads); otherwise [rows, H, 32] in the original
+// order, gathered through perm.  perm names the output row of every slot (or -1) either way.
 static bt_status launch_pair(const void *Q, const void *K, const void *V, const int32_t *perm, int64_t npad,
-                             int64_t rows, int lm, int H, void *O, cudaStream_t st)
+                             int64_t rows, int lm, int H, void *O, cudaStream_t st, bool tree = false)
 {
     static std::atomic<bool> set[64] = {};
     static int sms[64] = {0};
@@ -764,7 +792,9 @@ static bt_status launch_pair(const void *Q, const void *K, const void *V, const 
     if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
     if (dev < 0 || dev >= 64) return BT_ERR_UNSUPPORTED;
     const bt_status s0 = setup_once(set[dev], [&]() -> bt_status {
-        if (cudaFuncSetAttribute(k_ball_attn_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(k_ball_attn_pair<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(PairPipe::BYTES)) ||
+            cudaFuncSetAttribute(k_ball_attn_pair<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(PairPipe::BYTES)))
             return BT_ERR_CUDA;
         int n = 0;
@@ -789,14 +819,21 @@ static bt_status launch_pair(const void *Q, const void *K, const void *V, const 
     uint32_t *status = stream_status(st);
     if (!status) return BT_ERR_CUDA;
     CUtensorMap mq, mk, mv;
-    if (!row_map(&mq, Q, rows, H * 32, 64) || !row_map(&mk, K, rows, H * 32, 64) || !row_map(&mv, V, rows, H * 32, 64))
+    if (tree) {
+        if (!tile_map(&mq, Q, npad, H * 32, 64, 128) || !tile_map(&mk, K, npad, H * 32, 64, 128) ||
+            !tile_map(&mv, V, npad, H * 32, 64, 128))
+            return BT_ERR_CUDA;
+    } else if (!row_map(&mq, Q, rows, H * 32, 64) || !row_map(&mk, K, rows, H * 32, 64) ||
+               !row_map(&mv, V, rows, H * 32, 64)) {
         return BT_ERR_CUDA;
+    }
     const int nsm = dev < 64 && sms[dev] > 0 ? sms[dev] : 148;
     const int64_t items = (npad + 127) / 128 * (H / 2);
     if (items > 0x7FFFFFFF) return BT_ERR_UNSUPPORTED;
     const int64_t grid = items < int64_t(nsm) * PairPipe::PER_SM ? items : int64_t(nsm) * PairPipe::PER_SM;
     const float sl2 = 1.4426950408889634f / sqrtf(32.0f);
-    k_ball_attn_pair<<<unsigned(grid), PairPipe::THREADS, PairPipe::BYTES, st>>>(
+    auto kern = tree ? k_ball_attn_pair<true> : k_ball_attn_pair<false>;
+    kern<<<unsigned(grid), PairPipe::THREADS, PairPipe::BYTES, st>>>(
         mq, mk, mv, perm, npad, rows, lm, H, sl2, items, static_cast<__nv_bfloat16 *>(O), ctr, status);
     return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
 }
@@ -854,6 +891,7 @@ static bt_status launch_tc(const void *Q, const void *K, const void *V, const in
 }  // namespace bts
 
 #include "bts_bsa.cuh"
+#include "bts_project.cuh"
 
 using namespace bts;
 
@@ -885,3 +923,83 @@ extern "C" bt_status bt_ball_attention(const void *Q, const void *K, const void 
 }
 
 #include "bts_coarse.cuh"
+
+// ---------------------------------------------------------------------------
+// Projection into tree order and attention on tree-ordered Q/K/V
+// ---------------------------------------------------------------------------
+namespace bts {
+static bool pair_shape(int32_t m, int32_t H, int32_t d, bt_dtype dt, int64_t rows)
+{
+    return dt == BT_BF16 && d == 32 && H % 2 == 0 && (m == 16 || m == 32 || m == 64 || m == 128) &&
+           rows < 0x7FFFFFFF;
+}
+static int log2m(int32_t m) { return m == 16 ? 4 : m == 32 ? 5 : m == 64 ? 6 : 7; }
+}  // namespace bts
+
+extern "C" bt_status bt_qkv_project(const void *X, int64_t rows, int32_t C, const void *Wt, int32_t H, int32_t d,
+                                    bt_dtype dt, const int32_t *perm, const int32_t *inv, int64_t npad, void *Q,
+                                    void *K, void *V, void *stream)
+{
+    if (!X || !Wt || !Q || !K || !V || rows < 0 || C < 1 || H < 1 || d < 1) return BT_ERR_ARG;
+    if (dt != BT_F32 && dt != BT_BF16) return BT_ERR_ARG;
+    if (perm && (!inv || npad < 0)) return BT_ERR_ARG;
+    if (rows > 0x7FFFFFFF || npad > 0x7FFFFFFF || int64_t(H) * d * 3 > 65535) return BT_ERR_UNSUPPORTED;
+    if (!perm) npad = rows;
+    if (npad == 0 && rows == 0) return BT_OK;
+    return launch_project(X, rows, C, Wt, H, d, dt, perm, inv, npad, Q, K, V, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" bt_status bt_ball_attention_tree(const void *Qt, const void *Kt, const void *Vt, const int32_t *perm,
+                                            int64_t npad, int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt,
+                                            void *O, void *stream)
+{
+    if (!Qt || !Kt || !Vt || !O || !perm || npad < 0 || rows < 0 || H < 1) return BT_ERR_ARG;
+    if (m < 1 || npad % m) return BT_ERR_SHAPE;
+    if (npad == 0) return BT_OK;
+    // whole 128-slot tiles: the slot-ordered tensors must hold at least one
+    if (!pair_shape(m, H, d, dt, rows) || npad < 128 || npad > 0x7FFFFFFF) return BT_ERR_UNSUPPORTED;
+    const uintptr_t al = reinterpret_cast<uintptr_t>(Qt) | reinterpret_cast<uintptr_t>(Kt) |
+                         reinterpret_cast<uintptr_t>(Vt) | reinterpret_cast<uintptr_t>(O);
+    if (al % 16) return BT_ERR_ARG;
+    return launch_pair(Qt, Kt, Vt, perm, npad, rows, log2m(m), H, O, static_cast<cudaStream_t>(stream), true);
+}
+
+extern "C" size_t bt_projected_workspace_size(int64_t npad, int64_t rows, int32_t H, int32_t d, bt_dtype dt)
+{
+    if (npad < 0 || rows < 0 || H < 1 || d < 1 || (dt != BT_F32 && dt != BT_BF16)) return 0;
+    const int64_t n = npad > rows ? npad : rows;
+    const size_t one = (size_t(n) * H * d * (dt == BT_F32 ? 4 : 2) + 255) & ~size_t(255);
+    return 3 * one + ((size_t(rows) * 4 + 255) & ~size_t(255));  // Q, K, V and the inverse slot map
+}
+
+extern "C" bt_status bt_projected_ball_attention(const void *X, const int32_t *perm, int64_t npad, int64_t rows,
+                                                 int32_t C, const void *Wt, int32_t m, int32_t H, int32_t d,
+                                                 bt_dtype dt, void *O, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!X || !Wt || !O || npad < 0 || rows < 0 || C < 1 || H < 1) return BT_ERR_ARG;
+    if (m < 1 || m > 256 || (d != 32 && d != 64)) return BT_ERR_SHAPE;
+    if (npad % m) return BT_ERR_SHAPE;
+    if (!perm && rows < npad) return BT_ERR_ARG;
+    if (npad == 0) return BT_OK;
+    const size_t need = bt_projected_workspace_size(npad, rows, H, d, dt);
+    if (!ws || need == 0 || ws_bytes < need) return BT_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return BT_ERR_ARG;
+    const int64_t n = npad > rows ? npad : rows;
+    const size_t one = (size_t(n) * H * d * (dt == BT_F32 ? 4 : 2) + 255) & ~size_t(255);
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    void *Q = w, *K = w + one, *V = w + 2 * one;
+    int32_t *inv = reinterpret_cast<int32_t *>(w + 3 * one);
+    if (perm && pair_shape(m, H, d, dt, rows) && npad >= 128) {
+        // Q, K, V written in slot order (each feature row to its slot); the attention then loads every ball as one
+        // tile.  Every row must be named by a slot, as in a tree built over these rows.
+        bt_status s = bt_invert_perm(perm, npad, rows, inv, stream);
+        if (s != BT_OK) return s;
+        s = bt_qkv_project(X, rows, C, Wt, H, d, dt, perm, inv, npad, Q, K, V, stream);
+        if (s != BT_OK) return s;
+        return bt_ball_attention_tree(Q, K, V, perm, npad, rows, m, H, d, dt, O, stream);
+    }
+    // other shapes: Q, K, V in the original row order, then the gathering attention
+    bt_status s = bt_qkv_project(X, rows, C, Wt, H, d, dt, nullptr, nullptr, 0, Q, K, V, stream);
+    if (s != BT_OK) return s;
+    return bt_ball_attention(Q, K, V, perm, npad, rows, m, H, d, dt, O, stream);
+}

@@ -1353,6 +1353,51 @@ static size_t cluster_smem_bytes(int NC, int CS)
            size_t(6) * 256 * 4;
 }
 
+// Sorts the ids (field 3) of every leaf of 32*E slots in X[0..C) ascending, one warp per leaf: lane l holds the
+// leaf's slots l*E .. l*E+E-1 in registers; a bitonic network whose compare-exchanges are in-register for
+// partners in the same lane and shuffles across lanes otherwise.  emit(i, id) receives slot i's sorted id.
+template <int E, typename F>
+__device__ __forceinline__ void warp_sort_leaves(const unsigned long long *X, int C, int warp, int lane, int nwarps,
+                                                 F &&emit)
+{
+    constexpr int N = 32 * E;
+    for (int leaf = warp; leaf * N < C; leaf += nwarps) {
+        uint32_t v[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) v[e] = rfield(X[leaf * N + lane * E + e], 3);
+#pragma unroll
+        for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                if (j < E) {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        if ((e & j) == 0) {
+                            const bool up = ((lane * E + e) & k) == 0;
+                            const uint32_t a = v[e], c = v[e | j];
+                            if ((a > c) == up) {
+                                v[e] = c;
+                                v[e | j] = a;
+                            }
+                        }
+                    }
+                } else {
+                    const int lj = j / E;
+                    const bool lower = (lane & lj) == 0;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        const uint32_t o = __shfl_xor_sync(0xffffffffu, v[e], lj);
+                        const bool up = ((lane * E + e) & k) == 0;
+                        v[e] = (lower == up) ? min(v[e], o) : max(v[e], o);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) emit(leaf * N + lane * E + e, v[e]);
+    }
+}
+
 // NC CTAs per cluster; every cloud has a power-of-two slot count npad, and CTA r holds slots r*C..r*C+C-1
 // with C = npad / NC = 2^lc.  CS (>= every cloud's C, <= CMAX) is the list stride in shared memory.
 template <int NC, int CMAX>
@@ -1739,30 +1784,40 @@ __global__ void __launch_bounds__(kClusterThreads, 1)
     // the in-CTA levels read other CTAs' sorted-key tables: no CTA leaves before all of them are done
     cluster_arrive_release();
 
-    // --- perm: every leaf's ids (from list X), sorted ascending (bitonic in place) ----
-    uint32_t *ids = reinterpret_cast<uint32_t *>(scr);  // [C]
+    // --- perm: every leaf's ids (from list X), sorted ascending ----
+    // Leaves of 32..256 slots: one warp per leaf sorts the ids in registers (bitonic network, no block barrier);
+    // other leaf sizes: one bitonic network over the CTA's slots in shared memory.
     {
         const unsigned long long *X = L(cb, 0);
-        for (int i = tid; i < C; i += NT) ids[i] = rfield(X[i], 3);
-    }
-    __syncthreads();
-    for (int kk = 2; kk <= m; kk <<= 1) {
-        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-            for (int i = tid; i < C / 2; i += NT) {
-                const int lo = ((i & ~(jj - 1)) << 1) | (i & (jj - 1)), hi = lo + jj;
-                const bool up = kk == m || (lo & kk) == 0;  // every leaf of m slots ends ascending
-                const uint32_t x = ids[lo], y = ids[hi];
-                if ((x > y) == up) {
-                    ids[lo] = y;
-                    ids[hi] = x;
+        auto emit = [&](int i, uint32_t id) { perm[P.pad[b] + pos0 + i] = int(id) < n ? int32_t(P.row0[b] + id) : -1; };
+        if (m == 128)
+            warp_sort_leaves<4>(X, C, warp, lane, NT / 32, emit);
+        else if (m == 64)
+            warp_sort_leaves<2>(X, C, warp, lane, NT / 32, emit);
+        else if (m == 32)
+            warp_sort_leaves<1>(X, C, warp, lane, NT / 32, emit);
+        else if (m == 256)
+            warp_sort_leaves<8>(X, C, warp, lane, NT / 32, emit);
+        else {
+            uint32_t *ids = reinterpret_cast<uint32_t *>(scr);  // [C]
+            for (int i = tid; i < C; i += NT) ids[i] = rfield(X[i], 3);
+            __syncthreads();
+            for (int kk = 2; kk <= m; kk <<= 1) {
+                for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+                    for (int i = tid; i < C / 2; i += NT) {
+                        const int lo = ((i & ~(jj - 1)) << 1) | (i & (jj - 1)), hi = lo + jj;
+                        const bool up = kk == m || (lo & kk) == 0;  // every leaf of m slots ends ascending
+                        const uint32_t x = ids[lo], y = ids[hi];
+                        if ((x > y) == up) {
+                            ids[lo] = y;
+                            ids[hi] = x;
+                        }
+                    }
+                    __syncthreads();
                 }
             }
-            __syncthreads();
+            for (int i = tid; i < C; i += NT) emit(i, ids[i]);
         }
-    }
-    for (int i = tid; i < C; i += NT) {
-        const uint32_t id = ids[i];
-        perm[P.pad[b] + pos0 + i] = int(id) < n ? int32_t(P.row0[b] + id) : -1;
     }
     cluster_wait_acquire();
     __syncthreads();

@@ -85,7 +85,8 @@ def parse():
     p.add_argument("--no-suite", action="store_true", help="skip the other workloads")
     p.add_argument("--suite-steps", type=int, default=20)
     p.add_argument("--suite-only", default="",
-                   help="comma-separated suite workloads to time on their own (tiny, ellipsoid, ellipsoid_bsa, rows, "
+                   help="comma-separated suite workloads to time on their own (tiny, ellipsoid, ellipsoid_projected, "
+                        "ellipsoid_bsa, rows, "
                         "box_cluster, gauss_mix_coarse_levels, ragged); skips the headline step")
     return p.parse_args()
 
@@ -504,6 +505,8 @@ def suite(bts, dev, steps, flush, peak, only=None):
         _suite_tiny(bts, dev, steps, flush, res)
     if want("ellipsoid"):
         _suite_ellipsoid_layer(bts, dev, steps, flush, peak, res)
+    if want("ellipsoid_projected"):
+        _suite_ellipsoid_projected(bts, dev, steps, flush, peak, res)
     if want("ellipsoid_bsa"):
         _suite_ellipsoid(bts, dev, steps, flush, res)
     if want("rows"):
@@ -558,6 +561,49 @@ def _suite_ellipsoid_layer(bts, dev, steps, flush, peak, res):
                         "attention_gbs": nbytes / (a_ms / 1e3) / 1e9,
                         "attention_frac_of_measured_hbm": nbytes / (a_ms / 1e3) / 1e9 / peak}
     del q, k, v, out
+
+
+def _suite_ellipsoid_projected(bts, dev, steps, flush, peak, res):
+    # the ellipsoid layer from its features: tree build, inverse of perm, Q/K/V = X Wt^T written in slot order
+    # (tcgen05 projection of whole feature-row tiles, each output row stored at its slot), attention on whole
+    # slot-ordered tiles, O scattered back; beside it the present path's attention on given Q/K/V (gathered
+    # through perm)
+    wl = workloads.ellipsoid()
+    c = torch.from_numpy(wl.coords).to(dev)
+    x = _bf16_dev(wl.extra["x_bf16"], dev)
+    wt = _bf16_dev(np.ascontiguousarray(wl.extra["w_qkv_bf16"].T), dev)
+    n, C, H, d = wl.n_total, x.shape[1], wl.H, wl.d
+    perm = torch.empty(n, dtype=torch.int32, device=dev)
+    ws = bts.workspace([0, n], wl.m, dev)
+    pws = torch.empty(bts.bt_projected_workspace_size(n, n, H, d, torch.bfloat16), dtype=torch.uint8, device=dev)
+    out = torch.empty((n, H, d), dtype=torch.bfloat16, device=dev)
+    qkv = tuple(torch.empty((n, H, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    bts.bt_build(c, wl.m, perm=perm, ws=ws)
+
+    def layer():
+        bts.bt_build(c, wl.m, perm=perm, ws=ws)
+        bts.bt_projected_ball_attention(x, perm, wt, wl.m, H, d, out=out, ws=pws)
+    ms = statistics.mean(timed_graph(layer, steps, 3, flush))
+    inv = bts.bt_invert_perm(perm, n)
+    p_ms = statistics.mean(timed_graph(lambda: bts.bt_qkv_project(x, wt, H, d, perm=perm, inv=inv, out=qkv), steps, 3,
+                                       flush))
+    a_ms = statistics.mean(timed_graph(lambda: bts.bt_ball_attention_tree(*qkv, perm, wl.m, n, out=out), steps, 3,
+                                       flush))
+    row = H * d * 2
+    p_bytes = n * C * 2 + 3 * H * d * C * 2 + 3 * n * row + 4 * n  # X rows and Wt read, Q/K/V written, perm
+    a_bytes = 3 * n * row + n * row + 4 * n                         # Q/K/V tiles read, O written, perm
+    p_flop = 2 * n * C * 3 * H * d
+    res["ellipsoid_projected"] = {
+        "points": n, "C": C, "layers": 1, "ms_per_step": ms, "points_per_s_per_layer": n / (ms / 1e3),
+        "project_ms": p_ms, "project_gbs": p_bytes / (p_ms / 1e3) / 1e9,
+        "project_frac_of_measured_hbm": p_bytes / (p_ms / 1e3) / 1e9 / peak,
+        "project_tflops": p_flop / (p_ms / 1e3) / 1e12,
+        "attention_tree_ms": a_ms, "attention_tree_gbs": a_bytes / (a_ms / 1e3) / 1e9,
+        "attention_tree_frac_of_measured_hbm": a_bytes / (a_ms / 1e3) / 1e9 / peak,
+        "layer_bytes": p_bytes + a_bytes,
+        "note": "projection + attention from the features; compare the ellipsoid entry's attention_ms (given Q/K/V, "
+                "rows gathered through perm)"}
+    del x, wt, out, qkv, pws
 
 
 def _suite_rows(bts, dev, steps, flush, peak, res):

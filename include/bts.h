@@ -242,6 +242,67 @@ bt_status bt_ball_attention(const void *Q, const void *K, const void *V, const i
                             int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream);
 
 /*
+ * Q/K/V projection of the point features [E7][E9]: the attention layer's
+ * queries, keys and values are linear maps of each point's features, and a
+ * ball's points sit in consecutive slots, so writing the projections in slot
+ * order makes every ball one contiguous tile for bt_ball_attention_tree.
+ *   out[o(r), h, k] = sum_c X[r, c] * Wt[t*H*d + h*d + k, c]   (t = 0 Q, 1 K,
+ *   2 V) for every row r, with o(r) = inv[r] (slot order) when perm is given
+ *   and o(r) = r (original order) when perm is NULL.
+ *   X        dt [rows, C] device, original row order
+ *   Wt       dt [3*H*d, C] device: row j holds the weights of output column j
+ *            (the layout of a linear layer's weight)
+ *   perm     int32 [npad] device (slot -> row, -1 dummy) or NULL.  Given
+ *            perm, Q, K, V are [npad, H, d] in slot order and the rows of the
+ *            dummy slots are set to zero; inv (int32 [rows] device, inv[r] =
+ *            the slot of row r, as bt_invert_perm writes it) is required.  An
+ *            inv entry outside [0, npad) is skipped and recorded as
+ *            BT_ERR_INTERNAL.  NULL: Q, K, V are [rows, H, d] (inv, npad unused).
+ *   Q, K, V  dt device out
+ * The feature rows are read in their own order as whole tiles; each output
+ * row is stored at its slot.  BT_BF16 with C a multiple of 64 (at most 512),
+ * 3*H*d >= 256, rows >= 128 and 16-byte aligned pointers runs on the tcgen05
+ * tensor cores (fp32 accumulation, outputs rounded to bf16); every other shape
+ * on the CUDA cores in float.
+ */
+bt_status bt_qkv_project(const void *X, int64_t rows, int32_t C, const void *Wt, int32_t H, int32_t d, bt_dtype dt,
+                         const int32_t *perm, const int32_t *inv, int64_t npad, void *Q, void *K, void *V,
+                         void *stream);
+
+/*
+ * Ball attention of Q/K/V that are already in slot order (as bt_qkv_project
+ * writes them with tree_order): the same result as bt_ball_attention on the
+ * original-order tensors, with every ball loaded as one tile.
+ *   Qt, Kt, Vt  bf16 [npad, H, d] device, slot order
+ *   perm        int32 [npad] device: the output row of each slot, -1 for a
+ *               dummy slot (neither query nor key, nothing written)
+ *   O           bf16 [rows, H, d] device out, original row order
+ * Shapes: bf16, d = 32, even H, m in {16, 32, 64, 128}, npad >= 128
+ * (BT_ERR_UNSUPPORTED otherwise); the concurrency note of bt_ball_attention
+ * applies.
+ */
+bt_status bt_ball_attention_tree(const void *Qt, const void *Kt, const void *Vt, const int32_t *perm, int64_t npad,
+                                 int64_t rows, int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *stream);
+
+/*
+ * One attention layer from the features [E7][E9]: bt_qkv_project into a
+ * workspace, then ball attention.  For the shapes bt_ball_attention_tree takes
+ * (and a non-NULL perm) the projections are written in slot order and the
+ * attention loads whole tiles; otherwise they are written in the original
+ * order and bt_ball_attention gathers them.  Arguments as for the two calls;
+ * m and d as for bt_ball_attention.
+ *   ws  workspace of bt_projected_workspace_size(npad, rows, H, d, dt) bytes,
+ *       256-byte aligned (the projected Q, K and V, and the inverse of perm)
+ * With perm, every row must be named by a slot (as in a tree built over the
+ * rows); the slot-order path relies on it.
+ */
+size_t bt_projected_workspace_size(int64_t npad, int64_t rows, int32_t H, int32_t d, bt_dtype dt);
+
+bt_status bt_projected_ball_attention(const void *X, const int32_t *perm, int64_t npad, int64_t rows, int32_t C,
+                                      const void *Wt, int32_t m, int32_t H, int32_t d, bt_dtype dt, void *O, void *ws,
+                                      size_t ws_bytes, void *stream);
+
+/*
  * Ball Sparse Attention ("BSA: Ball Sparse Attention for Large-scale
  * Geometries", as reviewed on Pith: reading notes and referee report).  Three
  * branches per query row i and head h, mixed by sigmoid gates:

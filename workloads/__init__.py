@@ -105,12 +105,17 @@ def tiny(n: int = 1024, m: int = 32, C: int = 64, H: int = 2, d: int = 32) -> Wo
     wid = 1
     coords = _rng(wid, 1).random((n, 3)).astype(np.float32)
     x = _rng(wid, 2).standard_normal((n, C))
-    proj = []
+    proj, ws = [], []
     for j in range(3):
         w = _rng(wid, 3 + j).standard_normal((C, H * d)) / math.sqrt(C)
+        ws.append(w)
         proj.append((x @ w).astype(np.float32).reshape(n, H, d))
     wl = Workload("tiny", coords, np.array([0, n], np.int64), m, H, d, F32)
     wl.layers.append(Layer(proj[0], proj[1], proj[2], rotated=False))
+    # the same features and weights rounded to float, for a layer that projects on the device:
+    # X [n, C] and W [C, 3 H d] (Q, K, V column blocks)
+    wl.extra["x"] = x.astype(np.float32)
+    wl.extra["w_qkv"] = np.concatenate(ws, axis=1).astype(np.float32)
     return wl
 
 
@@ -131,7 +136,8 @@ def gauss_mix(n_per_cloud: int = 16384, batch: int = 4, m: int = 128, H: int = 8
 def ellipsoid(n: int = 65536, m: int = 128, C: int = 256, H: int = 8, d: int = 32,
               semi_axes=(2.0, 1.0, 0.7), jitter: float = 1e-3) -> Workload:
     """Points uniform on an ellipsoid surface (area-element rejection), plus Gaussian jitter.
-    Carries the gate features X [n, C] and gate weights W_g [C, 3H] ~ N(0, 1/C)."""
+    Carries the gate features X [n, C] and gate weights W_g [C, 3H] ~ N(0, 1/C); for a layer that projects its
+    own Q/K/V, X rounded to bf16 and projection weights W_qkv [C, 3 H d] ~ N(0, 1/C) in bf16 (raw bits)."""
     wid = 3
     a, b, c = semi_axes
     g = _rng(wid, 1)
@@ -154,6 +160,9 @@ def ellipsoid(n: int = 65536, m: int = 128, C: int = 256, H: int = 8, d: int = 3
     wl.layers.append(Layer(q, k, v, rotated=False))
     wl.extra["x"] = _rng(wid, 2).standard_normal((n, C), dtype=np.float32)
     wl.extra["w_g"] = (_rng(wid, 6).standard_normal((C, 3 * H)) / math.sqrt(C)).astype(np.float32)
+    wl.extra["x_bf16"] = f32_to_bf16_bits(wl.extra["x"])
+    wl.extra["w_qkv_bf16"] = f32_to_bf16_bits(
+        (_rng(wid, 7).standard_normal((C, 3 * H * d), dtype=np.float32) / np.float32(math.sqrt(C))).astype(np.float32))
     return wl
 
 
