@@ -514,9 +514,15 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                     if (cmask[q4] != 0u) {
                         uint32_t v[32];
                         tmem_ld32(tS + lanebase + q4 * 32, v);
+                        if (cmask[q4] == 0xffffffffu) {  // every key of the group valid: three-input max
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if ((cmask[q4] >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]));
+                            for (int j = 0; j < 32; j += 2)
+                                mx = fmax3(mx, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if ((cmask[q4] >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]));
+                        }
                     }
                 }
                 const float m_new = fmaxf(m_run, mx == -INFINITY ? -INFINITY : mx * sl2);
@@ -534,8 +540,10 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                         for (int j = 0; j < 32; j += 2) {
                             float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mref));
                             float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mref));
-                            p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
-                            p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                            if (cm != 0xffffffffu) {
+                                p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
+                                p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                            }
                             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                             pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
                             csum += p0 + p1;

@@ -12,14 +12,16 @@
 // The feature rows are read in their own order, as whole 128-row tiles (one TMA request per 64 columns), and
 // each output row is stored at its slot: scattered 16-byte stores cost the same as ordered ones, while
 // gathering the inputs row by row would cost one TMA request per four rows.
-// k_qkv_project (bf16, C a multiple of 64 up to 512): persistent CTAs over 128-row tiles, one per SM.
-//   warp 4     producer: loads the tile's feature rows (128 x 64 boxes, 128-byte swizzle; rows past the end
-//              read zeros), then streams 256 x 64 tiles of Wt;
-//   warp 5     one thread issues the tcgen05 products: for each chunk of 256 output columns, D (TMEM,
-//              fp32, two 256-column buffers) += X tile (K-major) * Wt tile (K-major), K = 64 per block;
-//   warps 0-3  epilogue: each thread reads its row of the finished chunk from TMEM, rounds to bf16 and
-//              stores 16-byte pieces to its row's slot of Q, K or V, while the next chunk accumulates in the
-//              other buffer.
+// k_qkv_project (bf16, C a multiple of 64 up to 512): weight-stationary, one CTA per SM.  The SMs are shared
+// out over the chunks of 256 output columns (128 when C > 256); a CTA loads its chunk of Wt into shared
+// memory once and walks its share of the 128-row tiles of X:
+//   warp 8     producer: the Wt chunk, then the tiles' 128 x 64 K blocks of X through a 4-stage ring (TMA
+//              tile loads, 128-byte swizzle; rows past the end read zeros);
+//   warp 9     one thread issues the tcgen05 products D (TMEM, fp32, two accumulator buffers) += X block
+//              (K-major) * Wt block (K-major), K = 64 per block;
+//   warps 0-7  epilogue: two warps per 32 rows (TMEM lanes), each reading half of the row's columns of a
+//              finished tile from TMEM, rounding to bf16 and storing 16-byte pieces to the row's slot of Q, K
+//              or V, while the next tile accumulates in the other buffer.
 // k_qkv_project_simt (float, or any shape the tensor-core kernel does not take): one thread per (row,
 // output column), features staged in shared memory.
 // k_zero_slots: zero rows of Q, K and V for the dummy slots (perm < 0), which no feature row fills.
@@ -29,20 +31,22 @@
 namespace bts {
 
 struct ProjPipe {
-    static constexpr int BM = 128;                    // slots per tile
+    static constexpr int BM = 128;                    // rows per tile
     static constexpr int BK = 64;                     // K elements per block: one 128-byte swizzle span
-    static constexpr int BN = 256;                    // output columns per accumulator buffer
-    static constexpr uint32_t XBLK = BM * BK * 2;     // 16 KB: one K block of the gathered X tile
-    static constexpr uint32_t WBLK = BN * BK * 2;     // 32 KB: one K block of a 256-column chunk of Wt
-    static constexpr int WS = 3;                      // Wt stages
-    static constexpr int THREADS = 192;
+    static constexpr uint32_t XBLK = BM * BK * 2;     // 16 KB: one K block of an X tile
+    static constexpr int XS = 4;                      // X ring stages (one K block each)
+    static constexpr int THREADS = 320;                // 8 epilogue warps, producer, tensor-core issuer
     static constexpr int CMAX = 512;
-    static uint32_t x_bufs(int C) { return C <= 256 ? 2u : 1u; }
-    static uint32_t bytes(int C) { return x_bufs(C) * (C / BK) * XBLK + WS * WBLK + 1024; }
+    // output columns per CTA (its Wt chunk stays in shared memory): 256, or 128 when C > 256
+    static int bn(int C) { return C <= 256 ? 256 : 128; }
+    static uint32_t bytes(int C) { return uint32_t(C / BK) * uint32_t(bn(C)) * 128u + XS * XBLK + 1024; }
 };
 
-// inv != NULL: feature row r goes to row inv[r] of Q/K/V (slot order; a slot outside [0, npad) is skipped and
-// recorded as BT_ERR_INTERNAL); inv == NULL: to row r (original order).
+// Weight-stationary: CTA b owns output chunk b % nch (bn columns of Wt, loaded once into shared memory) and
+// walks the 128-row tiles b / nch, b / nch + groups, ...  inv != NULL: feature row r goes to row inv[r] of
+// Q/K/V (slot order; a slot outside [0, npad) is skipped and recorded as BT_ERR_INTERNAL); inv == NULL: to
+// row r (original order).
+template <int BN>
 __global__ void __launch_bounds__(ProjPipe::THREADS, 1)
     k_qkv_project(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                   const int32_t *__restrict__ inv, int64_t npad, int64_t rows, int C, int nout, int hd,
@@ -51,17 +55,20 @@ __global__ void __launch_bounds__(ProjPipe::THREADS, 1)
 {
     using L = ProjPipe;
     constexpr uint32_t SBO8 = 8 * 128, SW128 = 2;
-    constexpr uint32_t IDESC = idesc_bf16(L::BN, false);
+    constexpr uint32_t IDESC = idesc_bf16(BN, false);
+    constexpr uint32_t WBLK = BN * 128;  // one K block of the Wt chunk
     extern __shared__ __align__(1024) uint8_t xsm[];
-    __shared__ __align__(8) uint64_t sXFull[2], sXEmpty[2], sWFull[L::WS], sWEmpty[L::WS], sAccFull[2], sAccEmpty[2];
+    __shared__ __align__(8) uint64_t sWFull, sXFull[L::XS], sXEmpty[L::XS], sAccFull[2], sAccEmpty[2];
     __shared__ uint32_t sTmem;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int KB = C / L::BK;
-    const int NCH = (nout + L::BN - 1) / L::BN;
-    const int XB = C <= 256 ? 2 : 1;
-    const uint32_t base = (smem_u32(xsm) + 1023u) & ~1023u;
-    const uint32_t wbase = base + uint32_t(XB * KB) * L::XBLK;
+    const int nch = (nout + BN - 1) / BN;
+    const int chunk = int(blockIdx.x) % nch;
+    const int64_t groups = int64_t(gridDim.x) / nch;
+    const int64_t first = int64_t(blockIdx.x) / nch;
+    const uint32_t base = (smem_u32(xsm) + 1023u) & ~1023u;   // Wt chunk: KB blocks of [BN][128 B]
+    const uint32_t xbase = base + uint32_t(KB) * WBLK;        // X ring
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sTmem)),
@@ -70,15 +77,14 @@ __global__ void __launch_bounds__(ProjPipe::THREADS, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sWFull)) : "memory");
+        for (int i = 0; i < L::XS; ++i) {
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sXFull[i])) : "memory");
             asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sXEmpty[i])) : "memory");
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sAccFull[i])) : "memory");
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 4;" ::"r"(smem_u32(&sAccEmpty[i])) : "memory");
         }
-        for (int i = 0; i < L::WS; ++i) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sWFull[i])) : "memory");
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sWEmpty[i])) : "memory");
+        for (int i = 0; i < 2; ++i) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sAccFull[i])) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 8;" ::"r"(smem_u32(&sAccEmpty[i])) : "memory");
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -87,119 +93,105 @@ __global__ void __launch_bounds__(ProjPipe::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = sTmem;
 
-    if (warp == 4) {
-        // ---------------- producer ----------------
-        bool ok = true;
-        int wi = 0;
-        int xi = 0;
-        for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++xi) {
-            const int xb = xi % XB;
-            if (xi >= XB) ok = mbar_wait(smem_u32(&sXEmpty[xb]), ((xi / XB) - 1) & 1, status);
-            if (!ok) break;
-            const uint32_t xfull = smem_u32(&sXFull[xb]);
-            if (lane == 0) {
-                mbar_expect_tx(xfull, uint32_t(KB) * L::XBLK);
-                const uint32_t xdst = base + uint32_t(xb * KB) * L::XBLK;
-                for (int k = 0; k < KB; ++k)
-                    tma_load_2d(xdst + k * L::XBLK, &tmX, k * L::BK, int32_t(tile * L::BM), xfull);
-            }
-            __syncwarp();
-            for (int n = 0; n < NCH && ok; ++n)
-                for (int k = 0; k < KB && ok; ++k, ++wi) {
-                    const int s = wi % L::WS;
-                    if (lane == 0) {
-                        if (wi >= L::WS) ok = mbar_wait(smem_u32(&sWEmpty[s]), ((wi / L::WS) - 1) & 1, status);
-                        if (ok) {
-                            mbar_expect_tx(smem_u32(&sWFull[s]), L::WBLK);
-                            tma_load_2d(wbase + s * L::WBLK, &tmW, k * L::BK, n * L::BN, smem_u32(&sWFull[s]));
-                        }
-                    }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                }
-        }
-    } else if (warp == 5) {
-        // ---------------- tensor-core issue (one thread) ----------------
+    if (warp == 8) {
+        // ---------------- producer (one thread): the Wt chunk once, then the X tiles' K blocks ----------------
         if (lane == 0) {
             bool ok = true;
-            int wi = 0, ai = 0, xi = 0;
-            for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++xi) {
-                const int xb = xi % XB;
-                ok = mbar_wait(smem_u32(&sXFull[xb]), (xi / XB) & 1, status);
-                tc_fence_after();
-                const uint32_t xs = base + uint32_t(xb * KB) * L::XBLK;
-                for (int n = 0; n < NCH && ok; ++n, ++ai) {
-                    const int ab = ai & 1;
-                    if (ai >= 2) ok = mbar_wait(smem_u32(&sAccEmpty[ab]), ((ai >> 1) - 1) & 1, status);
-                    tc_fence_after();
-                    const uint32_t tacc = tmem + uint32_t(ab) * L::BN;
-                    for (int k = 0; k < KB && ok; ++k, ++wi) {
-                        const int s = wi % L::WS;
-                        ok = mbar_wait(smem_u32(&sWFull[s]), (wi / L::WS) & 1, status);
-                        tc_fence_after();
-                        if (ok) {
-                            const uint32_t xa = xs + k * L::XBLK, wb = wbase + s * L::WBLK;
-#pragma unroll
-                            for (int kk = 0; kk < L::BK / 16; ++kk)
-                                mma_bf16(tacc, smem_desc_sw(xa + 32 * kk, 16, SBO8, SW128),
-                                         smem_desc_sw(wb + 32 * kk, 16, SBO8, SW128), IDESC, (k | kk) != 0);
-                        }
-                        mma_commit(smem_u32(&sWEmpty[s]));  // the Wt stage is free once these products finish
+            mbar_expect_tx(smem_u32(&sWFull), uint32_t(KB) * WBLK);
+            for (int k = 0; k < KB; ++k)
+                tma_load_2d(base + k * WBLK, &tmW, k * L::BK, chunk * BN, smem_u32(&sWFull));
+            int xi = 0;
+            for (int64_t tile = first; tile < tiles && ok; tile += groups)
+                for (int k = 0; k < KB && ok; ++k, ++xi) {
+                    const int s = xi % L::XS;
+                    if (xi >= L::XS) ok = mbar_wait(smem_u32(&sXEmpty[s]), ((xi / L::XS) - 1) & 1, status);
+                    if (ok) {
+                        mbar_expect_tx(smem_u32(&sXFull[s]), L::XBLK);
+                        tma_load_2d(xbase + s * L::XBLK, &tmX, k * L::BK, int32_t(tile * L::BM), smem_u32(&sXFull[s]));
                     }
-                    mma_commit(smem_u32(&sAccFull[ab]));
                 }
-                mma_commit(smem_u32(&sXEmpty[xb]));
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ---------------- tensor-core issue (one thread) ----------------
+        if (lane == 0) {
+            bool ok = mbar_wait(smem_u32(&sWFull), 0, status);
+            tc_fence_after();
+            int xi = 0, ai = 0;
+            for (int64_t tile = first; tile < tiles && ok; tile += groups, ++ai) {
+                const int ab = ai & 1;
+                if (ai >= 2) ok = mbar_wait(smem_u32(&sAccEmpty[ab]), ((ai >> 1) - 1) & 1, status);
+                tc_fence_after();
+                const uint32_t tacc = tmem + uint32_t(ab) * BN;
+                for (int k = 0; k < KB && ok; ++k, ++xi) {
+                    const int s = xi % L::XS;
+                    ok = mbar_wait(smem_u32(&sXFull[s]), (xi / L::XS) & 1, status);
+                    tc_fence_after();
+                    if (ok) {
+                        const uint32_t xa = xbase + s * L::XBLK, wb = base + k * WBLK;
+#pragma unroll
+                        for (int kk = 0; kk < L::BK / 16; ++kk)
+                            mma_bf16(tacc, smem_desc_sw(xa + 32 * kk, 16, SBO8, SW128),
+                                     smem_desc_sw(wb + 32 * kk, 16, SBO8, SW128), IDESC, (k | kk) != 0);
+                    }
+                    mma_commit(smem_u32(&sXEmpty[s]));  // the X stage is free once these products finish
+                }
+                mma_commit(smem_u32(&sAccFull[ab]));
             }
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue: thread r owns row r of the tile (TMEM lane r) ----------------
-        const int r = tid;
-        const uint32_t lanebase = uint32_t(warp * 32) << 16;
+        // ---------------- epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 (rows of the tile) and the
+        // column half w / 4 of the accumulator; two 32-column loads in flight per wait ----------------
+        const int r = (warp & 3) * 32 + lane;
+        const int half = warp >> 2;
+        const uint32_t lanebase = uint32_t((warp & 3) * 32) << 16;
         bool ok = true;
         int ai = 0;
-        for (int64_t tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            // the output row of this thread's feature row
+        for (int64_t tile = first; tile < tiles && ok; tile += groups, ++ai) {
             const int64_t row = tile * L::BM + r;
             int32_t orow = -1;
             if (row < rows) {
                 orow = inv ? __ldg(inv + row) : int32_t(row);
                 if (inv && (orow < 0 || orow >= npad)) {  // not a slot: never write it
-                    record_error(status, BT_ERR_INTERNAL);
+                    if (half == 0) record_error(status, BT_ERR_INTERNAL);
                     orow = -1;
                 }
             }
-            for (int n = 0; n < NCH && ok; ++n, ++ai) {
-                const int ab = ai & 1;
-                ok = mbar_wait(smem_u32(&sAccFull[ab]), (ai >> 1) & 1, status);
-                tc_fence_after();
-                const uint32_t tacc = tmem + uint32_t(ab) * L::BN + lanebase;
-                for (int c = 0; c < L::BN / 32; ++c) {
-                    const int col0 = n * L::BN + c * 32;
-                    if (col0 >= nout) break;  // the same for every thread of the warp
-                    uint32_t v[32];
-                    tmem_ld32(tacc + c * 32, v);
-                    if (ok && orow >= 0) {
+            const int ab = ai & 1;
+            ok = mbar_wait(smem_u32(&sAccFull[ab]), (ai >> 1) & 1, status);
+            tc_fence_after();
+            const uint32_t tacc = tmem + uint32_t(ab) * BN + uint32_t(half * (BN / 2)) + lanebase;
+#pragma unroll 1
+            for (int c = 0; c < BN / 2 / 32; c += 2) {
+                const int col0 = chunk * BN + half * (BN / 2) + c * 32;
+                if (col0 >= nout) break;  // the same for every thread of the warp
+                uint32_t v[2][32];
+                tmem_ld32_nowait(tacc + c * 32, v[0]);
+                tmem_ld32_nowait(tacc + (c + 1) * 32, v[1]);
+                tmem_wait_ld();
+                if (ok && orow >= 0) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            const int j0 = col0 + 8 * g;
-                            if (j0 >= nout) break;  // 3*H*d is a multiple of 8, so a group never straddles it
-                            const int t = j0 / hd, within = j0 - t * hd;
-                            __nv_bfloat16 *dst = (t == 0 ? Qo : t == 1 ? Ko : Vo) + size_t(orow) * hd + within;
-                            uint32_t w[4];
+                    for (int g = 0; g < 8; ++g) {
+                        const int j0 = col0 + 8 * g;
+                        if (j0 >= nout) break;  // 3*H*d is a multiple of 8, so a group never straddles it
+                        const int t = j0 / hd, within = j0 - t * hd;
+                        __nv_bfloat16 *dst = (t == 0 ? Qo : t == 1 ? Ko : Vo) + size_t(orow) * hd + within;
+                        const uint32_t *vv = v[g >> 2] + 8 * (g & 3);
+                        uint32_t w[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(v[8 * g + 2 * e]),
-                                                                                __uint_as_float(v[8 * g + 2 * e + 1]));
-                                w[e] = *reinterpret_cast<const uint32_t *>(&pb);
-                            }
-                            *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 pb =
+                                __floats2bfloat162_rn(__uint_as_float(vv[2 * e]), __uint_as_float(vv[2 * e + 1]));
+                            w[e] = *reinterpret_cast<const uint32_t *>(&pb);
                         }
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sAccEmpty[ab])) : "memory");
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sAccEmpty[ab])) : "memory");
         }
     }
     tc_fence_before();
@@ -294,7 +286,7 @@ static bt_status launch_project(const void *X, int64_t rows, int32_t C, const vo
     const uintptr_t al = reinterpret_cast<uintptr_t>(X) | reinterpret_cast<uintptr_t>(Wt) |
                          reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) |
                          reinterpret_cast<uintptr_t>(V);
-    if (dt == BT_BF16 && C % ProjPipe::BK == 0 && C <= ProjPipe::CMAX && hd % 8 == 0 && nout >= ProjPipe::BN &&
+    if (dt == BT_BF16 && C % ProjPipe::BK == 0 && C <= ProjPipe::CMAX && hd % 8 == 0 && nout >= ProjPipe::bn(C) &&
         al % 16 == 0 && rows >= ProjPipe::BM && rows < 0x7FFFFFFF) {
         static std::atomic<bool> set[64] = {};
         static int sms[64] = {0};
@@ -302,8 +294,10 @@ static bt_status launch_project(const void *X, int64_t rows, int32_t C, const vo
         if (cudaGetDevice(&dev) != cudaSuccess) return BT_ERR_CUDA;
         if (dev < 0 || dev >= 64) return BT_ERR_UNSUPPORTED;
         const bt_status s0 = setup_once(set[dev], [&]() -> bt_status {
-            const uint32_t mx = ProjPipe::bytes(256) > ProjPipe::bytes(512) ? ProjPipe::bytes(256) : ProjPipe::bytes(512);
-            if (cudaFuncSetAttribute(k_qkv_project, cudaFuncAttributeMaxDynamicSharedMemorySize, int(mx)))
+            if (cudaFuncSetAttribute(k_qkv_project<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(ProjPipe::bytes(256))) ||
+                cudaFuncSetAttribute(k_qkv_project<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(ProjPipe::bytes(512))))
                 return BT_ERR_CUDA;
             int n = 0;
             if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return BT_ERR_CUDA;
@@ -311,15 +305,25 @@ static bt_status launch_project(const void *X, int64_t rows, int32_t C, const vo
             return BT_OK;
         });
         if (s0 != BT_OK) return s0;
+        const int BN = ProjPipe::bn(C);
         CUtensorMap mx, mw;
-        if (!tile_map(&mx, X, rows, C, ProjPipe::BK, ProjPipe::BM) ||
-            !tile_map(&mw, Wt, nout, C, ProjPipe::BK, ProjPipe::BN))
+        if (!tile_map(&mx, X, rows, C, ProjPipe::BK, ProjPipe::BM) || !tile_map(&mw, Wt, nout, C, ProjPipe::BK, BN))
             return BT_ERR_CUDA;
         const int64_t tiles = (rows + ProjPipe::BM - 1) / ProjPipe::BM;
-        const int64_t grid = tiles < sms[dev] ? tiles : sms[dev];
-        k_qkv_project<<<unsigned(grid), ProjPipe::THREADS, ProjPipe::bytes(C), st>>>(
-            mx, mw, perm ? inv : nullptr, npad, rows, C, nout, hd, tiles, static_cast<__nv_bfloat16 *>(Q),
-            static_cast<__nv_bfloat16 *>(K), static_cast<__nv_bfloat16 *>(V), status);
+        const int nch = (nout + BN - 1) / BN;
+        // CTAs per output chunk: the SMs shared out, no more than there are tiles
+        int64_t groups = sms[dev] / nch;
+        if (groups < 1) groups = 1;
+        if (groups > tiles) groups = tiles;
+        const unsigned grid = unsigned(groups * nch);
+        if (BN == 256)
+            k_qkv_project<256><<<grid, ProjPipe::THREADS, ProjPipe::bytes(C), st>>>(
+                mx, mw, perm ? inv : nullptr, npad, rows, C, nout, hd, tiles, static_cast<__nv_bfloat16 *>(Q),
+                static_cast<__nv_bfloat16 *>(K), static_cast<__nv_bfloat16 *>(V), status);
+        else
+            k_qkv_project<128><<<grid, ProjPipe::THREADS, ProjPipe::bytes(C), st>>>(
+                mx, mw, perm ? inv : nullptr, npad, rows, C, nout, hd, tiles, static_cast<__nv_bfloat16 *>(Q),
+                static_cast<__nv_bfloat16 *>(K), static_cast<__nv_bfloat16 *>(V), status);
         return cudaPeekAtLastError() == cudaSuccess ? BT_OK : BT_ERR_CUDA;
     }
     const size_t smem = size_t(32) * C * sizeof(float);
