@@ -138,14 +138,14 @@ __global__ void __launch_bounds__(kMeanWarps * 32) k_bsa_means(const __nv_bfloat
 }
 
 // ---------------------------------------------------------------------------
-// Gates: two rows per thread (rows t and t + kGateThreads of the CTA's
-// kGateRows), kGateOut outputs at a time in registers.  W is staged once per
-// CTA with its rows padded to a multiple of kGateOut (zeros), so one column of
-// X costs two scalar reads of X and kGateOut/4 broadcast float4 reads of W
-// for 2 * kGateOut FMAs.  X streams through shared memory kGateCols columns at
-// a time, double-buffered: the next slice is loaded into registers (coalesced
-// float4) while the current one is used.
-constexpr int kGateThreads = 128, kGateRows = 2 * kGateThreads, kGateCols = 16, kGateOut = 24;
+// Gates: sigmoid(bg + X W) per row and output.  One CTA per kGateRows rows; thread t takes row t % kGateRows
+// and half t / kGateRows of every group of kGateOut outputs (kGateOut / 2 accumulators in registers).  W is
+// staged once per CTA with its rows padded to a multiple of kGateOut (zeros).  X streams through shared
+// memory kGateCols columns at a time, double-buffered (the next slice is loaded into registers as coalesced
+// float4 while the current one is used); its rows are padded by one word, so the 32 rows a warp reads at
+// one column sit in 32 banks, and the W reads of a warp are broadcasts.  Many small CTAs keep enough X in
+// flight per SM to stream it at memory speed.
+constexpr int kGateThreads = 256, kGateRows = 128, kGateCols = 32, kGateOut = 24, kGateHalf = kGateOut / 2;
 
 static int gate_out_padded(int H) { return (3 * H + kGateOut - 1) / kGateOut * kGateOut; }
 
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kGateThreads) k_bsa_gates(const float *__restr
                                                             float *__restrict__ gates)
 {
     extern __shared__ __align__(16) float gsm[];
-    constexpr int XP = kGateCols + 1;  // odd row stride: the 32 rows a warp reads sit in 32 banks
+    constexpr int XP = kGateCols + 1;
     constexpr int U = kGateRows * kGateCols / 4 / kGateThreads;  // float4 of a slice per thread
     const int NO = 3 * H;
     float *sW = gsm, *sX = gsm + size_t(C) * NOP;  // sX: [2][kGateRows][XP]
@@ -190,18 +190,19 @@ __global__ void __launch_bounds__(kGateThreads) k_bsa_gates(const float *__restr
         }
     }
     const int64_t r0 = int64_t(blockIdx.x) * kGateRows;
-    const int64_t ra = r0 + tid, rb = ra + kGateThreads;  // this thread's two rows
+    const int rr = tid % kGateRows, half = tid / kGateRows;
+    const int64_t row = r0 + rr;
     const bool vec4 = (C % 4) == 0 && (reinterpret_cast<uintptr_t>(X) % 16) == 0;
     const int nslice = (C + kGateCols - 1) / kGateCols;
-    // one slice of X into registers: row rr = i / (kGateCols/4), columns c0 + 4*(i % (kGateCols/4)) .. +3
+    // one slice of X into registers: row i / (kGateCols/4) of the tile, columns c0 + 4*(i % (kGateCols/4)) .. +3
     auto load_slice = [&](int c0, float4 (&t)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = tid + u * kGateThreads, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+            const int i = tid + u * kGateThreads, lr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
             const int c = c0 + 4 * c4;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r0 + rr < rows) {
-                const float *src = X + (r0 + rr) * C + c;
+            if (r0 + lr < rows) {
+                const float *src = X + (r0 + lr) * C + c;
                 if (vec4 && c + 4 <= C) {
                     v = *reinterpret_cast<const float4 *>(src);
                 } else {
@@ -217,36 +218,19 @@ __global__ void __launch_bounds__(kGateThreads) k_bsa_gates(const float *__restr
     auto store_slice = [&](int buf, const float4 (&t)[U]) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int i = tid + u * kGateThreads, rr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
-            float *d = sX + (size_t(buf) * kGateRows + rr) * XP + 4 * c4;
+            const int i = tid + u * kGateThreads, lr = i / (kGateCols / 4), c4 = i % (kGateCols / 4);
+            float *d = sX + (size_t(buf) * kGateRows + lr) * XP + 4 * c4;
             d[0] = t[u].x;
             d[1] = t[u].y;
             d[2] = t[u].z;
             d[3] = t[u].w;
         }
     };
-    // one column of the slice: x of both rows against kGateOut weights
-    auto column = [&](const float *xa, const float *xb, const float *wrow, float (&aa)[kGateOut],
-                      float (&ab)[kGateOut]) {
-        const float x0 = *xa, x1 = *xb;
-        const float4 *w4 = reinterpret_cast<const float4 *>(wrow);
-#pragma unroll
-        for (int j4 = 0; j4 < kGateOut / 4; ++j4) {
-            const float4 w = w4[j4];
-            aa[4 * j4] = fmaf(x0, w.x, aa[4 * j4]);
-            aa[4 * j4 + 1] = fmaf(x0, w.y, aa[4 * j4 + 1]);
-            aa[4 * j4 + 2] = fmaf(x0, w.z, aa[4 * j4 + 2]);
-            aa[4 * j4 + 3] = fmaf(x0, w.w, aa[4 * j4 + 3]);
-            ab[4 * j4] = fmaf(x1, w.x, ab[4 * j4]);
-            ab[4 * j4 + 1] = fmaf(x1, w.y, ab[4 * j4 + 1]);
-            ab[4 * j4 + 2] = fmaf(x1, w.z, ab[4 * j4 + 2]);
-            ab[4 * j4 + 3] = fmaf(x1, w.w, ab[4 * j4 + 3]);
-        }
-    };
     for (int j0 = 0; j0 < NO; j0 += kGateOut) {
-        float acc_a[kGateOut], acc_b[kGateOut];
+        const int jh = j0 + half * kGateHalf;  // this thread's first output
+        float acc[kGateHalf];
 #pragma unroll
-        for (int j = 0; j < kGateOut; ++j) acc_a[j] = acc_b[j] = (bg && j0 + j < NO) ? bg[j0 + j] : 0.0f;
+        for (int j = 0; j < kGateHalf; ++j) acc[j] = (bg && jh + j < NO) ? bg[jh + j] : 0.0f;
         float4 t[U];
         load_slice(0, t);
         __syncthreads();  // W is staged; neither buffer is read any more
@@ -255,27 +239,29 @@ __global__ void __launch_bounds__(kGateThreads) k_bsa_gates(const float *__restr
         for (int k = 0; k < nslice; ++k) {
             const int c0 = k * kGateCols;
             if (k + 1 < nslice) load_slice(c0 + kGateCols, t);  // in flight while slice k is used
-            const float *xa = sX + (size_t(k & 1) * kGateRows + tid) * XP;
-            const float *xb = xa + kGateThreads * XP;
-            const float *wr = sW + size_t(c0) * NOP + j0;
-            if (C - c0 >= kGateCols) {
-#pragma unroll 4
-                for (int cc = 0; cc < kGateCols; ++cc) column(xa + cc, xb + cc, wr + size_t(cc) * NOP, acc_a, acc_b);
-            } else {
-                for (int cc = 0; cc < C - c0; ++cc) column(xa + cc, xb + cc, wr + size_t(cc) * NOP, acc_a, acc_b);
+            const float *xr = sX + (size_t(k & 1) * kGateRows + rr) * XP;
+            const float *wr = sW + size_t(c0) * NOP + jh;
+            const int ncol = C - c0 < kGateCols ? C - c0 : kGateCols;
+#pragma unroll 8
+            for (int cc = 0; cc < ncol; ++cc) {
+                const float x = xr[cc];
+                const float4 *w4 = reinterpret_cast<const float4 *>(wr + size_t(cc) * NOP);
+#pragma unroll
+                for (int q = 0; q < kGateHalf / 4; ++q) {
+                    const float4 w = w4[q];
+                    acc[4 * q] = fmaf(x, w.x, acc[4 * q]);
+                    acc[4 * q + 1] = fmaf(x, w.y, acc[4 * q + 1]);
+                    acc[4 * q + 2] = fmaf(x, w.z, acc[4 * q + 2]);
+                    acc[4 * q + 3] = fmaf(x, w.w, acc[4 * q + 3]);
+                }
             }
             if (k + 1 < nslice) store_slice((k + 1) & 1, t);  // the other buffer: nobody reads it now
             __syncthreads();
         }
-        if (ra < rows) {
+        if (row < rows) {
 #pragma unroll
-            for (int j = 0; j < kGateOut; ++j)
-                if (j0 + j < NO) gates[ra * NO + j0 + j] = 1.0f / (1.0f + expf(-acc_a[j]));
-        }
-        if (rb < rows) {
-#pragma unroll
-            for (int j = 0; j < kGateOut; ++j)
-                if (j0 + j < NO) gates[rb * NO + j0 + j] = 1.0f / (1.0f + expf(-acc_b[j]));
+            for (int j = 0; j < kGateHalf; ++j)
+                if (jh + j < NO) gates[row * NO + jh + j] = 1.0f / (1.0f + expf(-acc[j]));
         }
     }
 }

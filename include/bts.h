@@ -324,7 +324,7 @@ bt_status bt_projected_ball_attention(const void *X, const int32_t *perm, int64_
  *   X        float [rows, C] gate features (original row order)
  *   Wg       float [C, 3H] gate weights;  bg  float [3H] or NULL (zero);
  *            W is staged in shared memory: C * (3H rounded up to 24) * 4
- *            bytes + 33,280 must not exceed 200 KiB (BT_ERR_UNSUPPORTED)
+ *            bytes + 33,792 must not exceed 200 KiB (BT_ERR_UNSUPPORTED)
  *   O        bf16 [rows, H, d] out
  *   sel_out  int32 [npad/m, H, topk] out (may be NULL): the selected balls per
  *            (group, head), -1 where fewer than topk balls can be selected

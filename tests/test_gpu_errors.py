@@ -39,9 +39,11 @@ def test_nonfinite_reported_on_device(bad):
     ws = bts.workspace([0, 4096], 32)
     bts.bt_build(torch.from_numpy(pts).cuda(), 32, ws=ws)
     assert bts.bt_build_device_status(ws) == 3  # BT_ERR_NONFINITE
+    assert bts.bt_last_device_status() == 3  # the stream's word says the same, and is cleared by reading it
     # the context stays usable: a clean build on the same workspace reports OK
     bts.bt_build(torch.from_numpy(workloads.uniform_cloud(4096, 4)).cuda(), 32, ws=ws)
     assert bts.bt_build_device_status(ws) == 0
+    assert bts.bt_last_device_status() == 0
 
 
 @pytest.mark.parametrize("n,m,flags", [(4096, 32, 1), (65536, 128, 0), (3000, 16, 1)])
@@ -53,8 +55,10 @@ def test_nonfinite_reported_on_every_build_shape(n, m, flags):
     ws = bts.workspace([0, n], m)
     bts.bt_build_segmented_ex(torch.from_numpy(pts).cuda(), [0, n], m, flags, ws=ws)
     assert bts.bt_build_device_status(ws) == 3
+    assert bts.bt_last_device_status() == 3
     bts.bt_build_segmented_ex(torch.from_numpy(workloads.uniform_cloud(n, 6)).cuda(), [0, n], m, flags, ws=ws)
     assert bts.bt_build_device_status(ws) == 0
+    assert bts.bt_last_device_status() == 0
 
 
 def test_segmented_argument_errors():
