@@ -8,8 +8,7 @@ points, m = 128, H = 8, d = 32, bf16):
            inverse of tree A and the A->B slot map, ball attention on tree B.
 The two trees depend only on the coordinates, so tree B is built on a second
 stream (narrow clusters: half the SMs per cloud) while tree A is built and
-layer A attends; layer B's attention follows the slot maps on that stream and
-takes the SMs as layer A's attention finishes.
+layer A attends; the attention layers run one after the other.
 Metric: points per second per layer = 2 layers * 65,536 points / step time.
 
 The step is captured once as a CUDA graph and replayed; every timed replay is
@@ -17,8 +16,8 @@ bracketed by CUDA events on the replay stream, with a 256 MB write between
 replays to flush L2.  Event nodes inside a graph cost about 17 us per step, so
 the timed graph has none: after every timed replay (outside its timing) an
 instrumented copy of the step graph, with event nodes between the phases, is
-replayed once for the per-phase breakdown, and a graph of layer B's attention
-alone, between event nodes, gives the dominant kernel's launch time.
+replayed once, and the dominant kernel's duration (ball attention of layer B,
+which runs alone on the GPU) and the per-phase breakdown come from it.
 `--impl reference` times the CPU oracle instead (bounded samples of the same
 workload on the host cores).
 """
@@ -49,12 +48,11 @@ UNIT = "points/s"
 LAYERS = 2
 
 # DRAM traffic of one launch of the dominant kernel on this workload (ncu dram__bytes_read.sum +
-# dram__bytes_write.sum, mean of two launches of the bench step) and the hash of the attention source it was
-# taken on (code lines only).  Reported only while that source is unchanged; null otherwise.  The hash was
-# refreshed once after a change to host-side launch set-up only (the kernel's code is the captured one).
+# dram__bytes_write.sum, mean of three launches of the bench step) and the hash of the attention source it was
+# taken on (code lines only).  Reported only while that source is unchanged; null otherwise.
 ROOF_KERNEL = "k_ball_attn_pair"
-ROOF_TRAFFIC = {"bytes": 107546752,
-                "source_sha256": "27fdbea8ffd5a457d312b2beccb0f7a9212b3a211f4c7ccf3790284394487b76"}
+ROOF_TRAFFIC = {"bytes": 109391445,
+                "source_sha256": "e68190086ffa588f369c44cd17bb0efc8de4922993da8dfaecb61b8b7ddafae3"}
 _ATTN_SOURCES = ("ball_tree_sparse_b200/csrc/bts_attn.cu", "ball_tree_sparse_b200/csrc/bts_tc.cuh")
 
 
@@ -217,7 +215,7 @@ class Step:
         self.side = torch.cuda.Stream(device=dev)
         self.rt = _cudart()
         self.rt.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
-        self.ev = {k: torch.cuda.Event(enable_timing=True) for k in ("a0", "a1", "a2", "b1", "b2", "x1", "x2")}
+        self.ev = {k: torch.cuda.Event(enable_timing=True) for k in ("a0", "a1", "a2", "b1", "b2")}
         self.marks = True
         self.graph = None
 
@@ -236,10 +234,10 @@ class Step:
     def body(self, capturing=False, marks=True):
         """Both trees are built concurrently (they depend only on the coordinates): tree A with the
         default (wide) clusters on the main stream, tree B with narrow ones on the side stream, so that
-        it leaves most SMs to tree A and then to layer A's attention.  Once tree A is built, the side
-        stream computes the slot maps (inverse of tree A, A->B map) and launches layer B's attention,
-        whose CTAs take the SMs as layer A's persistent CTAs finish; the main stream builds tree A and
-        runs layer A's attention, then joins the side stream.  marks=False leaves out the event nodes."""
+        it leaves most SMs to tree A and then to layer A's attention.  The slot maps (inverse of tree A,
+        A->B map) follow tree B on the side stream once tree A is built; the two attention layers run
+        one after the other on the main stream (each launch's persistent CTAs hold the SMs until it
+        ends, so a second stream would not overlap them).  marks=False leaves out the event nodes."""
         bts, wl = self.bts, self.wl
         main = torch.cuda.current_stream()
         self.marks = marks
@@ -255,26 +253,18 @@ class Step:
         with torch.cuda.stream(self.side):
             bts.bt_invert_perm(self.perm[0], self.n, inv=self.inv)
             bts.bt_compose(self.inv, self.perm[1], out=self.map)
-            self._mark("b1", capturing)
-            bts.bt_ball_attention(*self.qkv[1], self.perm[1], wl.m, out=self.out[1])
-            self._mark("b2", capturing)
         bts.bt_ball_attention(*self.qkv[0], self.perm[0], wl.m, out=self.out[0])
         self._mark("a2", capturing)
         main.wait_stream(self.side)
-
-    def attn_only(self, capturing=False):
-        """Layer B's attention alone, between event nodes: the dominant kernel's launch time."""
-        self.marks = True
-        self._mark("x1", capturing)
-        self.bts.bt_ball_attention(*self.qkv[1], self.perm[1], self.wl.m, out=self.out[1])
-        self._mark("x2", capturing)
+        self._mark("b1", capturing)
+        bts.bt_ball_attention(*self.qkv[1], self.perm[1], wl.m, out=self.out[1])
+        self._mark("b2", capturing)
 
     def capture(self):
         """self.graph: the step as timed (no event nodes); self.graph_marked: the same step with event
         nodes between its phases, for the kernel duration and the breakdown."""
         for _ in range(3):
-            self.body()
-            self.attn_only()  # also creates the events that the graph's event nodes record
+            self.body()  # also creates the events that the graph's event nodes record
         torch.cuda.synchronize()
         self.graph = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(self.graph):
@@ -284,19 +274,12 @@ class Step:
         self.graph_marked = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph_marked):
             self.body(capturing=True, marks=True)
-        self.graph_attn = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph_attn):
-            self.attn_only(capturing=True)
         torch.cuda.synchronize()
 
     def times(self):
         e = self.ev
         return {"build_a": e["a0"].elapsed_time(e["a1"]), "attn_a": e["a1"].elapsed_time(e["a2"]),
-                "maps_and_start_b": e["a1"].elapsed_time(e["b1"]), "attn_b_window": e["b1"].elapsed_time(e["b2"]),
-                "a_end_to_b_end": e["a2"].elapsed_time(e["b2"])}
-
-    def attn_time(self):
-        return self.ev["x1"].elapsed_time(self.ev["x2"])
+                "join_b_and_maps": e["a2"].elapsed_time(e["b1"]), "attn_b": e["b1"].elapsed_time(e["b2"])}
 
 
 def e2e_pipelined(st_a, st_b, host_in, steps) -> float:
@@ -812,8 +795,7 @@ def main():
     torch.cuda.synchronize()
     clocks.mark()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ms, attn_ms = [], []
-    parts = {"build_a": 0.0, "attn_a": 0.0, "maps_and_start_b": 0.0, "attn_b_window": 0.0, "a_end_to_b_end": 0.0}
+    step_ms, attn_ms, parts = [], [], {"build_a": 0.0, "attn_a": 0.0, "join_b_and_maps": 0.0, "attn_b": 0.0}
     for _ in range(args.steps):
         flush.zero_()
         s0.record()
@@ -825,12 +807,9 @@ def main():
         st.graph_marked.replay()
         torch.cuda.synchronize()
         tt = st.times()
+        attn_ms.append(tt["attn_b"])  # layer B's attention runs alone on the GPU
         for k in parts:
             parts[k] += tt[k]
-        flush.zero_()  # layer B's attention alone on the GPU, for the dominant kernel's launch time
-        st.graph_attn.replay()
-        torch.cuda.synchronize()
-        attn_ms.append(st.attn_time())
     torch.cuda.synchronize()
     clocks.mark()
     if dist:
@@ -883,8 +862,8 @@ def main():
         "roofline": {"bound": "hbm", "kernel": ROOF_KERNEL, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
                      "bytes_per_launch": attn_bytes, "avg_launch_ms": attn_avg_ms,
-                     "avg_launch_ms_source": "event nodes around layer B's attention alone in a graph of its own, "
-                                             "replayed (after an L2 flush) once after every timed replay",
+                     "avg_launch_ms_source": "event nodes around layer B's attention in the instrumented copy of "
+                                             "the step graph, replayed once after every timed replay",
                      "traffic": roof_traffic(),
                      # context: the same launch against the dense bf16 tensor peak (4 m d H flop per point); at
                      # 64 flop per byte the HBM roofline caps it near a quarter of that peak
@@ -892,8 +871,7 @@ def main():
                                         "frac_of_dense_bf16": attn_flop / (attn_avg_ms / 1e3) / 1e12 / tpeak,
                                         "peak_tflops": tpeak, "peak_source": tpeak_kind}},
         "breakdown_ms_per_step": {k: v / args.steps for k, v in parts.items()},
-        "breakdown_source": "instrumented copy of the step graph (its event nodes add to these phases); layer B's "
-                            "attention runs on the side stream and overlaps the end of layer A's",
+        "breakdown_source": "instrumented copy of the step graph (its event nodes add to these phases)",
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "pipelined": "two step buffers; copies in, step graph and copies out on "
                                                  "three streams, overlapped across steps",
