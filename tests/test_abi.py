@@ -97,3 +97,33 @@ def test_binding_constants_match_the_header():
     assert (b.BT_F32, b.BT_BF16) == (enum["BT_F32"], enum["BT_BF16"])
     assert b.MAX_CLOUDS == defines["BT_MAX_CLOUDS"]
     assert b.BT_BUILD_NARROW == defines["BT_BUILD_NARROW"]
+
+
+def test_projection_calls_check_arguments_before_any_launch(lib):
+    P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    one = ctypes.c_void_p(16)
+    lib.bt_qkv_project.argtypes = [P, i64, i32, P, i32, i32, ctypes.c_int, P, P, i64, P, P, P, P]
+    assert lib.bt_qkv_project(None, 128, 64, one, 2, 32, 1, None, None, 0, one, one, one, None) == 1  # no X
+    assert lib.bt_qkv_project(one, 128, 64, one, 2, 32, 1, one, None, 128, one, one, one, None) == 1  # perm, no inv
+    assert lib.bt_qkv_project(one, 128, 0, one, 2, 32, 1, None, None, 0, one, one, one, None) == 1     # C < 1
+    assert lib.bt_qkv_project(one, 128, 64, one, 2, 32, 7, None, None, 0, one, one, one, None) == 1    # dtype
+    assert lib.bt_qkv_project(one, 128, 64, one, 2048, 32, 1, None, None, 0, one, one, one, None) == 7  # 3Hd too big
+    lib.bt_ball_attention_tree.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, ctypes.c_int, P, P]
+    assert lib.bt_ball_attention_tree(one, one, one, None, 256, 256, 128, 2, 32, 1, one, None) == 1  # perm required
+    assert lib.bt_ball_attention_tree(one, one, one, one, 200, 256, 128, 2, 32, 1, one, None) == 2   # npad % m
+    assert lib.bt_ball_attention_tree(one, one, one, one, 256, 256, 128, 2, 64, 1, one, None) == 7   # d = 64
+    assert lib.bt_ball_attention_tree(one, one, one, one, 256, 256, 128, 3, 32, 1, one, None) == 7   # odd H
+    assert lib.bt_ball_attention_tree(one, one, one, one, 64, 64, 32, 2, 32, 1, one, None) == 7      # npad < 128
+    lib.bt_projected_workspace_size.argtypes = [i64, i64, i32, i32, ctypes.c_int]
+    lib.bt_projected_workspace_size.restype = ctypes.c_size_t
+    ws = lib.bt_projected_workspace_size(1024, 1000, 8, 32, 1)
+    assert ws >= 3 * 1024 * 8 * 32 * 2 + 1000 * 4          # Q, K, V in slot order and the inverse slot map
+    assert lib.bt_projected_workspace_size(1024, 1000, 8, 32, 5) == 0
+    lib.bt_projected_ball_attention.argtypes = [P, P, i64, i64, i32, P, i32, i32, i32, ctypes.c_int, P, P,
+                                                ctypes.c_size_t, P]
+    assert lib.bt_projected_ball_attention(one, one, 1024, 1000, 64, one, 128, 8, 48, 1, one, one, ws,
+                                           None) == 2       # d = 48
+    assert lib.bt_projected_ball_attention(one, one, 1024, 1000, 64, one, 128, 8, 32, 1, one, one, ws - 1,
+                                           None) == 4       # workspace too small
+    assert lib.bt_projected_ball_attention(one, one, 1024, 1000, 64, one, 128, 8, 32, 1, one, ctypes.c_void_p(272),
+                                           ws, None) == 1   # workspace not 256-byte aligned
