@@ -349,6 +349,25 @@ __global__ void __launch_bounds__(kTopkWarps * 32) k_bsa_topk(const float *__res
 }
 
 // ---------------------------------------------------------------------------
+// TMEM accesses of 16 / 8 consecutive 32-bit columns, one lane per thread (the load waits for its data).
+__device__ __forceinline__ void bsa_tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void bsa_tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 template <int D>
 struct BsaPipe {
     static constexpr uint32_t QK_BYTES = 128 * D * 2;
@@ -377,6 +396,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
     constexpr uint32_t IDESC_O = idesc_bf16(D, true);
     extern __shared__ __align__(1024) uint8_t bsm[];
     __shared__ uint32_t sKeyMask[4];
+    __shared__ int32_t sSel[kBsaMaxTopk];  // the item's selected balls
     __shared__ __align__(8) uint64_t sBarS, sBarO;
     __shared__ uint32_t sTmem;
 
@@ -412,21 +432,31 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
         }
         return r;
     };
-    // row r (0..127) of key chunk c of item (g, h): its source row, or -1
-    auto chunk_row = [&](int g, int h, int c, int r) -> int32_t {
+    // The source rows of a key chunk are fetched one chunk ahead (raw values: the ball's point count for a
+    // compression key, the perm entry for a selected one) and decoded when the chunk is issued, so the loads
+    // of perm and of the counts never stall the chunk in flight.
+    auto chunk_live = [&](int c) -> bool { return c < ncc || sSel[c - ncc] >= 0; };
+    auto fetch_raw = [&](int c, int r) -> int32_t {
+        if (c >= ncc + topk || !chunk_live(c)) return -1;
         if (c < ncc) {
             const int t = c * 128 + r;
-            return (t < nb && cnt[t] > 0) ? t : -1;
+            return t < nb ? cnt[t] : 0;
         }
-        const int s = sel[(size_t(g) * H + h) * topk + (c - ncc)];
-        if (s < 0) return -1;
-        return perm ? valid_row(perm[int64_t(s) * 128 + r]) : int32_t(int64_t(s) * 128 + r);
+        const int64_t slot = int64_t(sSel[c - ncc]) * 128 + r;
+        return perm ? perm[slot] : int32_t(slot);
     };
-    auto chunk_live = [&](int g, int h, int c) -> bool {
-        return c < ncc || sel[(size_t(g) * H + h) * topk + (c - ncc)] >= 0;
+    auto decode = [&](int c, int r, int32_t raw) -> int32_t {
+        if (c < ncc) return raw > 0 ? c * 128 + r : -1;
+        return raw >= 0 ? valid_row(raw) : -1;
     };
-    auto issue_chunk = [&](int g, int h, int c) {
-        if (c < ncc + topk && chunk_live(g, h, c)) {
+    int32_t nraw[UPT], nkey;  // the next chunk's raw values: the rows this thread loads, and key row tid
+    auto fetch_chunk = [&](int c) {
+#pragma unroll
+        for (int i = 0; i < UPT; ++i) nraw[i] = fetch_raw(c, (tid + i * kTcThreads) / KCH);
+        nkey = fetch_raw(c, tid);
+    };
+    auto issue_chunk = [&](int h, int c) {
+        if (c < ncc + topk && chunk_live(c)) {
             const bool cmp = c < ncc;
             const __nv_bfloat16 *kb = cmp ? kc : K, *vb = cmp ? vc : V;
             uint8_t *sk = bsm + L::STAGE_OFF + (c & 1) * L::STAGE, *sv = sk + L::QK_BYTES;
@@ -434,7 +464,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
             for (int i = 0; i < UPT; ++i) {
                 const int u = tid + i * kTcThreads;
                 const int r = u / KCH, cc = u - r * KCH;
-                const int32_t rr = chunk_row(g, h, c, r);
+                const int32_t rr = decode(c, r, nraw[i]);
                 const size_t goff = rr >= 0 ? (size_t(rr) * H + h) * D + cc * 8 : 0;
                 cp_async16(sk + (r >> 3) * QK_SBO + cc * 128 + (r & 7) * 16, kb + goff, rr >= 0);
                 cp_async16(sv + cc * V_SBO + r * 16, vb + goff, rr >= 0);
@@ -445,6 +475,8 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
 
     for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
         const int g = int(item / H), h = int(item - int64_t(g) * H);
+        if (tid < topk) sSel[tid] = sel[(size_t(g) * H + h) * topk + tid];
+        __syncthreads();  // the previous item's chunks are done with sSel
         // Q rows of the group (as the ball attention gathers them)
         {
             uint8_t *sq = bsm + L::Q_OFF;
@@ -457,14 +489,19 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                 cp_async16(sq + (r >> 3) * QK_SBO + cc * 128 + (r & 7) * 16, Q + goff, rr >= 0);
             }
         }
-        issue_chunk(g, h, 0);  // committed together with Q
+        fetch_chunk(0);
+        issue_chunk(h, 0);  // committed together with Q
+        int32_t ckey = nkey;  // key row tid of the chunk in flight
+        fetch_chunk(1);
         float o_acc[D], o_cmp[D];
         float m_run = -INFINITY, l_run = 0.0f;
         const int nchunks = ncc + topk;
         for (int c = 0; c < nchunks; ++c) {
-            issue_chunk(g, h, c + 1);
-            const bool live = chunk_live(g, h, c);
-            const int32_t kr = live ? chunk_row(g, h, c, tid) : -1;
+            issue_chunk(h, c + 1);
+            const bool live = chunk_live(c);
+            const int32_t kr = live ? decode(c, tid, ckey) : -1;
+            ckey = nkey;
+            fetch_chunk(c + 2);
             const uint32_t kb = __ballot_sync(0xffffffffu, kr >= 0);
             if (lane == 0) sKeyMask[warp] = kb;
             asm volatile("cp.async.wait_group 1;" ::: "memory");
@@ -516,17 +553,18 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                 const float alpha = m_run == -INFINITY ? 0.0f : ex2(m_run - mref);
                 float csum = 0.0f;  // this chunk's row sum of the weights, on the FMA pipe
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t pk[16];
-                    if (cmask[q4] != 0u) {
-                        uint32_t v[32];
-                        tmem_ld32(tS + lanebase + q4 * 32, v);
-                        const uint32_t cm = cmask[q4];
+                // sixteen keys at a time (the weights of 16 keys are 8 packed columns): few registers live
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    uint32_t pk[8];
+                    const uint32_t cm = (cmask[q8 >> 1] >> (16 * (q8 & 1))) & 0xFFFFu;
+                    if (cm != 0u) {
+                        uint32_t v[16];
+                        bsa_tmem_ld16(tS + lanebase + q8 * 16, v);
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
+                        for (int j = 0; j < 16; j += 2) {
                             float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mref));
                             float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mref));
-                            if (cm != 0xffffffffu) {
+                            if (cm != 0xFFFFu) {
                                 p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
                                 p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
                             }
@@ -536,9 +574,9 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                        for (int j = 0; j < 8; ++j) pk[j] = 0u;
                     }
-                    tmem_st16(tS + lanebase + q4 * 16, pk);
+                    bsa_tmem_st8(tS + lanebase + q8 * 8, pk);
                 }
                 asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                 tc_fence_before();
