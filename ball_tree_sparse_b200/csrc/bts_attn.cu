@@ -295,16 +295,24 @@ __global__ void __launch_bounds__(kTcThreads, TcPipe<D>::PER_SM)
                 uint32_t v[32];
                 tmem_ld32(tS + lanebase + c * 32, v);
                 const uint32_t cm = cmask[c];
+                if (__all_sync(0xffffffffu, cm == 0xffffffffu)) {  // every key valid: no per-key selects
 #pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
-                    float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
-                    if (cm != 0xffffffffu) {
+                    for (int j = 0; j < 32; j += 2) {
+                        const float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+                        const float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mxs));
+                        float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mxs));
                         p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
                         p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
                     }
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
                 }
             } else {
 #pragma unroll
@@ -636,19 +644,28 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
                     uint32_t v[32];
                     tmem_ld32(tS + lanebase + c * 32, v);
                     const uint32_t cm = cmask[c];
+                    if (__all_sync(0xffffffffu, cm == 0xffffffffu)) {  // every key valid: no per-key selects
 #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        float p0, p1;
-                        ffma2_bcast(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), sl2, -mxs, p0, p1);
-                        p0 = ex2(p0);
-                        p1 = ex2(p1);
-                        if (cm != 0xffffffffu) {
-                            p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
-                            p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                        for (int j = 0; j < 32; j += 2) {
+                            float p0, p1;
+                            ffma2_bcast(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), sl2, -mxs, p0, p1);
+                            p0 = ex2(p0);
+                            p1 = ex2(p1);
+                            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                            pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                            fadd2_acc(rs0, rs1, p0, p1);
                         }
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                        pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-                        fadd2_acc(rs0, rs1, p0, p1);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            float p0, p1;
+                            ffma2_bcast(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), sl2, -mxs, p0, p1);
+                            p0 = ((cm >> j) & 1u) ? ex2(p0) : 0.0f;
+                            p1 = ((cm >> (j + 1)) & 1u) ? ex2(p1) : 0.0f;
+                            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                            pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                            fadd2_acc(rs0, rs1, p0, p1);
+                        }
                     }
                 } else {
 #pragma unroll

@@ -557,17 +557,26 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                 for (int q8 = 0; q8 < 8; ++q8) {
                     uint32_t pk[8];
                     const uint32_t cm = (cmask[q8 >> 1] >> (16 * (q8 & 1))) & 0xFFFFu;
-                    if (cm != 0u) {
+                    if (cm == 0xFFFFu) {  // every key valid: no per-key selects
+                        uint32_t v[16];
+                        bsa_tmem_ld16(tS + lanebase + q8 * 16, v);
+#pragma unroll
+                        for (int j = 0; j < 16; j += 2) {
+                            const float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mref));
+                            const float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mref));
+                            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                            pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+                            csum += p0 + p1;
+                        }
+                    } else if (cm != 0u) {
                         uint32_t v[16];
                         bsa_tmem_ld16(tS + lanebase + q8 * 16, v);
 #pragma unroll
                         for (int j = 0; j < 16; j += 2) {
                             float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mref));
                             float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mref));
-                            if (cm != 0xFFFFu) {
-                                p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
-                                p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
-                            }
+                            p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
+                            p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
                             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                             pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
                             csum += p0 + p1;
