@@ -551,7 +551,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                 const float m_new = fmaxf(m_run, mx == -INFINITY ? -INFINITY : mx * sl2);
                 const float mref = m_new == -INFINITY ? 0.0f : m_new;
                 const float alpha = m_run == -INFINITY ? 0.0f : ex2(m_run - mref);
-                float csum = 0.0f;  // this chunk's row sum of the weights, on the FMA pipe
+                float cs0 = 0.0f, cs1 = 0.0f;  // this chunk's row sum of the weights (even and odd keys)
 #pragma unroll
                 // sixteen keys at a time (the weights of 16 keys are 8 packed columns): few registers live
                 for (int q8 = 0; q8 < 8; ++q8) {
@@ -562,24 +562,26 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                         bsa_tmem_ld16(tS + lanebase + q8 * 16, v);
 #pragma unroll
                         for (int j = 0; j < 16; j += 2) {
-                            const float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mref));
-                            const float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mref));
+                            float p0, p1;
+                            ffma2_bcast(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), sl2, -mref, p0, p1);
+                            p0 = ex2(p0);
+                            p1 = ex2(p1);
                             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                             pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-                            csum += p0 + p1;
+                            fadd2_acc(cs0, cs1, p0, p1);
                         }
                     } else if (cm != 0u) {
                         uint32_t v[16];
                         bsa_tmem_ld16(tS + lanebase + q8 * 16, v);
 #pragma unroll
                         for (int j = 0; j < 16; j += 2) {
-                            float p0 = ex2(fmaf(__uint_as_float(v[j]), sl2, -mref));
-                            float p1 = ex2(fmaf(__uint_as_float(v[j + 1]), sl2, -mref));
-                            p0 = ((cm >> j) & 1u) ? p0 : 0.0f;
-                            p1 = ((cm >> (j + 1)) & 1u) ? p1 : 0.0f;
+                            float p0, p1;
+                            ffma2_bcast(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), sl2, -mref, p0, p1);
+                            p0 = ((cm >> j) & 1u) ? ex2(p0) : 0.0f;
+                            p1 = ((cm >> (j + 1)) & 1u) ? ex2(p1) : 0.0f;
                             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                             pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-                            csum += p0 + p1;
+                            fadd2_acc(cs0, cs1, p0, p1);
                         }
                     } else {
 #pragma unroll
@@ -601,7 +603,7 @@ __global__ void __launch_bounds__(kTcThreads, BsaPipe<D>::PER_SM)
                 ++nO;
                 tc_fence_after();
                 if (ok) {
-                    l_run = l_run * alpha + csum;
+                    l_run = l_run * alpha + (cs0 + cs1);
 #pragma unroll
                     for (int c32 = 0; c32 < D; c32 += 32) {
                         uint32_t o[32];
