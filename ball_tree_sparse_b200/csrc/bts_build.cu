@@ -57,6 +57,10 @@ struct Plan {
     int32_t tail0[BT_MAX_CLOUDS + 1];
 };
 
+// A wide level's per-tile counts words sit one cache line (16 words) apart: every later tile of the node polls
+// each of them, and packed into a few lines they were a hot spot.
+constexpr size_t kAggStride = 16;
+
 struct Layout {
     size_t counters, hist, sst, lst, ctrl_end, keys, sk, sv, lists, total;
 };
@@ -164,7 +168,7 @@ static Layout make_layout(const Plan &P)
     L.hist = 512;
     L.sst = L.hist + size_t(3) * P.B * 4 * 256 * 4;
     L.lst = L.sst + size_t(4) * 3 * P.sort_tiles * 256 * 4;
-    L.ctrl_end = align256(L.lst + size_t(std::max(P.nlev, 1)) * (np / P.TP) * 8);
+    L.ctrl_end = align256(L.lst + size_t(std::max(P.nlev, 1)) * (np / P.TP) * 8 * kAggStride);
     L.keys = L.ctrl_end;
     L.sk = align256(L.keys + 3 * np * 4);
     L.sv = align256(L.sk + 2 * 3 * np * 4);
@@ -584,18 +588,18 @@ __global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level(Plan 
         }
     unsigned long long tot = 0;
     const unsigned long long ex = block_exclusive_scan<NT, unsigned long long>(packed, scratch, &tot);
-    unsigned long long *node_agg = agg + size_t(lev) * (np / TP) + (id - j);
+    unsigned long long *node_agg = agg + (size_t(lev) * (np / TP) + (id - j)) * kAggStride;
     if (tid == 0) {
         unsigned long long w = kAggPublished;
 #pragma unroll
         for (int l = 0; l < 4; ++l) w |= ((tot >> (16 * l)) & 0xFFFFull) << (15 * l);
-        st_relaxed_u64(node_agg + j, w);
+        st_relaxed_u64(node_agg + size_t(j) * kAggStride, w);
     }
     {
         // left counts of the tiles before this one in the node: two 32-bit sums per 64-bit word
         unsigned long long a01 = 0, a23 = 0;
         for (int t = tid; t < j; t += NT) {
-            unsigned long long w = ld_relaxed_u64(node_agg + t);
+            unsigned long long w = ld_relaxed_u64(node_agg + size_t(t) * kAggStride);
             int spins = 0;
             while (!(w & kAggPublished)) {
                 if (++spins > kSpinLimit) {
@@ -604,7 +608,7 @@ __global__ void __launch_bounds__(kLevelThreads, EPT <= 2 ? 2 : 1) k_level(Plan 
                     break;
                 }
                 __nanosleep(32);
-                w = ld_relaxed_u64(node_agg + t);
+                w = ld_relaxed_u64(node_agg + size_t(t) * kAggStride);
             }
             a01 += (w & 0x7FFFull) | (((w >> 15) & 0x7FFFull) << 32);
             a23 += ((w >> 30) & 0x7FFFull) | (((w >> 45) & 0x7FFFull) << 32);
@@ -1027,17 +1031,17 @@ __global__ void __launch_bounds__(kLevelThreads, 2) k_level_r(
     __syncthreads();
     const unsigned long long tot =
         uint64_t(s_ltot[0]) | (uint64_t(s_ltot[1]) << 16) | (uint64_t(s_ltot[2]) << 32);
-    unsigned long long *node_agg = agg + size_t(lev) * (np / TP) + (id - j);
+    unsigned long long *node_agg = agg + (size_t(lev) * (np / TP) + (id - j)) * kAggStride;
     if (tid == 0) {
         unsigned long long w = kAggPublished;
 #pragma unroll
         for (int l = 0; l < 3; ++l) w |= ((tot >> (16 * l)) & 0xFFFFull) << (15 * l);
-        st_relaxed_u64(node_agg + j, w);
+        st_relaxed_u64(node_agg + size_t(j) * kAggStride, w);
     }
     {
         unsigned long long a01 = 0, a2 = 0;
         for (int t = tid; t < j; t += NT) {
-            unsigned long long w = ld_relaxed_u64(node_agg + t);
+            unsigned long long w = ld_relaxed_u64(node_agg + size_t(t) * kAggStride);
             int spins = 0;
             while (!(w & kAggPublished)) {
                 if (++spins > kSpinLimit) {
@@ -1046,7 +1050,7 @@ __global__ void __launch_bounds__(kLevelThreads, 2) k_level_r(
                     break;
                 }
                 __nanosleep(32);
-                w = ld_relaxed_u64(node_agg + t);
+                w = ld_relaxed_u64(node_agg + size_t(t) * kAggStride);
             }
             a01 += (w & 0x7FFFull) | (((w >> 15) & 0x7FFFull) << 32);
             a2 += (w >> 30) & 0x7FFFull;
