@@ -4,9 +4,11 @@ The block selection is a discrete decision taken from float scores: the GPU
 scores in float32, the oracle in float64.  Selected sets must be equal, except
 where the blocks that differ tie with the k-th best block to within 1e-4 in the
 oracle's own scores; the outputs are then compared with the oracle recomputed
-on the GPU's selection (max-abs 2e-2, bf16 inputs and outputs).  The
-query-coarsening variant (compression and selection with each group's pooled
-query) is compared with the oracle's coarsened BSA the same way.
+on the GPU's selection: max-abs 2e-2 and max-abs at most REL_BF16 = 0.08 of the
+output RMS (bf16 inputs and outputs; each branch is a ball-attention-like softmax
+whose error is bounded that way, see the ball attention tests, and the gates are
+below one).  The query-coarsening variant (compression and selection with each
+group's pooled query) is compared with the oracle's coarsened BSA the same way.
 """
 import numpy as np
 import pytest
@@ -20,6 +22,14 @@ bts = pytest.importorskip("ball_tree_sparse_b200")
 
 TIE = 1e-4
 TOL = 2e-2
+REL_BF16 = 0.08
+
+
+def _check(got, want):
+    err, rms = np.abs(got - want).max(), np.sqrt((want.astype(np.float64) ** 2).mean())
+    print(f"parity: max_abs {err:.3e} rms {rms:.3e} max_abs/rms {err / rms:.3e}")
+    assert err <= TOL, f"max abs err {err}"
+    assert err / rms <= REL_BF16, f"max abs err {err} is {err / rms:.3f} of the output rms {rms}"
 
 
 def _dev(a):
@@ -83,8 +93,7 @@ def test_bsa_matches_oracle(orc, sizes, H, topk, mask_own, d, coarsen):
         ref = orc.bsa(q, k, v, 128, perm, x, w, b, topk=topk, mask_own=mask_own, sel_in=sel, branches=True,
                       coarsen=coarsen)
     real = perm[perm >= 0]
-    err = np.abs(got[real] - ref["O"][real]).max()
-    assert err <= TOL, f"max abs err {err}"
+    _check(got[real], ref["O"][real])
 
 
 @pytest.mark.parametrize("C,H", [(13, 10), (40, 2)])
@@ -96,8 +105,7 @@ def test_bsa_gate_shapes(orc, C, H):
     _check_selection(sel, orc.bsa(q, k, v, 128, perm, x, w, b, topk=3, mask_own=True, branches=True), 3)
     ref = orc.bsa(q, k, v, 128, perm, x, w, b, topk=3, mask_own=True, sel_in=sel, branches=True)
     real = perm[perm >= 0]
-    err = np.abs(got[real] - ref["O"][real]).max()
-    assert err <= TOL, f"max abs err {err}"
+    _check(got[real], ref["O"][real])
 
 
 def test_bsa_selection_pinned_by_exact_ties(orc):
@@ -123,5 +131,4 @@ def test_bsa_ellipsoid_full_size_sampled_groups(orc, coarsen):
     ref = orc.bsa(L.q, L.k, L.v, 128, perm, wl.extra["x"], wl.extra["w_g"], topk=8, sel_in=sel, groups=groups,
                   coarsen=coarsen)
     rows = np.concatenate([perm[gi * 128:(gi + 1) * 128] for gi in groups])
-    err = np.abs(got[rows] - ref[rows]).max()
-    assert err <= TOL, f"max abs err {err}"
+    _check(got[rows], ref[rows])

@@ -4,7 +4,8 @@ Pooling accumulates in float32 and rounds to the tensor's dtype: float32 is
 compared at 1e-5 (relative to the value's scale), bf16 at one bf16 rounding
 (2^-8 relative).  The coarse slot map and unpooling (a copy) are bit-exact.
 Coarse-level attention follows the ball attention tolerances: 1e-4 for
-float32, 2e-2 for bf16 (max abs).  At stride 1 the coarse path must give the
+float32, 2e-2 for bf16 (max abs) and, for bf16, a max-abs error of at most 0.08 of the
+output RMS.  At stride 1 the coarse path must give the
 fine ball attention bit for bit (same rows, same order, same kernel).
 """
 import numpy as np
@@ -16,6 +17,16 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 bts = pytest.importorskip("ball_tree_sparse_b200")
+
+REL_BF16 = 0.08  # max-abs error at most this share of the output RMS (the ball attention tests' bound)
+
+
+def _check_attention(got, want, bf16):
+    err, rms = np.abs(got - want).max(), np.sqrt((np.asarray(want, np.float64) ** 2).mean())
+    print(f"parity: max_abs {err:.3e} rms {rms:.3e} max_abs/rms {err / rms:.3e}")
+    assert err <= (2e-2 if bf16 else 1e-4), f"max abs err {err}"
+    if bf16:
+        assert err / rms <= REL_BF16, f"max abs err {err} is {err / rms:.3f} of the output rms {rms}"
 
 
 def _dev(a):
@@ -99,8 +110,7 @@ def test_coarse_ball_attention_matches_oracle(orc, sizes, leaf, m, stride, H, d,
     got = _host(bts.bt_coarse_ball_attention(qd, kd, vd, perm, m, stride))
     assert bts.bt_last_device_status() == 0
     want = orc.coarse_ball_attention(q, k, v, m, perm.cpu().numpy(), stride)
-    err = np.abs(got - want).max()
-    assert err <= (2e-2 if dtype == "bf16" else 1e-4), f"max abs err {err}"
+    _check_attention(got, want, dtype == "bf16")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -127,5 +137,4 @@ def test_gauss_mix_full_size_sampled_coarse_balls(orc):
     want = orc.unpool(oc, p, 4, len(wl.coords))
     slots = np.concatenate([np.arange(b * 512, (b + 1) * 512) for b in balls])
     rows = p[slots][p[slots] >= 0]
-    err = np.abs(got[rows] - want[rows]).max()
-    assert err <= 2e-2, f"max abs err {err}"
+    _check_attention(got[rows], want[rows], True)
