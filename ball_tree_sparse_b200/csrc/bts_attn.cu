@@ -563,6 +563,16 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
             for (int i = 0; i < 4; ++i) crow[i] = lane < 16 ? raw_row(item, 4 * g + i) : -1;
             skip_dead();
         }
+        if (tid == 8 * 32 && ctr) {
+            // this CTA claims no more work: the last CTA to get here sets the launch's counters back to zero for
+            // the next launch that uses them (every CTA's claims come before its count: release and acquire)
+            uint32_t prev;
+            asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ctr + 1) : "memory");
+            if (prev == gridDim.x - 1) {
+                ctr[0] = 0u;
+                ctr[1] = 0u;
+            }
+        }
     } else {
         // ---------------- consumers ----------------
         // Per item: S = Q K^T, softmax (row sums in registers, on the FMA pipe), P V, O read into registers; then this
@@ -727,15 +737,6 @@ __global__ void __launch_bounds__(PairPipe::THREADS, PairPipe::PER_SM)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::COLS) : "memory");
     }
-    if (tid == 0 && ctr) {
-        // the last CTA to finish resets the launch's counters for the next launch that uses them
-        __threadfence();
-        if (atomicAdd(ctr + 1, 1u) == gridDim.x - 1) {
-            ctr[0] = 0u;
-            ctr[1] = 0u;
-            __threadfence();
-        }
-    }
 }
 
 // Tensor maps that view a [rows, H, d] bf16 tensor as rows of H*d elements with a `box`-element window
@@ -784,7 +785,7 @@ static bool tile_map(CUtensorMap *map, const void *base, int64_t rows, int cols,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Work counters of the head-pair kernel ([0] items claimed so far, [1] CTAs finished; the last CTA of a launch
+// Work counters of the head-pair kernel ([0] items claimed so far, [1] CTAs done claiming; the last CTA of a launch
 // sets both back to zero).  Launches that run at the same time need distinct pairs:
 //  - eager launches take pair k mod kEagerPairs (the k-th eager launch on the device), so up to kEagerPairs of
 //    them may be in flight together;
